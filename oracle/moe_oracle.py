@@ -1,0 +1,248 @@
+"""CPU oracle of the single-GPU MoE dispatch-compute-combine layer.
+
+TEST INFRASTRUCTURE ONLY. Only tests/, __graft_entry__.smoke() and bench.py's CPU
+baseline (and its reference arm) may import this module. The product path never does:
+it shares no code, header, table or helper with this file.
+
+It is plain, slow and meant to be checked by eye against the pages it follows:
+
+* "Distributed expert parallelism" (open-llm-engineering), section "The
+  dispatch-compute-combine lifecycle": a token picks k experts, is copied k times,
+  the copies are sorted by expert, experts run grouped FFNs, then the original token
+  order is restored, each result is multiplied by its route weight and the k results
+  of a token are summed.
+* same page, "Token permutation and metadata": expert-contiguous order
+  (expert0 tokens | expert1 tokens | ...) plus the metadata that reverses it
+  (original token index, slot index, per-expert counts).
+* same page, "Duplicate route accumulation": a token's top-k results are added,
+  never overwritten.
+* "Mixture of Kittens" teaching digest, Step 1 (The Math): every routed expert is
+  Down_i(SwiGLU(Up_i x, Gate_i x)); Up and Gate expand d_model to d_expert, Down
+  compresses back.
+* MoonEP README, "Integration" / "Weight buffer": one contiguous weight tensor per
+  projection, experts addressed purely by row index, and a cu_seqlens that selects
+  each expert's rows; dispatch and combine carry bf16 hidden states and fp32 route
+  weights ("API walkthrough").
+* MoonEP README, "Performance": maxvio = max_e(T_e / T_bar) - 1 with T_bar the
+  tokens per expert under perfect balance.
+
+Readings where the pages are silent:
+  SwiGLU(Up x, Gate x) = silu(Gate x) * (Up x), silu(z) = z / (1 + exp(-z));
+  Down is stored [E, H', H] and applied as h @ W_down[e];
+  inside one expert, rows keep flat order f = t*K + k (stable by token, then slot);
+  cu_seqlens has E+1 entries with cu[0] = 0 (MoonEP's end offsets are cu[1:]);
+  no padding rows; stored tensors (x_perm, h, y, out) are bf16 as on the pages,
+  everything between two stores is exact-rounded fp64 and rounded once to bf16
+  (round to nearest, ties to even); T_bar = S*K/E.
+
+Arrays: bf16 tensors are numpy uint16 bit patterns; everything else is int32,
+float32 (route weights) or float64.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+# ----------------------------------------------------------------------------- bf16
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> exact float64 values."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def f64_to_bf16_bits(v: np.ndarray) -> np.ndarray:
+    """Round float64 values once to bf16 (nearest, ties to even) and return the bits.
+
+    bf16 keeps 8 significant bits and fp32's exponent range: a value m * 2^e
+    (0.5 <= |m| < 1) is rounded to a multiple of 2^(e-8), or of 2^-133 in the
+    subnormal range. Overflow gives +-inf.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    _, e = np.frexp(v)
+    q = np.maximum(e.astype(np.int64) - 8, -133)
+    r = np.ldexp(np.rint(np.ldexp(v, -q)), q)  # exact power-of-two scalings; rint ties to even
+    with np.errstate(over="ignore"):
+        f = r.astype(np.float32)  # exact: r is a bf16 value (or overflows to inf)
+    return (f.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def silu(z: np.ndarray) -> np.ndarray:
+    """silu(z) = z * sigmoid(z) = z / (1 + exp(-z)), in float64."""
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+# ----------------------------------------------------------------------------- permute
+
+
+def permute_counting_sort(topk_ids: np.ndarray, E: int):
+    """Expert-contiguous permutation by a counting sort over flat slots f = t*K + k.
+
+    Pure-Python loops: for small cases and as a cross-check of `permute_metadata`.
+    Returns (counts[E], cu_seqlens[E+1], row_id_map[S*K], perm_src[S*K]).
+    """
+    flat = [int(v) for v in np.asarray(topk_ids).reshape(-1)]
+    for e in flat:
+        if not 0 <= e < E:
+            raise ValueError(f"expert id {e} outside [0, {E})")
+    counts = [0] * E
+    for e in flat:  # per-expert token counts
+        counts[e] += 1
+    cu = [0] * (E + 1)
+    for e in range(E):  # exclusive scan
+        cu[e + 1] = cu[e] + counts[e]
+    cursor = list(cu[:E])
+    row_id_map = [0] * len(flat)
+    perm_src = [0] * len(flat)
+    for f, e in enumerate(flat):  # increasing f keeps (token, slot) order inside an expert
+        row_id_map[f] = cursor[e]
+        perm_src[cursor[e]] = f
+        cursor[e] += 1
+    i32 = lambda a: np.asarray(a, dtype=np.int32)
+    return i32(counts), i32(cu), i32(row_id_map), i32(perm_src)
+
+
+def permute_metadata(topk_ids: np.ndarray, E: int):
+    """Same result as `permute_counting_sort`, by a stable sort of slots by expert id.
+
+    Returns (counts[E], cu_seqlens[E+1], row_id_map[S*K], perm_src[S*K]).
+    """
+    flat = np.asarray(topk_ids, dtype=np.int64).reshape(-1)
+    if flat.size and (flat.min() < 0 or flat.max() >= E):
+        raise ValueError("expert id outside [0, E)")
+    counts = np.bincount(flat, minlength=E).astype(np.int64)
+    cu = np.zeros(E + 1, dtype=np.int64)
+    np.cumsum(counts, out=cu[1:])
+    perm_src = np.argsort(flat, kind="stable")  # row -> flat slot
+    row_id_map = np.empty_like(perm_src)
+    row_id_map[perm_src] = np.arange(flat.size)  # flat slot -> row
+    return (counts.astype(np.int32), cu.astype(np.int32), row_id_map.astype(np.int32),
+            perm_src.astype(np.int32))
+
+
+def permute_rows(x_bits: np.ndarray, perm_src: np.ndarray, K: int) -> np.ndarray:
+    """x_perm[row] = x[perm_src[row] // K] (a bit copy of the token's bf16 row)."""
+    return np.asarray(x_bits)[np.asarray(perm_src, dtype=np.int64) // K]
+
+
+def maxvio(counts: np.ndarray, S: int, K: int):
+    """maxvio = max_e(T_e / T_bar) - 1 with T_bar = S*K/E.
+
+    Evaluated as ((double)maxcount * E) / ((double)S * K) - 1: two exact products,
+    one correctly rounded division, one subtraction. Returns (maxvio, max_count).
+    """
+    counts = np.asarray(counts)
+    E = counts.size
+    mc = int(counts.max()) if E else 0
+    num = float(mc) * float(E)
+    den = float(S) * float(K)
+    return (num / den) - 1.0, mc
+
+
+# ----------------------------------------------------------------------------- expert FFN
+
+
+def expert_ffn_rows(x_rows_bits: np.ndarray, w_gate_e: np.ndarray, w_up_e: np.ndarray,
+                    w_down_e: np.ndarray):
+    """One expert on a block of rows: h = bf16(silu(x Wg) * (x Wu)), y = bf16(h Wd).
+
+    x_rows_bits [n,H] bf16 bits; w_gate_e, w_up_e [H,H'] and w_down_e [H',H] as bf16
+    bits. Products accumulate in float64. Returns (h_bits [n,H'], y_bits [n,H]).
+    """
+    x = bf16_bits_to_f64(x_rows_bits)
+    g = x @ bf16_bits_to_f64(w_gate_e)
+    u = x @ bf16_bits_to_f64(w_up_e)
+    h_bits = f64_to_bf16_bits(silu(g) * u)
+    y_bits = f64_to_bf16_bits(bf16_bits_to_f64(h_bits) @ bf16_bits_to_f64(w_down_e))
+    return h_bits, y_bits
+
+
+def grouped_ffn(x_perm_bits: np.ndarray, cu_seqlens: np.ndarray, get_weights, Hp: int):
+    """Grouped expert FFN over expert-contiguous rows.
+
+    Rows [cu[e], cu[e+1]) belong to expert e; get_weights(e) returns
+    (w_gate_e [H,H'], w_up_e [H,H'], w_down_e [H',H]) as bf16 bits. Experts with no
+    rows are skipped. Returns (h_bits [M,H'], y_bits [M,H]).
+    """
+    M, H = x_perm_bits.shape
+    h = np.zeros((M, Hp), dtype=np.uint16)
+    y = np.zeros((M, H), dtype=np.uint16)
+    E = len(cu_seqlens) - 1
+    for e in range(E):
+        r0, r1 = int(cu_seqlens[e]), int(cu_seqlens[e + 1])
+        if r1 == r0:
+            continue
+        h[r0:r1], y[r0:r1] = expert_ffn_rows(x_perm_bits[r0:r1], *get_weights(e))
+    return h, y
+
+
+def expert_of_rows(cu_seqlens: np.ndarray, rows: np.ndarray) -> np.ndarray:
+    """Expert owning each row: the e with cu[e] <= row < cu[e+1]."""
+    return np.searchsorted(np.asarray(cu_seqlens), np.asarray(rows), side="right") - 1
+
+
+# ----------------------------------------------------------------------------- combine
+
+
+def unpermute_combine(y_bits: np.ndarray, row_id_map: np.ndarray, route_w: np.ndarray, S: int,
+                      K: int) -> np.ndarray:
+    """out[t] = bf16(sum over k ascending of w[t,k] * y[row_id_map[t*K+k]]), float64 sum.
+
+    Scatter-add semantics: a token routed twice to the same expert gets both copies.
+    """
+    rmap = np.asarray(row_id_map, dtype=np.int64).reshape(S, K)
+    w = np.asarray(route_w, dtype=np.float32).astype(np.float64).reshape(S, K)
+    H = y_bits.shape[1]
+    acc = np.zeros((S, H), dtype=np.float64)
+    for k in range(K):
+        acc += w[:, k:k + 1] * bf16_bits_to_f64(y_bits[rmap[:, k]])
+    return f64_to_bf16_bits(acc)
+
+
+def combine_token(y_rows_bits: np.ndarray, w_row: np.ndarray) -> np.ndarray:
+    """One token: bf16(sum_k w[k] * y_k) with y_rows_bits [K,H] in slot order."""
+    w = np.asarray(w_row, dtype=np.float32).astype(np.float64)
+    acc = np.zeros(y_rows_bits.shape[1], dtype=np.float64)
+    for k in range(len(w)):
+        acc += w[k] * bf16_bits_to_f64(y_rows_bits[k])
+    return f64_to_bf16_bits(acc)
+
+
+# ----------------------------------------------------------------------------- whole layer
+
+
+def moe_layer(x_bits: np.ndarray, topk_ids: np.ndarray, route_w: np.ndarray, E: int, get_weights,
+              Hp: int, identity_ffn: bool = False):
+    """permute -> grouped FFN (or identity experts) -> weighted combine, plus maxvio.
+
+    Returns a dict with counts, cu_seqlens, row_id_map, perm_src, maxvio, max_count,
+    x_perm, h (None for identity experts), y and out.
+    """
+    S, K = np.asarray(topk_ids).shape
+    counts, cu, rmap, psrc = permute_metadata(topk_ids, E)
+    mv, mc = maxvio(counts, S, K)
+    x_perm = permute_rows(x_bits, psrc, K)
+    if identity_ffn:
+        h, y = None, x_perm
+    else:
+        h, y = grouped_ffn(x_perm, cu, get_weights, Hp)
+    out = unpermute_combine(y, rmap, route_w, S, K)
+    return dict(counts=counts, cu_seqlens=cu, row_id_map=rmap, perm_src=psrc, maxvio=mv,
+                max_count=mc, x_perm=x_perm, h=h, y=y, out=out)
+
+
+def direct_expert_loop(x_bits: np.ndarray, topk_ids: np.ndarray, route_w: np.ndarray, get_weights):
+    """The same layer without any permutation: for every token, run each of its K
+    experts on the token's own row and add the weighted results ("Distributed expert parallelism", Exercises, item 3).
+    Returns out bits [S,H]."""
+    S, K = np.asarray(topk_ids).shape
+    H = x_bits.shape[1]
+    out = np.zeros((S, H), dtype=np.uint16)
+    for t in range(S):
+        ys = np.zeros((K, H), dtype=np.uint16)
+        for k in range(K):
+            e = int(topk_ids[t, k])
+            _, ys[k] = expert_ffn_rows(x_bits[t:t + 1], *get_weights(e))
+        out[t] = combine_token(ys, route_w[t])
+    return out

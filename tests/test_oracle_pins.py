@@ -1,0 +1,307 @@
+"""Pins of the CPU oracle to facts fixed by the pages and by mathematics, not by itself.
+
+Every oracle function is checked here against something independent of its own code:
+the pages' worked example, brute force over all tiny routings, invariants, closed
+forms and library routines (torch CPU) on special cases that reduce to them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bits_of(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def torch_bf16_of(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+
+# ----------------------------------------------------------------------------- worked example
+
+def test_four_rank_worked_example():
+    g = json.load(open(os.path.join(GOLDEN, "four_rank_example.json")))
+    ids = np.array(g["topk_ids"], dtype=np.int32)
+    for fn in (O.permute_counting_sort, O.permute_metadata):
+        counts, cu, rmap, psrc = fn(ids, g["E"])
+        assert counts.tolist() == g["counts"]
+        assert cu.tolist() == g["cu_seqlens"]
+        assert psrc.tolist() == g["perm_src"]
+        assert rmap.tolist() == g["row_id_map"]
+    # rank r owns experts [2r, 2r+2): copies sent to each rank
+    per_rank = [int(counts[2 * r] + counts[2 * r + 1]) for r in range(g["ranks"])]
+    assert per_rank == g["rank_send_splits"]
+    mv, mc = O.maxvio(counts, g["S"], g["K"])
+    assert mc == g["max_count"]
+    assert abs(mv - g["maxvio_num"] / g["maxvio_den"]) <= 4 * np.finfo(float).eps
+
+
+def test_four_rank_example_weighted_reconstruction():
+    """Token A's output is w_A0*Expert1(A) + w_A1*Expert5(A) (the example's last
+    sentence), with hand-computable experts Expert_e(x) = (e+1) * x * x elementwise.
+    """
+    H = 8
+    x = np.full((3, H), 1.0)
+    x[0] *= 2.0  # A
+    x[1] *= 3.0  # B
+    x[2] *= 4.0  # C
+    x_bits = O.f64_to_bf16_bits(x)
+    ids = np.array([[1, 5], [3, 5], [0, 6]], dtype=np.int32)
+    w = np.array([[0.25, 0.75], [0.5, 0.5], [0.125, 0.875]], dtype=np.float32)
+
+    def weights(e):
+        # g = 64 x_j (>= 64, so silu(g) == g after bf16 rounding), u = x_j / 64,
+        # h = g * u = x_j^2, y = (e+1) * h. Every value is an exact small integer.
+        wg = O.f64_to_bf16_bits(64.0 * np.eye(H))
+        wu = O.f64_to_bf16_bits(np.eye(H) / 64.0)
+        wd = O.f64_to_bf16_bits((e + 1.0) * np.eye(H))
+        return wg, wu, wd
+
+    res = O.moe_layer(x_bits, ids, w, 8, weights, H)
+    out = O.bf16_bits_to_f64(res["out"])
+    # A (x=2, h=4):  0.25 * 2*4 + 0.75 * 6*4 = 2 + 18 = 20
+    assert np.all(out[0] == 20.0)
+    # B (x=3, h=9):  0.5 * 4*9 + 0.5 * 6*9 = 18 + 27 = 45
+    assert np.all(out[1] == 45.0)
+    # C (x=4, h=16): 0.125 * 1*16 + 0.875 * 7*16 = 2 + 98 = 100
+    assert np.all(out[2] == 100.0)
+
+
+# ----------------------------------------------------------------------------- brute force
+
+def _all_routings(S, K, E):
+    per_token = list(itertools.product(range(E), repeat=K))
+    for combo in itertools.product(per_token, repeat=S):
+        yield np.array(combo, dtype=np.int32).reshape(S, K)
+
+
+@pytest.mark.parametrize("S,K,E", [(1, 1, 3), (2, 2, 3), (3, 2, 2), (3, 1, 4), (2, 2, 4)])
+def test_permutation_brute_force(S, K, E):
+    """Every routing of tiny shapes (duplicates within a token included)."""
+    for ids in _all_routings(S, K, E):
+        a = O.permute_counting_sort(ids, E)
+        b = O.permute_metadata(ids, E)
+        for u, v in zip(a, b):
+            assert np.array_equal(u, v)
+        counts, cu, rmap, psrc = b
+        flat = ids.reshape(-1).tolist()
+        # counts by direct enumeration
+        assert counts.tolist() == [flat.count(e) for e in range(E)]
+        assert cu[0] == 0 and cu[-1] == S * K
+        assert all(cu[e + 1] - cu[e] == counts[e] for e in range(E))
+        # bijection
+        assert sorted(rmap.tolist()) == list(range(S * K))
+        assert all(psrc[rmap[f]] == f for f in range(S * K))
+        # expert-contiguous and stable: rows of expert e are its flat slots ascending
+        for e in range(E):
+            rows = psrc[cu[e]:cu[e + 1]].tolist()
+            assert rows == [f for f in range(S * K) if flat[f] == e]
+
+
+def test_permute_rows_and_identity_roundtrip():
+    rng = np.random.default_rng(0)
+    S, K, E, H = 5, 3, 4, 16
+    ids = rng.integers(0, E, size=(S, K)).astype(np.int32)
+    x = O.f64_to_bf16_bits(rng.standard_normal((S, H)))
+    counts, cu, rmap, psrc = O.permute_metadata(ids, E)
+    xp = O.permute_rows(x, psrc, K)
+    for t in range(S):
+        for k in range(K):
+            assert np.array_equal(xp[rmap[t * K + k]], x[t])
+    # identity experts, K copies with unit weight: out = bf16(K * x), exact sums
+    out = O.unpermute_combine(xp, rmap, np.ones((S, K), np.float32), S, K)
+    expect = bits_of((torch_bf16_of(x).to(torch.float32) * K).to(torch.bfloat16))
+    assert np.array_equal(out, expect)
+
+
+def test_k1_unit_weight_is_identity():
+    rng = np.random.default_rng(1)
+    S, E, H = 9, 3, 8
+    ids = rng.integers(0, E, size=(S, 1)).astype(np.int32)
+    x = O.f64_to_bf16_bits(rng.standard_normal((S, H)))
+    res = O.moe_layer(x, ids, np.ones((S, 1), np.float32), E, None, 0, identity_ffn=True)
+    assert np.array_equal(res["out"], x)
+
+
+def test_duplicate_route_is_added_not_overwritten():
+    """A token sent twice to the same expert gets both weighted copies."""
+    H = 4
+    x = O.f64_to_bf16_bits(np.array([[1.0, 2.0, 3.0, 4.0]]))
+    ids = np.array([[2, 2]], dtype=np.int32)
+    w = np.array([[0.5, 0.25]], dtype=np.float32)
+    res = O.moe_layer(x, ids, w, 3, None, 0, identity_ffn=True)
+    assert res["counts"].tolist() == [0, 0, 2]
+    np.testing.assert_array_equal(O.bf16_bits_to_f64(res["out"]), 0.75 * np.array([[1, 2, 3, 4.0]]))
+
+
+def test_empty_experts():
+    ids = np.array([[0, 3], [3, 0]], dtype=np.int32)
+    counts, cu, rmap, psrc = O.permute_metadata(ids, 6)
+    assert counts.tolist() == [2, 0, 0, 2, 0, 0]
+    assert cu.tolist() == [0, 2, 2, 2, 4, 4, 4]
+
+
+def test_rejects_bad_routing():
+    with pytest.raises(ValueError):
+        O.permute_metadata(np.array([[0, 5]], np.int32), 5)
+    with pytest.raises(ValueError):
+        O.permute_counting_sort(np.array([[-1, 0]], np.int32), 5)
+
+
+# ----------------------------------------------------------------------------- maxvio
+
+def test_maxvio_closed_forms():
+    S, K, E = 48, 4, 8  # E | S*K
+    f = np.arange(S * K)
+    ids = (f % E).astype(np.int32).reshape(S, K)
+    counts, *_ = O.permute_metadata(ids, E)
+    assert O.maxvio(counts, S, K) == (0.0, S * K // E)
+    # all tokens on one expert with K=1: maxvio = E - 1 exactly
+    ids1 = np.zeros((S, 1), np.int32)
+    counts1, *_ = O.permute_metadata(ids1, E)
+    assert O.maxvio(counts1, S, 1) == (float(E - 1), S)
+    # large-geometry values: hot counts 204, 341, 1877, 3584 of 65536 rows over 384 experts
+    for hot, expect in [(204, 0.1953125), (341, 0.998046875), (1877, 9.998046875), (3584, 20.0)]:
+        c = np.zeros(384, np.int64)
+        c[0] = hot
+        assert O.maxvio(c, 8192, 8)[0] == expect
+
+
+# ----------------------------------------------------------------------------- bf16 rounding
+
+def test_bf16_round_matches_torch_on_float32_values():
+    rng = np.random.default_rng(2)
+    v = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.integers(-30, 30, 20000),
+        rng.standard_normal(2000).astype(np.float32) * np.float32(1e-39),  # subnormals
+    ]).astype(np.float32)
+    ties = (np.arange(1, 2000, dtype=np.uint32) << 16 | 0x8000).view(np.float32)  # exact halves
+    v = np.concatenate([v, ties, -ties, np.float32([0.0, -0.0, 3.3895e38])])
+    ours = O.f64_to_bf16_bits(v.astype(np.float64))
+    ref = bits_of(torch.from_numpy(v).to(torch.bfloat16))
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_bf16_round_single_rounding_from_double():
+    # 1 + 2^-8 + 2^-30 is just above the tie between 1 and 1+2^-7: rounds up. Going
+    # through float32 first would drop the 2^-30 and the tie would round to even (1.0).
+    v = np.array([1.0 + 2.0 ** -8 + 2.0 ** -30, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8])
+    assert O.bf16_bits_to_f64(O.f64_to_bf16_bits(v)).tolist() == [1.0 + 2.0 ** -7, 1.0, 1.0 + 2.0 ** -6]
+    assert O.f64_to_bf16_bits(np.array([1e39]))[0] == 0x7F80  # overflow -> +inf
+
+
+# ----------------------------------------------------------------------------- SiLU / FFN
+
+def test_silu_identities_and_library():
+    z = np.linspace(-40, 40, 2001)
+    s = O.silu(z)
+    np.testing.assert_allclose(s - O.silu(-z), z, rtol=0, atol=1e-12)  # silu(z) - silu(-z) = z
+    assert O.silu(np.array([0.0]))[0] == 0.0
+    ref = torch.nn.functional.silu(torch.from_numpy(z)).numpy()
+    np.testing.assert_allclose(s, ref, rtol=1e-14, atol=1e-300)
+    assert O.silu(np.array([-1000.0]))[0] == 0.0
+
+
+def _weights_getter(wg, wu, wd):
+    return lambda e: (wg[e], wu[e], wd[e])
+
+
+def _rand_layer(rng, S, H, Hp, E, K):
+    x = O.f64_to_bf16_bits(rng.standard_normal((S, H)))
+    wg = O.f64_to_bf16_bits(rng.standard_normal((E, H, Hp)) / math.sqrt(H))
+    wu = O.f64_to_bf16_bits(rng.standard_normal((E, H, Hp)) / math.sqrt(H))
+    wd = O.f64_to_bf16_bits(rng.standard_normal((E, Hp, H)) / math.sqrt(Hp))
+    ids = np.stack([rng.permutation(E)[:K] for _ in range(S)]).astype(np.int32)
+    z = rng.standard_normal((S, K))
+    w = (np.exp(z) / np.exp(z).sum(1, keepdims=True)).astype(np.float32)
+    return x, wg, wu, wd, ids, w
+
+
+def test_dense_special_case_against_torch():
+    """K=1 with every token on expert 0 is a dense SwiGLU FFN: compare with torch CPU
+    (matmul + F.silu in float64, rounded to bf16 by torch at the same points)."""
+    rng = np.random.default_rng(3)
+    S, H, Hp, E = 24, 32, 48, 3
+    x, wg, wu, wd, _, _ = _rand_layer(rng, S, H, Hp, E, 1)
+    ids = np.zeros((S, 1), np.int32)
+    res = O.moe_layer(x, ids, np.ones((S, 1), np.float32), E, _weights_getter(wg, wu, wd), Hp)
+    assert res["maxvio"] == float(E - 1)
+    T = lambda b: torch_bf16_of(b).to(torch.float64)
+    g, u = T(x) @ T(wg[0]), T(x) @ T(wu[0])
+    h = (torch.nn.functional.silu(g) * u).to(torch.float32).to(torch.bfloat16)
+    y = (h.to(torch.float64) @ T(wd[0])).to(torch.float32).to(torch.bfloat16)
+    # torch rounds through float32 (double rounding); allow 1 bf16 ulp where that matters
+    hd = np.abs(O.bf16_bits_to_f64(res["h"]) - h.to(torch.float64).numpy())
+    assert np.all(hd <= 2.0 ** -7 * np.abs(h.to(torch.float64).numpy()) + 1e-30)
+    assert (O.bf16_bits_to_f64(res["h"]) == h.to(torch.float64).numpy()).mean() > 0.999
+    yd = np.abs(O.bf16_bits_to_f64(res["y"]) - y.to(torch.float64).numpy())
+    assert np.all(yd <= 2.0 ** -6 * np.abs(y.to(torch.float64).numpy()) + 1e-6)
+    # unit weight, K=1: out == y
+    assert np.array_equal(res["out"], res["y"])
+
+
+def test_layer_matches_direct_expert_loop():
+    """Permute -> grouped FFN -> combine equals running each token's experts directly
+    ("Distributed expert parallelism", Exercises, item 3)."""
+    rng = np.random.default_rng(4)
+    S, H, Hp, E, K = 13, 16, 24, 5, 2
+    x, wg, wu, wd, ids, w = _rand_layer(rng, S, H, Hp, E, K)
+    get = _weights_getter(wg, wu, wd)
+    res = O.moe_layer(x, ids, w, E, get, Hp)
+    direct = O.direct_expert_loop(x, ids, w, get)
+    a, b = O.bf16_bits_to_f64(res["out"]), O.bf16_bits_to_f64(direct)
+    # the only difference is BLAS summation order inside fp64 dot products
+    assert (a == b).mean() > 0.99
+    np.testing.assert_allclose(a, b, rtol=2 ** -7, atol=1e-6)
+
+
+def test_hand_computable_ffn_values():
+    """H = H' = 8 with a gate so large that silu(g) == g in bf16: the expert is then
+    bilinear and every value below is an exact dyadic rational."""
+    H = 8
+    x = O.f64_to_bf16_bits(np.arange(1, 9, dtype=np.float64)[None, :] / 4.0)  # 0.25..2
+    wg = O.f64_to_bf16_bits(128.0 * np.eye(H))  # g_j = 128 x_j >= 32
+    wu = O.f64_to_bf16_bits(np.diag(np.full(H, 0.5)))  # u_j = x_j / 2
+    wd = O.f64_to_bf16_bits(np.ones((H, H)) / 64.0)  # y_n = sum_j h_j / 64
+    h, y = O.expert_ffn_rows(x, wg, wu, wd)
+    xv = np.arange(1, 9) / 4.0
+    np.testing.assert_array_equal(O.bf16_bits_to_f64(h)[0], 64.0 * xv * xv)  # 128 x * x/2
+    np.testing.assert_array_equal(O.bf16_bits_to_f64(y)[0], np.full(H, (64.0 * xv * xv).sum() / 64.0))
+    # a large negative gate drives h to (almost) zero: silu(-128 x) * u
+    h2, _ = O.expert_ffn_rows(x, O.f64_to_bf16_bits(-128.0 * np.eye(H)), wu, wd)
+    assert np.all(np.abs(O.bf16_bits_to_f64(h2)) < 1e-10)
+
+
+def test_swiglu_roles_gate_vs_up():
+    """silu applies to the Gate branch only: swapping Gate and Up changes the result."""
+    H = 8
+    x = O.f64_to_bf16_bits(np.full((1, H), 1.0))
+    a = O.f64_to_bf16_bits(np.eye(H))  # projection giving 1
+    b = O.f64_to_bf16_bits(-np.eye(H))  # projection giving -1
+    wd = O.f64_to_bf16_bits(np.eye(H))
+    h_ab, _ = O.expert_ffn_rows(x, a, b, wd)  # silu(1) * (-1)
+    h_ba, _ = O.expert_ffn_rows(x, b, a, wd)  # silu(-1) * 1
+    s1 = 1.0 / (1.0 + math.exp(-1.0))
+    assert O.bf16_bits_to_f64(h_ab)[0, 0] == O.bf16_bits_to_f64(O.f64_to_bf16_bits(np.array([-s1])))[0]
+    assert O.bf16_bits_to_f64(h_ba)[0, 0] == O.bf16_bits_to_f64(O.f64_to_bf16_bits(np.array([-(1 - s1)])))[0]
+
+
+def test_mis_addressed_expert_is_visible():
+    """Distinct weights per expert: routing a row to the wrong expert changes y a lot."""
+    rng = np.random.default_rng(5)
+    S, H, Hp, E, K = 8, 16, 16, 4, 1
+    x, wg, wu, wd, ids, w = _rand_layer(rng, S, H, Hp, E, K)
+    get = _weights_getter(wg, wu, wd)
+    good = O.moe_layer(x, ids, w, E, get, Hp)
+    bad = O.moe_layer(x, (ids + 1) % E, w, E, get, Hp)
+    a, b = O.bf16_bits_to_f64(good["out"]), O.bf16_bits_to_f64(bad["out"])
+    assert np.linalg.norm(a - b) > 0.3 * np.linalg.norm(a)
