@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Benchmark of the single-GPU MoE layer: permute -> grouped SwiGLU FFN -> weighted combine.
+
+One step = one pass of the whole hot path over one batch of synthetic tokens that are
+already resident in HBM: moe_permute (histogram, scan, stable rank, row copy; maxvio
+fused), moe_grouped_ffn_up_gate, moe_grouped_ffn_down, moe_unpermute_combine. The L2
+is flushed (a 256 MiB write, outside the timed events) before every timed step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload medium]
+    python bench.py --impl reference ...     (the CPU oracle on the host cores)
+
+Multi-GPU: replicas only (one process per GPU under torchrun, each running the whole
+layer on its own batch; no data-path collective). Time = max over ranks.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/sec on 1 B200; grouped-FFN TFLOP/s; permute+combine HBM GB/s"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "medium"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="CPU work budget for the oracle baseline sample")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- work model
+
+def work_model(w, counts=None):
+    """Algorithmic bytes and flops per stage (real rows only; no padding credited)."""
+    S, H, Hp, E, K = w.S, w.H, w.Hp, w.E, w.K
+    M = S * K
+    active = E if counts is None else int((counts > 0).sum())
+    m = {
+        "permute_bytes": 2 * (S + M) * H + 12 * M + 8 * E,
+        "combine_bytes": 2 * (M + S) * H + 8 * M,
+        "active_experts": active,
+    }
+    if not w.identity_ffn:
+        m["up_gate_flops"] = 4 * M * H * Hp
+        m["up_gate_bytes"] = 2 * 2 * active * H * Hp + 2 * M * H + 2 * M * Hp
+        m["down_flops"] = 2 * M * H * Hp
+        m["down_bytes"] = 2 * active * Hp * H + 2 * M * Hp + 2 * M * H
+    return m
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (every 50 ms) with host timestamps."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_id}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        inside = [p for (t, p) in self.samples if t0 <= t <= t1]
+        window = "timed region"
+        if len(inside) < 3:  # short timed region: use every sample taken under load
+            inside = [p for (t, p) in self.samples]
+            window = "warm-up and timed region"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [v for v in (num(p[0]) for p in inside) if v is not None]
+        mx = [v for v in (num(p[1]) for p in inside) if v is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in inside for i in range(4) if p[4 + i] == "Active"})
+        pw = [v for v in (num(p[2]) for p in inside) if v is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "power_w_max": max(pw) if pw else None, "samples": len(inside),
+                "window": window}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import grouped_ffn_moe_b200 as moe
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload]
+    inp = synth.make_layer_inputs(w, device=str(dev))
+    buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev, with_ffn=not w.identity_ffn)
+    flush = torch.empty(256 << 18, dtype=torch.float32, device=dev)  # 256 MiB > 126 MB L2
+    E = w.E
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        moe.moe_permute(inp["x"], inp["topk_ids"], E, buf.x_perm, buf.counts, buf.cu_seqlens,
+                        buf.row_id_map, buf.perm_src, buf.maxvio, buf.max_count, buf.workspace,
+                        buf.d_status)
+        if ev is not None:
+            ev[1].record()
+        y = buf.x_perm
+        if not w.identity_ffn:
+            moe.moe_grouped_ffn_up_gate(buf.x_perm, inp["w_gate"], inp["w_up"], buf.cu_seqlens,
+                                        buf.h, buf.d_status)
+            if ev is not None:
+                ev[2].record()
+            moe.moe_grouped_ffn_down(buf.h, inp["w_down"], buf.cu_seqlens, buf.y, buf.d_status)
+            y = buf.y
+        elif ev is not None:
+            ev[2].record()
+        if ev is not None:
+            ev[3].record()
+        moe.moe_unpermute_combine(y, buf.row_id_map, inp["route_w"], buf.out)
+        if ev is not None:
+            ev[4].record()
+
+    launches_per_step = moe.LAUNCHES["moe_permute"] + moe.LAUNCHES["moe_unpermute_combine"] + (
+        0 if w.identity_ffn else moe.LAUNCHES["moe_grouped_ffn"])
+
+    gpu_id = str(local)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(gpu_id) if rank == 0 else None
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if int(buf.d_status.item()) != 0:
+        raise RuntimeError(f"device status {int(buf.d_status.item())} during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t1 = time.time()
+
+    per = {k: [] for k in ("permute", "up_gate", "down", "ffn", "combine", "step")}
+    for e in evs:
+        per["permute"].append(e[0].elapsed_time(e[1]))
+        per["up_gate"].append(e[1].elapsed_time(e[2]))
+        per["down"].append(e[2].elapsed_time(e[3]))
+        per["ffn"].append(e[1].elapsed_time(e[3]))
+        per["combine"].append(e[3].elapsed_time(e[4]))
+        per["step"].append(e[0].elapsed_time(e[4]))
+    mean = {k: sum(v) / len(v) for k, v in per.items()}
+    ms_step = mean["step"]
+    if world > 1:
+        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    status = int(buf.d_status.item())
+    counts = buf.counts.cpu().numpy()
+    maxvio = float(buf.maxvio.item())
+
+    # e2e: host (pinned) inputs -> device -> layer -> host output, every step
+    e2e = None
+    if not args.no_e2e:
+        hx = inp["x"].cpu().pin_memory()
+        hids = inp["topk_ids"].cpu().pin_memory()
+        hw = inp["route_w"].cpu().pin_memory()
+        hout = torch.empty(w.S, w.H, dtype=torch.bfloat16).pin_memory()
+        dx, dids, dw = torch.empty_like(inp["x"]), torch.empty_like(inp["topk_ids"]), \
+            torch.empty_like(inp["route_w"])
+
+        def e2e_step():
+            dx.copy_(hx, non_blocking=True)
+            dids.copy_(hids, non_blocking=True)
+            dw.copy_(hw, non_blocking=True)
+            out = moe.moe_layer_forward(dx, dids, dw, inp.get("w_gate"), inp.get("w_up"),
+                                        inp.get("w_down"), buf)
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        e_ms = []
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            e2e_step()
+            b.record()
+            e_ms.append((a, b))
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in e_ms) / len(e_ms)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * w.S / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": hx.numel() * 2 + hids.numel() * 4 + hw.numel() * 4,
+               "d2h_bytes_per_step": hout.numel() * 2, "ms_per_step": e2e_ms}
+        if not torch.equal(hout.to(dev), buf.out):
+            raise RuntimeError("e2e output differs from the device-resident run")
+
+    if clocks is not None:
+        clocks.stop()
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        wm = work_model(w, counts)
+        stages = {
+            "permute": {"ms": mean["permute"],
+                        "GB/s": wm["permute_bytes"] / (mean["permute"] / 1e3) / 1e9},
+            "combine": {"ms": mean["combine"],
+                        "GB/s": wm["combine_bytes"] / (mean["combine"] / 1e3) / 1e9},
+        }
+        if not w.identity_ffn:
+            stages["up_gate"] = {"ms": mean["up_gate"],
+                                 "TFLOP/s": wm["up_gate_flops"] / (mean["up_gate"] / 1e3) / 1e12}
+            stages["down"] = {"ms": mean["down"],
+                              "TFLOP/s": wm["down_flops"] / (mean["down"] / 1e3) / 1e12}
+            stages["grouped_ffn"] = {
+                "ms": mean["ffn"],
+                "TFLOP/s": (wm["up_gate_flops"] + wm["down_flops"]) / (mean["ffn"] / 1e3) / 1e12}
+            # dominant kernel: the SwiGLU (up/gate) pass
+            flops, byts, t_s = wm["up_gate_flops"], wm["up_gate_bytes"], mean["up_gate"] / 1e3
+            ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+            if flops / byts >= ridge:
+                roof = {"kernel": "grouped_ffn_kernel<true> (up/gate + SwiGLU)", "bound": "tensor",
+                        "achieved": flops / t_s / 1e12, "peak": peaks["bf16_tflops"],
+                        "unit": "TFLOP/s"}
+            else:
+                roof = {"kernel": "grouped_ffn_kernel<true> (up/gate + SwiGLU)", "bound": "hbm",
+                        "achieved": byts / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        else:
+            byts, t_s = wm["permute_bytes"], mean["permute"] / 1e3
+            roof = {"kernel": "moe_permute (4 kernels)", "bound": "hbm", "achieved": byts / t_s / 1e9,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["peak_source"] = f"{peak_src} (burst)"
+        roof["traffic"] = None
+        line = {
+            "metric": METRIC, "value": world * w.S / (ms_step / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded SplitMix64/Box-Muller inputs, random-init expert weights)",
+            "config": {"workload": w.name, "S": w.S, "H": w.H, "Hp": w.Hp, "E": w.E, "K": w.K,
+                       "routing": w.routing, "maxvio_measured": maxvio,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed before every step (256 MiB write outside the timed events)"},
+            "stages": stages, "roofline": roof, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "device_status": status,
+            "clocks": clocks.summary(t0, t1) if clocks else None,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_sample(w, S_sample, host):
+    """Oracle layer on the first S_sample tokens of the workload. host: dict of numpy bits."""
+    from oracle import moe_oracle as O
+
+    ids = host["topk_ids"][:S_sample]
+    return O.moe_layer(host["x"][:S_sample], ids, host["route_w"][:S_sample], w.E, host["get"],
+                       w.Hp, identity_ffn=w.identity_ffn)
+
+
+def _host_inputs_from_device(w, inp):
+    import numpy as np
+    import torch
+
+    def bits(t):
+        return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+    host = {"x": bits(inp["x"]), "topk_ids": inp["topk_ids"].cpu().numpy(),
+            "route_w": inp["route_w"].cpu().numpy()}
+    if not w.identity_ffn:
+        wg, wu, wd = bits(inp["w_gate"]), bits(inp["w_up"]), bits(inp["w_down"])
+        host["get"] = lambda e: (wg[e], wu[e], wd[e])
+    else:
+        host["get"] = None
+    return host
+
+
+def _sample_tokens(w):
+    return {"tiny": 256, "medium": 128}.get(w.name, 16 if not w.identity_ffn else 1024)
+
+
+def cpu_baseline(w, inp, budget_s):
+    host = _host_inputs_from_device(w, inp)
+    S_sample = min(w.S, _sample_tokens(w))
+    done, t_start = 0, time.perf_counter()
+    while True:
+        _oracle_sample(w, S_sample, host)
+        done += S_sample
+        el = time.perf_counter() - t_start
+        if el >= budget_s:
+            break
+    return {"value": done / el, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "sample": f"first {S_sample} tokens of workload {w.name} (full weights), "
+                      f"repeated for {el:.1f} s; numpy fp64"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import synth
+
+    w = synth.WORKLOADS[args.workload]
+    inp = synth.make_layer_inputs(w, device="cpu")
+    host = _host_inputs_from_device(w, inp)
+    S_sample = min(w.S, _sample_tokens(w))
+    for _ in range(args.warmup):
+        _oracle_sample(w, S_sample, host)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        _oracle_sample(w, S_sample, host)
+        times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = S_sample / sec
+    sample = (f"first {S_sample} of {w.S} tokens of workload {w.name} per step (full weights); "
+              f"numpy fp64 oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "S": w.S, "H": w.H, "Hp": w.Hp,
+                                        "E": w.E, "K": w.K, "routing": w.routing},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

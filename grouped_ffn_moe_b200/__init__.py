@@ -1,0 +1,294 @@
+"""Python binding of libmoe_b200.so (include/moe_b200.h): the single-GPU MoE hot path.
+
+Argument marshalling only. Every step runs in the CUDA kernels of libmoe_b200.so;
+PyTorch provides device memory and the current stream. There is no CPU fallback: if
+the library is missing, every call raises.
+
+Functions carry the C ABI's names:
+    moe_permute, moe_grouped_ffn (= moe_grouped_ffn_up_gate + moe_grouped_ffn_down),
+    moe_unpermute_combine, moe_maxvio, moe_permute_workspace_bytes, moe_status_string
+plus `LayerBuffers` / `moe_layer_forward`, which allocate the layer's buffers once and
+chain the three calls (permute -> grouped FFN -> combine) on one stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARGUMENT = 1
+MOE_ERR_UNSUPPORTED_SHAPE = 2
+MOE_ERR_CUDA = 3
+MOE_ERR_BAD_ROUTING = 4
+MOE_ERR_DEVICE_TIMEOUT = 8
+MOE_MAX_EXPERTS = 1024
+
+# Kernels launched by one call of each entry point (permute with a row copy).
+LAUNCHES = {"moe_permute": 4, "moe_grouped_ffn": 2, "moe_grouped_ffn_up_gate": 1,
+            "moe_grouped_ffn_down": 1, "moe_unpermute_combine": 1, "moe_maxvio": 1}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {moe_status_string(status)} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run grouped_ffn_moe_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        i32, i64, p, sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_status_string.argtypes = [i32]
+        L.moe_abi_version.restype = i32
+        L.moe_abi_version.argtypes = []
+        L.moe_permute_workspace_bytes.restype = sz
+        L.moe_permute_workspace_bytes.argtypes = [i64, i32, i32]
+        L.moe_permute.restype = i32
+        L.moe_permute.argtypes = [p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p, sz, p, p]
+        L.moe_grouped_ffn.restype = i32
+        L.moe_grouped_ffn.argtypes = [p, p, p, p, p, i64, i64, i64, i32, p, p, p, p]
+        L.moe_grouped_ffn_up_gate.restype = i32
+        L.moe_grouped_ffn_up_gate.argtypes = [p, p, p, p, i64, i64, i64, i32, p, p, p]
+        L.moe_grouped_ffn_down.restype = i32
+        L.moe_grouped_ffn_down.argtypes = [p, p, p, i64, i64, i64, i32, p, p, p]
+        L.moe_unpermute_combine.restype = i32
+        L.moe_unpermute_combine.argtypes = [p, p, p, i64, i64, i32, p, p]
+        L.moe_maxvio.restype = i32
+        L.moe_maxvio.argtypes = [p, i32, i64, i32, p, p, p]
+        _lib = L
+    return _lib
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device=None):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != MOE_OK:
+        raise MoeError(fn, status)
+
+
+def _need(t, name, dtype, device=None, ndim=None):
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim} dims, got {t.dim()}")
+
+
+def moe_permute_workspace_bytes(S: int, K: int, E: int) -> int:
+    return int(lib().moe_permute_workspace_bytes(S, K, E))
+
+
+def moe_permute(x, topk_ids, E, x_perm, counts, cu_seqlens, row_id_map, perm_src=None, maxvio=None,
+                max_count=None, workspace=None, d_status=None, stream=None):
+    """Route top-k copies into expert-contiguous order (see include/moe_b200.h)."""
+    S, K = topk_ids.shape
+    dev = topk_ids.device
+    _need(topk_ids, "topk_ids", torch.int32, dev, 2)
+    _need(x, "x", torch.bfloat16, dev, 2)
+    _need(x_perm, "x_perm", torch.bfloat16, dev, 2)
+    for t, n in ((counts, "counts"), (cu_seqlens, "cu_seqlens"), (row_id_map, "row_id_map"),
+                 (perm_src, "perm_src"), (max_count, "max_count"), (d_status, "d_status")):
+        _need(t, n, torch.int32, dev)
+    _need(maxvio, "maxvio", torch.float64, dev)
+    H = x.shape[1] if x is not None else 0
+    if x_perm is not None and tuple(x_perm.shape) != (S * K, H):
+        raise ValueError(f"x_perm: expected {(S * K, H)}, got {tuple(x_perm.shape)}")
+    if counts.numel() != E or cu_seqlens.numel() != E + 1 or row_id_map.numel() != S * K:
+        raise ValueError("counts/cu_seqlens/row_id_map sizes do not match (S, K, E)")
+    if perm_src is not None and perm_src.numel() != S * K:
+        raise ValueError("perm_src: expected S*K entries")
+    need = moe_permute_workspace_bytes(S, K, E)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().moe_permute(_ptr(x), _ptr(topk_ids), S, H, K, E, _ptr(x_perm), _ptr(counts),
+                           _ptr(cu_seqlens), _ptr(row_id_map), _ptr(perm_src), _ptr(maxvio),
+                           _ptr(max_count), _ptr(workspace), wbytes, _ptr(d_status),
+                           _stream(stream, dev))
+    _check("moe_permute", st)
+
+
+def moe_grouped_ffn(x_perm, w_gate, w_up, w_down, cu_seqlens, h_scratch, y, d_status=None,
+                    stream=None):
+    """Grouped SwiGLU expert FFN over expert-contiguous rows (see include/moe_b200.h)."""
+    M, H = x_perm.shape
+    E, H2, Hp = w_gate.shape
+    dev = x_perm.device
+    for t, n in ((x_perm, "x_perm"), (h_scratch, "h_scratch"), (y, "y")):
+        _need(t, n, torch.bfloat16, dev, 2)
+    for t, n in ((w_gate, "w_gate"), (w_up, "w_up"), (w_down, "w_down")):
+        _need(t, n, torch.bfloat16, dev, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(d_status, "d_status", torch.int32, dev)
+    if H2 != H or tuple(w_up.shape) != (E, H, Hp) or tuple(w_down.shape) != (E, Hp, H):
+        raise ValueError("weight shapes must be w_gate/w_up [E,H,H'] and w_down [E,H',H]")
+    if tuple(h_scratch.shape) != (M, Hp) or tuple(y.shape) != (M, H):
+        raise ValueError("h_scratch must be [M,H'] and y [M,H]")
+    if cu_seqlens.numel() != E + 1:
+        raise ValueError("cu_seqlens must have E+1 entries")
+    st = lib().moe_grouped_ffn(_ptr(x_perm), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                               _ptr(cu_seqlens), M, H, Hp, E, _ptr(h_scratch), _ptr(y),
+                               _ptr(d_status), _stream(stream, dev))
+    _check("moe_grouped_ffn", st)
+
+
+def _ffn_check(x_perm, w_gate, w_up, w_down, cu_seqlens, h_scratch, y, d_status):
+    M, H = x_perm.shape
+    Hp = h_scratch.shape[1]
+    E = cu_seqlens.numel() - 1
+    dev = x_perm.device
+    for t, n in ((x_perm, "x_perm"), (h_scratch, "h_scratch"), (y, "y")):
+        _need(t, n, torch.bfloat16, dev, 2)
+    for t, n in ((w_gate, "w_gate"), (w_up, "w_up"), (w_down, "w_down")):
+        _need(t, n, torch.bfloat16, dev, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(d_status, "d_status", torch.int32, dev)
+    if w_gate is not None and tuple(w_gate.shape) != (E, H, Hp):
+        raise ValueError(f"w_gate must be [E,H,H'] = {(E, H, Hp)}")
+    if w_up is not None and tuple(w_up.shape) != (E, H, Hp):
+        raise ValueError(f"w_up must be [E,H,H'] = {(E, H, Hp)}")
+    if w_down is not None and tuple(w_down.shape) != (E, Hp, H):
+        raise ValueError(f"w_down must be [E,H',H] = {(E, Hp, H)}")
+    if h_scratch.shape[0] != M or (y is not None and tuple(y.shape) != (M, H)):
+        raise ValueError("h_scratch must be [M,H'] and y [M,H]")
+    return M, H, Hp, E, dev
+
+
+def moe_grouped_ffn_up_gate(x_perm, w_gate, w_up, cu_seqlens, h_scratch, d_status=None,
+                            stream=None):
+    """First pass of moe_grouped_ffn: h = bf16(silu(x_perm W_gate[e]) * (x_perm W_up[e]))."""
+    M, H, Hp, E, dev = _ffn_check(x_perm, w_gate, w_up, None, cu_seqlens, h_scratch, None, d_status)
+    st = lib().moe_grouped_ffn_up_gate(_ptr(x_perm), _ptr(w_gate), _ptr(w_up), _ptr(cu_seqlens), M,
+                                       H, Hp, E, _ptr(h_scratch), _ptr(d_status),
+                                       _stream(stream, dev))
+    _check("moe_grouped_ffn_up_gate", st)
+
+
+def moe_grouped_ffn_down(h_scratch, w_down, cu_seqlens, y, d_status=None, stream=None):
+    """Second pass of moe_grouped_ffn: y = bf16(h W_down[e])."""
+    M, H = y.shape
+    Hp = h_scratch.shape[1]
+    E = cu_seqlens.numel() - 1
+    dev = y.device
+    _need(h_scratch, "h_scratch", torch.bfloat16, dev, 2)
+    _need(y, "y", torch.bfloat16, dev, 2)
+    _need(w_down, "w_down", torch.bfloat16, dev, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(d_status, "d_status", torch.int32, dev)
+    if tuple(w_down.shape) != (E, Hp, H) or h_scratch.shape[0] != M:
+        raise ValueError("w_down must be [E,H',H] and h_scratch [M,H']")
+    st = lib().moe_grouped_ffn_down(_ptr(h_scratch), _ptr(w_down), _ptr(cu_seqlens), M, H, Hp, E,
+                                    _ptr(y), _ptr(d_status), _stream(stream, dev))
+    _check("moe_grouped_ffn_down", st)
+
+
+def moe_unpermute_combine(y, row_id_map, route_w, out, stream=None):
+    """out[t] = sum_k route_w[t,k] * y[row_id_map[t*K+k]] (see include/moe_b200.h)."""
+    S, K = route_w.shape
+    dev = y.device
+    _need(y, "y", torch.bfloat16, dev, 2)
+    _need(out, "out", torch.bfloat16, dev, 2)
+    _need(row_id_map, "row_id_map", torch.int32, dev)
+    _need(route_w, "route_w", torch.float32, dev, 2)
+    H = y.shape[1]
+    if tuple(out.shape) != (S, H) or row_id_map.numel() != S * K:
+        raise ValueError("out must be [S,H] and row_id_map S*K entries")
+    st = lib().moe_unpermute_combine(_ptr(y), _ptr(row_id_map), _ptr(route_w), S, H, K, _ptr(out),
+                                     _stream(stream, dev))
+    _check("moe_unpermute_combine", st)
+
+
+def moe_maxvio(counts, S, K, maxvio, max_count=None, stream=None):
+    """maxvio = max_e(counts[e] * E / (S*K)) - 1 into a device double (see include/moe_b200.h)."""
+    dev = counts.device
+    _need(counts, "counts", torch.int32, dev)
+    _need(maxvio, "maxvio", torch.float64, dev)
+    _need(max_count, "max_count", torch.int32, dev)
+    st = lib().moe_maxvio(_ptr(counts), counts.numel(), S, K, _ptr(maxvio), _ptr(max_count),
+                          _stream(stream, dev))
+    _check("moe_maxvio", st)
+
+
+@dataclass
+class LayerBuffers:
+    """Device buffers of one layer call, allocated once and reused (static shapes)."""
+
+    x_perm: torch.Tensor
+    counts: torch.Tensor
+    cu_seqlens: torch.Tensor
+    row_id_map: torch.Tensor
+    perm_src: torch.Tensor
+    maxvio: torch.Tensor
+    max_count: torch.Tensor
+    workspace: torch.Tensor
+    h: torch.Tensor | None
+    y: torch.Tensor | None
+    out: torch.Tensor
+    d_status: torch.Tensor
+
+    @staticmethod
+    def allocate(S: int, H: int, Hp: int, E: int, K: int, device, with_ffn: bool = True):
+        M = S * K
+        i32 = dict(dtype=torch.int32, device=device)
+        bf = dict(dtype=torch.bfloat16, device=device)
+        return LayerBuffers(
+            x_perm=torch.empty(M, H, **bf), counts=torch.empty(E, **i32),
+            cu_seqlens=torch.empty(E + 1, **i32), row_id_map=torch.empty(M, **i32),
+            perm_src=torch.empty(M, **i32),
+            maxvio=torch.empty(1, dtype=torch.float64, device=device),
+            max_count=torch.empty(1, **i32),
+            workspace=torch.empty(max(moe_permute_workspace_bytes(S, K, E), 16), dtype=torch.uint8,
+                                  device=device),
+            h=torch.empty(M, Hp, **bf) if with_ffn else None,
+            y=torch.empty(M, H, **bf) if with_ffn else None,
+            out=torch.empty(S, H, **bf), d_status=torch.zeros(1, **i32))
+
+
+def moe_layer_forward(x, topk_ids, route_w, w_gate, w_up, w_down, buf: LayerBuffers, stream=None):
+    """permute -> grouped FFN -> combine on one stream; returns buf.out.
+
+    With w_gate None the experts are the identity (y = x_perm): permute/combine only.
+    """
+    E = buf.counts.numel()
+    moe_permute(x, topk_ids, E, buf.x_perm, buf.counts, buf.cu_seqlens, buf.row_id_map,
+                buf.perm_src, buf.maxvio, buf.max_count, buf.workspace, buf.d_status, stream)
+    y = buf.x_perm
+    if w_gate is not None:
+        moe_grouped_ffn(buf.x_perm, w_gate, w_up, w_down, buf.cu_seqlens, buf.h, buf.y,
+                        buf.d_status, stream)
+        y = buf.y
+    moe_unpermute_combine(y, buf.row_id_map, route_w, buf.out, stream)
+    return buf.out

@@ -1,0 +1,182 @@
+// C ABI entry points (include/moe_b200.h): argument validation, workspace sizing, launch.
+// Nothing here allocates device memory or synchronises the host.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+
+#include "internal.h"
+
+namespace moe {
+
+int num_sms() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < 64) {
+    const int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+namespace {
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr int64_t kMaxRows = (int64_t{1} << 31) - 1;
+
+}  // namespace
+}  // namespace moe
+
+using moe::aligned;
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_BAD_ROUTING: return "expert id outside [0, E)";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_BAD_ROUTING | MOE_ERR_DEVICE_TIMEOUT:
+      return "expert id outside [0, E); device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int32_t moe_abi_version(void) { return (1 << 16) | 0; }
+
+size_t moe_permute_workspace_bytes(int64_t S, int32_t K, int32_t E) {
+  if (S <= 0 || K <= 0 || E <= 0) return 0;
+  const int64_t nchunk = moe::permute_num_chunks(S * K);
+  const size_t bytes = sizeof(int32_t) * static_cast<size_t>(nchunk) * static_cast<size_t>(E);
+  return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+moe_status moe_permute(const void* x, const int32_t* topk_ids, int64_t S, int64_t H, int32_t K,
+                       int32_t E, void* x_perm, int32_t* counts, int32_t* cu_seqlens,
+                       int32_t* row_id_map, int32_t* perm_src, double* maxvio, int32_t* max_count,
+                       void* workspace, size_t workspace_bytes, int32_t* d_status,
+                       void* cuda_stream) {
+  if (S < 0 || K < 1 || E < 1 || K > E) return MOE_ERR_INVALID_ARGUMENT;
+  if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (S * K > moe::kMaxRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!counts || !cu_seqlens) return MOE_ERR_INVALID_ARGUMENT;
+  if (S > 0 && (!row_id_map || !topk_ids)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned(counts, 4) || !aligned(cu_seqlens, 4) || !aligned(row_id_map, 4) ||
+      !aligned(topk_ids, 4) || !aligned(perm_src, 4) || !aligned(max_count, 4) ||
+      !aligned(maxvio, 8) || !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (x_perm != nullptr) {
+    if ((S > 0 && x == nullptr) || H <= 0) return MOE_ERR_INVALID_ARGUMENT;
+    if (H % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(x, 16) || !aligned(x_perm, 16)) return MOE_ERR_INVALID_ARGUMENT;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  if (S == 0) {
+    // Nothing routed: zero counts and offsets; maxvio is undefined (T_bar = 0) -> NaN.
+    if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, stream) != cudaSuccess ||
+        cudaMemsetAsync(cu_seqlens, 0, sizeof(int32_t) * (E + 1), stream) != cudaSuccess ||
+        (max_count && cudaMemsetAsync(max_count, 0, sizeof(int32_t), stream) != cudaSuccess) ||
+        (maxvio && cudaMemsetAsync(maxvio, 0xFF, sizeof(double), stream) != cudaSuccess))
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  const size_t need = moe_permute_workspace_bytes(S, K, E);
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16))
+    return MOE_ERR_INVALID_ARGUMENT;
+  return moe::launch_permute(x, topk_ids, S, H, K, E, x_perm, counts, cu_seqlens, row_id_map,
+                             perm_src, maxvio, max_count, static_cast<int32_t*>(workspace),
+                             d_status, stream);
+}
+
+namespace {
+
+moe_status check_ffn_shapes(int64_t M, int64_t H, int64_t Hp, int32_t E) {
+  if (M < 0 || H <= 0 || Hp <= 0 || E < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (E > MOE_MAX_EXPERTS || M > moe::kMaxRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (H % 128 != 0 || Hp % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<int64_t>(E) * H > moe::kMaxRows || static_cast<int64_t>(E) * Hp > moe::kMaxRows)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+bool ok_ptr16(const void* p) { return p != nullptr && aligned(p, 16); }
+
+}  // namespace
+
+moe_status moe_grouped_ffn_up_gate(const void* x_perm, const void* w_gate, const void* w_up,
+                                   const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp,
+                                   int32_t E, void* h_scratch, int32_t* d_status,
+                                   void* cuda_stream) {
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  if (!ok_ptr16(x_perm) || !ok_ptr16(w_gate) || !ok_ptr16(w_up) || !ok_ptr16(h_scratch) ||
+      cu_seqlens == nullptr || !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M == 0) return MOE_OK;
+  return moe::launch_ffn_pass(true, x_perm, w_gate, w_up, cu_seqlens, M, H, Hp, E, h_scratch,
+                              d_status, static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_grouped_ffn_down(const void* h_scratch, const void* w_down,
+                                const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp,
+                                int32_t E, void* y, int32_t* d_status, void* cuda_stream) {
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  if (!ok_ptr16(h_scratch) || !ok_ptr16(w_down) || !ok_ptr16(y) || cu_seqlens == nullptr ||
+      !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M == 0) return MOE_OK;
+  return moe::launch_ffn_pass(false, h_scratch, w_down, nullptr, cu_seqlens, M, H, Hp, E, y,
+                              d_status, static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_grouped_ffn(const void* x_perm, const void* w_gate, const void* w_up,
+                           const void* w_down, const int32_t* cu_seqlens, int64_t M, int64_t H,
+                           int64_t Hp, int32_t E, void* h_scratch, void* y, int32_t* d_status,
+                           void* cuda_stream) {
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  // validate both passes before launching either
+  if (!ok_ptr16(x_perm) || !ok_ptr16(w_gate) || !ok_ptr16(w_up) || !ok_ptr16(w_down) ||
+      !ok_ptr16(h_scratch) || !ok_ptr16(y) || cu_seqlens == nullptr || !aligned(cu_seqlens, 4) ||
+      !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M == 0) return MOE_OK;
+  const moe_status s1 = moe_grouped_ffn_up_gate(x_perm, w_gate, w_up, cu_seqlens, M, H, Hp, E,
+                                                h_scratch, d_status, cuda_stream);
+  if (s1 != MOE_OK) return s1;
+  return moe_grouped_ffn_down(h_scratch, w_down, cu_seqlens, M, H, Hp, E, y, d_status,
+                              cuda_stream);
+}
+
+moe_status moe_unpermute_combine(const void* y, const int32_t* row_id_map, const float* route_w,
+                                 int64_t S, int64_t H, int32_t K, void* out, void* cuda_stream) {
+  if (S < 0 || H <= 0 || K < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (H % 8 != 0 || S * K > moe::kMaxRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (S == 0) return MOE_OK;
+  if (!y || !row_id_map || !route_w || !out) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned(y, 16) || !aligned(out, 16) || !aligned(row_id_map, 4) || !aligned(route_w, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  return moe::launch_combine(y, row_id_map, route_w, S, H, K, out,
+                             static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_maxvio(const int32_t* counts, int32_t E, int64_t S, int32_t K, double* maxvio,
+                      int32_t* max_count, void* cuda_stream) {
+  if (E < 1 || S < 1 || K < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (!counts || !maxvio || !aligned(counts, 4) || !aligned(maxvio, 8) || !aligned(max_count, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  return moe::launch_maxvio(counts, E, S, K, maxvio, max_count,
+                            static_cast<cudaStream_t>(cuda_stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+// Unpermute-combine: restore token order, scale by route weight, sum the K results.
+//
+// "Distributed expert parallelism" (open-llm-engineering), lifecycle step 8 (restore the
+// original token indexes, multiply by route weights, sum the k results per token) and
+// "Duplicate route accumulation" (add, never assign). MoonEP README, "combine fwd": bf16
+// expert outputs in, bf16 token-major output, fp32 route weights.
+//
+//   out[t] = bf16( sum_{k ascending} w[t,k] * float(y[row_id_map[t*K+k]]) )
+//
+// One warp per token. Each lane owns U 16-byte vectors (8 bf16) per pass and keeps their
+// fp32 sums in registers; the K source rows of a pass are loaded four slots at a time so
+// that several loads are in flight before the fixed-order FMAs consume them.
+#include <algorithm>
+#include <cuda_bf16.h>
+
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ void fma_bf16x8(float (&acc)[8], const uint4& v, float w) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] = fmaf(w, __uint_as_float(u[i] << 16), acc[2 * i]);
+    acc[2 * i + 1] = fmaf(w, __uint_as_float(u[i] & 0xFFFF0000u), acc[2 * i + 1]);
+  }
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float (&acc)[8]) {
+  uint32_t u[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i]));
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i + 1]));
+    u[i] = lo | (hi << 16);
+  }
+  return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+template <int U>
+__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y,
+                                                      const int32_t* __restrict__ row_id_map,
+                                                      const float* __restrict__ route_w, int64_t S,
+                                                      int64_t nvec, int32_t K,
+                                                      uint4* __restrict__ out) {
+  constexpr int kSlots = 4;  // slots loaded together
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       t < S; t += nwarps) {
+    const int32_t my_row = (lane < K) ? row_id_map[t * K + lane] : -1;
+    const float my_w = (lane < K) ? route_w[t * K + lane] : 0.0f;
+    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
+      float acc[U][8];
+#pragma unroll
+      for (int j = 0; j < U; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[j][i] = 0.0f;
+      for (int k0 = 0; k0 < K; k0 += kSlots) {
+        uint4 r[kSlots][U];
+        int32_t rows[kSlots];
+        float ws[kSlots];
+#pragma unroll
+        for (int s = 0; s < kSlots; ++s) {
+          const int k = k0 + s;
+          if (K <= 32) {
+            rows[s] = __shfl_sync(kFull, my_row, k & 31);
+            ws[s] = __shfl_sync(kFull, my_w, k & 31);
+          } else {
+            rows[s] = (k < K) ? row_id_map[t * K + k] : -1;
+            ws[s] = (k < K) ? route_w[t * K + k] : 0.0f;
+          }
+          if (k >= K) rows[s] = -1;
+#pragma unroll
+          for (int j = 0; j < U; ++j) {
+            const int64_t v = v0 + j * 32 + lane;
+            r[s][j] = (rows[s] >= 0 && v < nvec)
+                          ? __ldg(y + static_cast<int64_t>(rows[s]) * nvec + v)
+                          : make_uint4(0, 0, 0, 0);
+          }
+        }
+#pragma unroll
+        for (int s = 0; s < kSlots; ++s) {
+          if (rows[s] < 0) continue;
+#pragma unroll
+          for (int j = 0; j < U; ++j) fma_bf16x8(acc[j], r[s][j], ws[s]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const int64_t v = v0 + j * 32 + lane;
+        if (v < nvec) out[t * nvec + v] = pack_bf16x8(acc[j]);
+      }
+    }
+  }
+}
+
+}  // namespace
+
+moe_status launch_combine(const void* y, const int32_t* row_id_map, const float* route_w,
+                          int64_t S, int64_t H, int32_t K, void* out, cudaStream_t stream) {
+  const int64_t nvec = H / 8;
+  const int64_t blocks = std::min<int64_t>(ceil_div(S, 8), static_cast<int64_t>(num_sms()) * 8);
+  combine_kernel<2><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      static_cast<const uint4*>(y), row_id_map, route_w, S, nvec, K, static_cast<uint4*>(out));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

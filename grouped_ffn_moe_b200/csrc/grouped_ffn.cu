@@ -1,0 +1,467 @@
+// Grouped expert SwiGLU FFN on 5th-generation tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+//
+// Computes, for every expert e and every row r of e's contiguous block
+// [cu_seqlens[e], cu_seqlens[e+1]) ("Mixture of Kittens" digest, Step 1; MoonEP README,
+// "Integration" and "Weight buffer": experts addressed by row index of one contiguous
+// [E, H, H'] tensor per projection, cu_seqlens selects the rows):
+//
+//   pass 1 (kDual):  h[r] = bf16( silu(x[r] . W_gate[e]) * (x[r] . W_up[e]) )
+//   pass 2:          y[r] = bf16( h[r] . W_down[e] )
+//
+// Design ("swap AB"): the tensor-core M side (128) runs over output features and the N side
+// over an expert's tokens, D^T[f, tok] = sum_k W[e][k, f] * X[tok, k]. Expert sizes are
+// ragged and often small (171 rows on average at S=8192, K=8, E=384); with tokens on N the
+// MMA shape follows the expert exactly up to the next multiple of 16 (N = 16..256), where
+// tokens on M would pad every expert to multiples of 128. The weight tile (A) is
+// MN-major (features contiguous, as stored), the token tile (B) K-major; both are loaded
+// by TMA with 128-byte swizzle, which is the canonical UMMA shared-memory layout.
+//
+// Work unit = (expert, 128-feature block, chunk of <= 256 of the expert's tokens). Units are
+// enumerated expert-major, then feature block, then chunk, and a persistent grid of one CTA
+// per SM strides over them: CTAs that run at the same time share the expert's token rows
+// (and, for an expert split into chunks, its weight tile) through L2, so each weight byte
+// crosses HBM about once, and a hot expert's chunks spread over all SMs.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads into a kStages-deep shared-memory ring;
+// warp 1 owns TMEM (alloc/dealloc) and issues the MMAs from one thread; warps 2-5 drain the
+// fp32 accumulators with tcgen05.ld, apply SiLU*up (pass 1) and rounding, transpose through
+// shared memory and store whole 16-byte vectors of the expert's rows only.
+// Every wait is bounded (globaltimer); on expiry the CTA records MOE_ERR_DEVICE_TIMEOUT,
+// drains its own copies and MMAs with bounded waits, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdlib>
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;                       // output features per unit (UMMA M)
+constexpr int kBK = 64;                        // reduction elements per stage (128 bytes)
+constexpr int kNMax = 256;                     // tokens per unit (UMMA N max)
+constexpr int kRowsPerBox = 16;                // token rows per TMA box
+constexpr int kABytes = kBM * kBK * 2;         // 16 KB: two [64 k][64 f] boxes
+constexpr int kABoxBytes = 64 * kBK * 2;       // 8 KB
+constexpr int kBBytes = kNMax * kBK * 2;       // 32 KB
+constexpr int kBBoxBytes = kRowsPerBox * kBK * 2;  // 2 KB
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kOutChunk = 32;                  // tokens per epilogue chunk
+constexpr int kOutBytes = kOutChunk * kBM * 2;  // 8 KB staging buffer
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCols = 256;
+
+template <bool kDual>
+struct Cfg {
+  static constexpr int kNumA = kDual ? 2 : 1;
+  static constexpr int kStages = kDual ? 3 : 4;
+  static constexpr int kAccStages = kDual ? 1 : 2;
+  static constexpr int kStageBytes = kNumA * kABytes + kBBytes;
+  static constexpr int kPipeBytes = kStages * kStageBytes;
+  static constexpr int kOffOut = kPipeBytes;
+  static constexpr int kOffCu = kOffOut + 2 * kOutBytes;
+  static constexpr int kOffUnits = kOffCu + 4 * (MOE_MAX_EXPERTS + 1);
+  static constexpr int kOffBars = (kOffUnits + 4 * (MOE_MAX_EXPERTS + 1) + 7) & ~7;
+  static constexpr int kNumBars = 2 * kStages + 2 * 2 + 1;
+  static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
+  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+};
+static_assert(Cfg<true>::kSmemBytes <= 232448, "shared memory budget (dual)");
+static_assert(Cfg<false>::kSmemBytes <= 232448, "shared memory budget (single)");
+
+struct FfnArgs {
+  const int32_t* cu;     // [E+1]
+  __nv_bfloat16* out;    // [M, n_feat]
+  int32_t* d_status;
+  int64_t M;
+  int32_t E;
+  int32_t k_dim;         // reduction length: H (pass 1) or H' (pass 2)
+  int32_t n_feat;        // output features: H' (pass 1) or H (pass 2)
+  uint64_t budget_ns;
+};
+
+struct Unit {
+  int e, fb, row0, nrows;
+};
+
+// Unit u -> (expert, feature block, token rows). s_ustart[e] is the first unit of expert e.
+__device__ __forceinline__ Unit decode_unit(int u, const int32_t* s_ustart, const int32_t* s_cu,
+                                            int E) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_ustart[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  Unit U;
+  U.e = lo;
+  const int local = u - s_ustart[lo];
+  const int cnt = s_cu[lo + 1] - s_cu[lo];
+  const int ntc = (cnt + kNMax - 1) / kNMax;
+  U.fb = local / ntc;
+  const int tc = local - U.fb * ntc;
+  const int cs = (((cnt + ntc - 1) / ntc) + 15) & ~15;  // balanced chunks, multiple of 16
+  const int r0 = tc * cs;
+  U.row0 = s_cu[lo] + r0;
+  U.nrows = min(cnt - r0, cs);
+  return U;
+}
+
+__device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
+  const uint32_t a = smem_u32(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+template <bool kDual>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_ffn_kernel(const __grid_constant__ CUtensorMap tmA0,
+                       const __grid_constant__ CUtensorMap tmA1,
+                       const __grid_constant__ CUtensorMap tmB, const FfnArgs args) {
+  using C = Cfg<kDual>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  uint8_t* s_out = smem + C::kOffOut;
+  int32_t* s_cu = reinterpret_cast<int32_t*>(smem + C::kOffCu);
+  int32_t* s_ustart = reinterpret_cast<int32_t*>(smem + C::kOffUnits);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::kStages;
+  uint64_t* tfull = bars + 2 * C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  int32_t* s_scan = reinterpret_cast<int32_t*>(smem + C::kOffMisc + 8);  // [8]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int E = args.E;
+  const int nfb = args.n_feat / kBM;
+  const int KT = args.k_dim / kBK;
+
+  // ------------------------------------------------------------------ prologue
+  if (tid == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&tfull[s], 1);
+      mbar_init(&tempty[s], kEpiThreads / 32);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmA0);
+    if (kDual) tma_prefetch_map(&tmA1);
+    tma_prefetch_map(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  // cu_seqlens, clamped to [0, M] so that no row outside [0, M) is ever addressed
+  for (int e = tid; e <= E; e += kThreads) {
+    int64_t v = args.cu[e];
+    v = v < 0 ? 0 : (v > args.M ? args.M : v);
+    s_cu[e] = static_cast<int32_t>(v);
+  }
+  __syncthreads();
+  // units per expert, then an exclusive scan into s_ustart[0..E]
+  {
+    const int per = (E + kThreads - 1) / kThreads;  // <= 6 for E <= 1024
+    const int beg = min(tid * per, E), end = min(beg + per, E);
+    int local = 0;
+    for (int e = beg; e < end; ++e) {
+      const int cnt = s_cu[e + 1] - s_cu[e];
+      const int units = cnt > 0 ? ((cnt + kNMax - 1) / kNMax) * nfb : 0;
+      s_ustart[e] = units;
+      local += units;
+    }
+    int incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += n;
+    }
+    if (lane == 31) s_scan[warp] = incl;
+    __syncthreads();
+    int off = 0;
+    for (int w = 0; w < warp; ++w) off += s_scan[w];
+    int run = off + incl - local;
+    for (int e = beg; e < end; ++e) {
+      const int units = s_ustart[e];
+      s_ustart[e] = run;
+      run += units;
+    }
+    if (tid == kThreads - 1) s_ustart[E] = off + incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int total_units = s_ustart[E];
+
+  // ------------------------------------------------------------------ roles
+  if (warp == 0) {
+    // TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();  // weights: streamed once
+      const uint64_t pol_x = policy_evict_last();   // token rows: reused by all feature blocks
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      for (int u = blockIdx.x; u < total_units && !*s_abort; u += gridDim.x) {
+        const Unit U = decode_unit(u, s_ustart, s_cu, E);
+        if (U.nrows <= 0) continue;
+        const int nbox = (U.nrows + kRowsPerBox - 1) / kRowsPerBox;
+        const uint32_t bytes = C::kNumA * kABytes + nbox * kBBoxBytes;
+        const int fx = U.fb * kBM;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, s_abort, args.budget_ns)) break;
+          uint8_t* st = smem + stage * C::kStageBytes;
+          const int ky = U.e * args.k_dim + kt * kBK;
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_2d_hint(st, &tmA0, &full[stage], fx, ky, pol_w);
+          tma_load_2d_hint(st + kABoxBytes, &tmA0, &full[stage], fx + 64, ky, pol_w);
+          if (kDual) {
+            tma_load_2d_hint(st + kABytes, &tmA1, &full[stage], fx, ky, pol_w);
+            tma_load_2d_hint(st + kABytes + kABoxBytes, &tmA1, &full[stage], fx + 64, ky, pol_w);
+          }
+          uint8_t* sb = st + C::kNumA * kABytes;
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d_hint(sb + b * kBBoxBytes, &tmB, &full[stage], kt * kBK,
+                             U.row0 + b * kRowsPerBox, pol_x);
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*s_abort) {
+        // let this CTA's own copies land before the CTA exits (bounded)
+        volatile int dummy = 0;
+        for (int s = 0; s < C::kStages; ++s)
+          if (issued_mask & (1u << s))
+            mbar_wait_bounded(&full[s], (issued_phase >> s) & 1u, &dummy, args.budget_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int astage = 0;
+      uint32_t aphase = 0;
+      bool issued_any = false;
+      for (int u = blockIdx.x; u < total_units && !*s_abort; u += gridDim.x) {
+        const Unit U = decode_unit(u, s_ustart, s_cu, E);
+        if (U.nrows <= 0) continue;
+        const uint32_t n = static_cast<uint32_t>((U.nrows + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_m128_amn_bk(n);
+        if (!mbar_wait_bounded(&tempty[astage], aphase ^ 1u, s_abort, args.budget_ns)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + (kDual ? 0u : astage * kAccCols);
+        const uint32_t d1 = tmem_base + kAccCols;
+        bool ok = true;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait_bounded(&full[stage], phase, s_abort, args.budget_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t a1 = a0 + kABytes;
+          const uint32_t b0 = a0 + C::kNumA * kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t bdesc = smem_desc_sw128(b0 + kk * 32, 16, 1024);
+            const uint32_t acc = (kt | kk) != 0 ? 1u : 0u;
+            umma_f16(d0, smem_desc_sw128(a0 + kk * 2048, kABoxBytes, 1024), bdesc, idesc, acc);
+            if (kDual)
+              umma_f16(d1, smem_desc_sw128(a1 + kk * 2048, kABoxBytes, 1024), bdesc, idesc, acc);
+          }
+          issued_any = true;
+          umma_commit(&empty[stage]);  // frees the smem stage when these MMAs complete
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[astage]);  // accumulator ready for the epilogue
+        if (++astage == C::kAccStages) {
+          astage = 0;
+          aphase ^= 1u;
+        }
+      }
+      if (*s_abort && issued_any) {
+        umma_commit(drain);
+        volatile int dummy = 0;
+        mbar_wait_bounded(drain, 0, &dummy, args.budget_ns);
+      }
+    }
+  } else {
+    // Epilogue: warps 2..5; warp w reads TMEM lanes 32*(w%4) .. +31 (its feature rows)
+    const int q = warp & 3;
+    const int f_local = q * 32 + lane;
+    const int et = tid - 64;  // 0..127
+    int astage = 0;
+    uint32_t aphase = 0;
+    uint32_t chunk_ctr = 0;
+    for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+      const Unit U = decode_unit(u, s_ustart, s_cu, E);
+      if (U.nrows <= 0) continue;
+      mbar_wait_bounded(&tfull[astage], aphase, s_abort, args.budget_ns);
+      named_bar_sync(1, kEpiThreads);  // all four warps take the same abort decision
+      if (*s_abort) break;
+      tc_fence_after();
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (kDual ? 0u : astage * kAccCols);
+      for (int c = 0; c < U.nrows; c += kOutChunk) {
+        __syncwarp();  // tcgen05.ld is .sync.aligned: whole warp, converged
+        uint32_t r0[32];
+        tmem_ld_32x32b_x32(tbase + c, r0);
+        __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(s_out + (chunk_ctr & 1u) * kOutBytes);
+        if (kDual) {
+          uint32_t r1[32];
+          tmem_ld_32x32b_x32(tbase + kAccCols + c, r1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float g = __uint_as_float(r0[j]);
+            const float v = __uint_as_float(r1[j]);
+            const float hval = (g / (1.0f + expf(-g))) * v;
+            so[j * kBM + f_local] = __float2bfloat16_rn(hval);
+          }
+        } else {
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) so[j * kBM + f_local] = __float2bfloat16_rn(__uint_as_float(r0[j]));
+        }
+        named_bar_sync(1, kEpiThreads);
+        const uint8_t* sob = reinterpret_cast<const uint8_t*>(so);
+#pragma unroll
+        for (int p = 0; p < (kOutChunk * kBM * 2 / 16) / kEpiThreads; ++p) {
+          const int vid = et + kEpiThreads * p;
+          const int j = vid >> 4, c16 = vid & 15;
+          if (c + j < U.nrows) {
+            const uint4 val = *reinterpret_cast<const uint4*>(sob + j * (kBM * 2) + c16 * 16);
+            __nv_bfloat16* dst = args.out + static_cast<int64_t>(U.row0 + c + j) * args.n_feat +
+                                 U.fb * kBM + c16 * 8;
+            *reinterpret_cast<uint4*>(dst) = val;
+          }
+        }
+        ++chunk_ctr;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[astage]);
+      if (++astage == C::kAccStages) {
+        astage = 0;
+        aphase ^= 1u;
+      }
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  __syncthreads();
+  if (tid == 0 && *s_abort && args.d_status != nullptr) atomicOr(args.d_status, MOE_ERR_DEVICE_TIMEOUT);
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [outer, inner] with a (box_inner x box_outer) box, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+              uint32_t box_outer) {
+  auto enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+uint64_t wait_budget_ns() {
+  static uint64_t budget = [] {
+    const char* s = std::getenv("MOE_WAIT_BUDGET_NS");
+    if (s != nullptr && *s) return static_cast<uint64_t>(std::strtoull(s, nullptr, 10));
+    return static_cast<uint64_t>(2000000000ull);  // 2 s
+  }();
+  return budget;
+}
+
+template <bool kDual>
+bool ensure_smem_attr() {
+  static std::atomic<int> done_dev_mask{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const int bit = 1 << (dev & 31);
+  if (done_dev_mask.load() & bit) return true;
+  if (cudaFuncSetAttribute(grouped_ffn_kernel<kDual>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Cfg<kDual>::kSmemBytes) != cudaSuccess)
+    return false;
+  done_dev_mask.fetch_or(bit);
+  return true;
+}
+
+}  // namespace
+
+moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const void* w1,
+                           const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp, int32_t E,
+                           void* out, int32_t* d_status, cudaStream_t stream) {
+  const int grid = num_sms();
+  if (dual) {
+    CUtensorMap m_wg, m_wu, m_x;
+    if (!make_map(&m_wg, w0, Hp, static_cast<uint64_t>(E) * H, 64, 64) ||
+        !make_map(&m_wu, w1, Hp, static_cast<uint64_t>(E) * H, 64, 64) ||
+        !make_map(&m_x, act, H, M, 64, kRowsPerBox) || !ensure_smem_attr<true>())
+      return MOE_ERR_CUDA;
+    const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
+                    static_cast<int32_t>(H), static_cast<int32_t>(Hp), wait_budget_ns()};
+    grouped_ffn_kernel<true><<<grid, kThreads, Cfg<true>::kSmemBytes, stream>>>(m_wg, m_wu, m_x, a);
+  } else {
+    CUtensorMap m_wd, m_h;
+    if (!make_map(&m_wd, w0, H, static_cast<uint64_t>(E) * Hp, 64, 64) ||
+        !make_map(&m_h, act, Hp, M, 64, kRowsPerBox) || !ensure_smem_attr<false>())
+      return MOE_ERR_CUDA;
+    const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
+                    static_cast<int32_t>(Hp), static_cast<int32_t>(H), wait_budget_ns()};
+    grouped_ffn_kernel<false><<<grid, kThreads, Cfg<false>::kSmemBytes, stream>>>(m_wd, m_wd, m_h,
+                                                                                  a);
+  }
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

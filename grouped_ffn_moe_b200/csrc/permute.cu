@@ -1,0 +1,274 @@
+// Route permutation into expert-contiguous order, and the row copy that goes with it.
+//
+// Follows "Distributed expert parallelism" (open-llm-engineering): "The
+// dispatch-compute-combine lifecycle" steps 2-3 (copy every token k times, sort the copies
+// by expert) and "Token permutation and metadata" (expert-contiguous rows plus the map that
+// reverses them). The order inside an expert is the flat slot order f = t*K + k, which
+// makes the permutation a stable counting sort and the output independent of scheduling.
+//
+// Four launches, no host synchronisation, no atomics on data:
+//   route_hist  per 512-slot chunk (one warp), per-expert counts via __match_any_sync
+//   route_scan  per expert (one warp), exclusive scan over chunks -> chunk bases + counts
+//   route_rank  exclusive scan of counts -> cu_seqlens (+ max count, maxvio); every warp
+//               replays its chunk with per-expert cursors -> row_id_map, perm_src
+//   permute_rows one warp per token: read the row once (16-byte vectors), write K copies
+#include <algorithm>
+
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ void flag_status(int32_t* d_status, int32_t bit) {
+  if (d_status != nullptr) atomicOr(d_status, bit);
+}
+
+// chunk_counts[e * nchunk + c] = #{f in chunk c : ids[f] == e}. Warp w of block b owns
+// chunk b*8 + w. Ids outside [0, E) are not counted and set MOE_ERR_BAD_ROUTING.
+__global__ void __launch_bounds__(256) route_hist_kernel(const int32_t* __restrict__ ids,
+                                                         int64_t F, int32_t E, int64_t nchunk,
+                                                         int32_t* __restrict__ chunk_counts,
+                                                         int32_t* d_status) {
+  extern __shared__ int32_t s_hist[];  // [8][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kWarpsPerTile * E; i += blockDim.x) s_hist[i] = 0;
+  __syncthreads();
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * kWarpsPerTile + warp;
+  int32_t* hist = s_hist + warp * E;
+  if (c < nchunk) {
+    bool bad = false;
+    for (int step = 0; step < kChunk / 32; ++step) {
+      const int64_t f0 = c * kChunk + step * 32;
+      if (f0 >= F) break;  // warp-uniform
+      const int64_t f = f0 + lane;
+      const int32_t e = (f < F) ? ids[f] : -1;
+      const bool ok = (f < F) && e >= 0 && e < E;
+      bad |= (f < F) && !ok;
+      const unsigned peers = __match_any_sync(kFull, ok ? e : -1);
+      if (ok && lane == __ffs(peers) - 1) hist[e] += __popc(peers);
+      __syncwarp();
+    }
+    if (__any_sync(kFull, bad) && lane == 0) flag_status(d_status, MOE_ERR_BAD_ROUTING);
+  }
+  __syncthreads();
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kWarpsPerTile;
+  for (int j = threadIdx.x; j < kWarpsPerTile * E; j += blockDim.x) {
+    const int e = j / kWarpsPerTile, w = j % kWarpsPerTile;
+    if (c0 + w < nchunk) chunk_counts[static_cast<int64_t>(e) * nchunk + c0 + w] = s_hist[w * E + e];
+  }
+}
+
+// In place: chunk_counts[e][c] -> sum_{c' < c} chunk_counts[e][c']; counts[e] = total.
+__global__ void __launch_bounds__(256) route_scan_kernel(int32_t* __restrict__ chunk_counts,
+                                                         int64_t nchunk, int32_t E,
+                                                         int32_t* __restrict__ counts) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 8 + warp;
+  if (e >= E) return;
+  int32_t* row = chunk_counts + static_cast<int64_t>(e) * nchunk;
+  int32_t carry = 0;
+  for (int64_t base = 0; base < nchunk; base += 32) {
+    const int64_t i = base + lane;
+    const int32_t v = (i < nchunk) ? row[i] : 0;
+    int32_t incl = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t n = __shfl_up_sync(kFull, incl, d);
+      if (lane >= d) incl += n;
+    }
+    if (i < nchunk) row[i] = carry + incl - v;
+    carry += __shfl_sync(kFull, incl, 31);
+  }
+  if (lane == 0) counts[e] = carry;
+}
+
+// maxvio = ((double)mc * E) / ((double)S * K) - 1, every operation rounded once (no FMA).
+__device__ __forceinline__ double maxvio_expr(int32_t mc, int32_t E, int64_t S, int32_t K) {
+  const double num = __dmul_rn(static_cast<double>(mc), static_cast<double>(E));
+  const double den = __dmul_rn(static_cast<double>(S), static_cast<double>(K));
+  return __dsub_rn(__ddiv_rn(num, den), 1.0);
+}
+
+// Exclusive scan of counts (E <= 1024, 4 per thread) into s_cu[0..E]; returns the max count
+// in *s_max. Whole block (256 threads).
+__device__ void block_scan_counts(const int32_t* __restrict__ counts, int32_t E, int32_t* s_cu,
+                                  int32_t* s_tmp /*[16]*/, int32_t* s_max) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int32_t v[4];
+  int32_t local = 0, lmax = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = tid * 4 + j;
+    v[j] = (e < E) ? counts[e] : 0;
+    local += v[j];
+    lmax = max(lmax, v[j]);
+  }
+  int32_t incl = local;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int32_t n = __shfl_up_sync(kFull, incl, d);
+    if (lane >= d) incl += n;
+  }
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) lmax = max(lmax, __shfl_xor_sync(kFull, lmax, d));
+  if (lane == 31) s_tmp[warp] = incl;
+  if (lane == 0) s_tmp[8 + warp] = lmax;
+  __syncthreads();
+  int32_t woff = 0;
+  for (int w = 0; w < warp; ++w) woff += s_tmp[w];
+  int32_t run = woff + incl - local;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = tid * 4 + j;
+    if (e < E) s_cu[e] = run;
+    run += v[j];
+  }
+  if (tid == blockDim.x - 1) s_cu[E] = woff + incl;
+  if (tid == 0) {
+    int32_t m = 0;
+    for (int w = 0; w < 8; ++w) m = max(m, s_tmp[8 + w]);
+    *s_max = m;
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(256) route_rank_kernel(
+    const int32_t* __restrict__ ids, int64_t F, int64_t S, int32_t K, int32_t E, int64_t nchunk,
+    const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ counts,
+    int32_t* __restrict__ cu_seqlens, int32_t* __restrict__ row_id_map,
+    int32_t* __restrict__ perm_src, double* maxvio, int32_t* max_count) {
+  extern __shared__ int32_t smem[];
+  int32_t* s_cu = smem;                 // [E+1]
+  int32_t* s_cursor = smem + (E + 1);   // [8][E]
+  __shared__ int32_t s_tmp[16];
+  __shared__ int32_t s_max;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  block_scan_counts(counts, E, s_cu, s_tmp, &s_max);
+  if (blockIdx.x == 0) {
+    for (int e = tid; e <= E; e += blockDim.x) cu_seqlens[e] = s_cu[e];
+    if (tid == 0) {
+      if (max_count != nullptr) *max_count = s_max;
+      if (maxvio != nullptr) *maxvio = maxvio_expr(s_max, E, S, K);
+    }
+  }
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kWarpsPerTile;
+  for (int j = tid; j < kWarpsPerTile * E; j += blockDim.x) {
+    const int e = j / kWarpsPerTile, w = j % kWarpsPerTile;
+    if (c0 + w < nchunk)
+      s_cursor[w * E + e] = s_cu[e] + chunk_base[static_cast<int64_t>(e) * nchunk + c0 + w];
+  }
+  __syncthreads();
+
+  const int64_t c = c0 + warp;
+  if (c >= nchunk) return;
+  int32_t* cur = s_cursor + warp * E;
+  for (int step = 0; step < kChunk / 32; ++step) {
+    const int64_t f0 = c * kChunk + step * 32;
+    if (f0 >= F) break;  // warp-uniform
+    const int64_t f = f0 + lane;
+    const int32_t e = (f < F) ? ids[f] : -1;
+    const bool ok = (f < F) && e >= 0 && e < E;
+    const unsigned peers = __match_any_sync(kFull, ok ? e : -1);
+    int32_t row = -1;
+    if (ok) row = cur[e] + __popc(peers & ((1u << lane) - 1u));
+    __syncwarp();
+    if (ok && lane == __ffs(peers) - 1) cur[e] += __popc(peers);
+    __syncwarp();
+    if (f < F) {
+      row_id_map[f] = row;
+      if (perm_src != nullptr && ok) perm_src[row] = static_cast<int32_t>(f);
+    }
+  }
+}
+
+// One warp per token: the token's row is read once (U 16-byte vectors per lane per pass)
+// and written to its K destination rows.
+template <int U>
+__global__ void __launch_bounds__(256) permute_rows_kernel(const uint4* __restrict__ x, int64_t S,
+                                                           int64_t nvec, int32_t K,
+                                                           const int32_t* __restrict__ row_id_map,
+                                                           uint4* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       t < S; t += nwarps) {
+    const int32_t my_row = (lane < K) ? row_id_map[t * K + lane] : -1;
+    const uint4* src = x + t * nvec;
+    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
+      uint4 r[U];
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const int64_t v = v0 + j * 32 + lane;
+        if (v < nvec) r[j] = __ldg(src + v);
+      }
+      for (int k = 0; k < K; ++k) {
+        const int32_t row = (K <= 32) ? __shfl_sync(kFull, my_row, k) : row_id_map[t * K + k];
+        if (row < 0) continue;
+        uint4* dst = x_perm + static_cast<int64_t>(row) * nvec;
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+          const int64_t v = v0 + j * 32 + lane;
+          if (v < nvec) dst[v] = r[j];
+        }
+      }
+    }
+  }
+}
+
+__global__ void maxvio_kernel(const int32_t* __restrict__ counts, int32_t E, int64_t S, int32_t K,
+                              double* maxvio, int32_t* max_count) {
+  __shared__ int32_t s_w[32];
+  int32_t m = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) m = max(m, counts[e]);
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) m = max(m, __shfl_xor_sync(kFull, m, d));
+  if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t mc = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) mc = max(mc, s_w[w]);
+    if (max_count != nullptr) *max_count = mc;
+    *maxvio = maxvio_expr(mc, E, S, K);
+  }
+}
+
+}  // namespace
+
+moe_status launch_permute(const void* x, const int32_t* topk_ids, int64_t S, int64_t H, int32_t K,
+                          int32_t E, void* x_perm, int32_t* counts, int32_t* cu_seqlens,
+                          int32_t* row_id_map, int32_t* perm_src, double* maxvio,
+                          int32_t* max_count, int32_t* chunk_counts, int32_t* d_status,
+                          cudaStream_t stream) {
+  const int64_t F = S * K;
+  const int64_t nchunk = permute_num_chunks(F);
+  const int64_t tiles = ceil_div(nchunk, kWarpsPerTile);
+  const size_t hist_smem = sizeof(int32_t) * kWarpsPerTile * E;
+  const size_t rank_smem = sizeof(int32_t) * (E + 1 + kWarpsPerTile * E);
+  // E <= 1024: at most 32 KB (hist) and 37 KB (rank), under the 48 KB default limit.
+
+  route_hist_kernel<<<static_cast<unsigned>(tiles), 256, hist_smem, stream>>>(
+      topk_ids, F, E, nchunk, chunk_counts, d_status);
+  route_scan_kernel<<<static_cast<unsigned>(ceil_div(E, 8)), 256, 0, stream>>>(chunk_counts,
+                                                                             nchunk, E, counts);
+  route_rank_kernel<<<static_cast<unsigned>(tiles), 256, rank_smem, stream>>>(
+      topk_ids, F, S, K, E, nchunk, chunk_counts, counts, cu_seqlens, row_id_map, perm_src,
+      maxvio, max_count);
+  if (x_perm != nullptr) {
+    const int64_t nvec = H / 8;
+    const int64_t blocks = std::min<int64_t>(ceil_div(S, 8), static_cast<int64_t>(num_sms()) * 8);
+    permute_rows_kernel<4><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const uint4*>(x), S, nvec, K, row_id_map, static_cast<uint4*>(x_perm));
+  }
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status launch_maxvio(const int32_t* counts, int32_t E, int64_t S, int32_t K, double* maxvio,
+                         int32_t* max_count, cudaStream_t stream) {
+  maxvio_kernel<<<1, 256, 0, stream>>>(counts, E, S, K, maxvio, max_count);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

@@ -1,0 +1,174 @@
+/*
+ * moe_b200.h - C ABI of the single-GPU MoE dispatch-compute-combine hot path on B200.
+ *
+ * The layer (one GPU, no inter-GPU exchange):
+ *
+ *   moe_permute            route top-k copies into expert-contiguous order
+ *   moe_grouped_ffn        y = Down_e(SwiGLU(Up_e x, Gate_e x)) for every expert's rows
+ *   moe_unpermute_combine  out[t] = sum_k w[t,k] * y[row of (t,k)]
+ *   moe_maxvio             max_e(T_e / T_bar) - 1
+ *
+ * Sources (page title, section):
+ *   "Distributed expert parallelism" (open-llm-engineering): "The dispatch-compute-combine
+ *     lifecycle" (copy each token k times, sort copies by expert, grouped expert FFNs,
+ *     restore token order, scale by route weight, sum the k results); "Token permutation
+ *     and metadata" (expert-contiguous order plus the metadata that reverses it);
+ *     "Failure modes ..." (empty experts, scatter-add rather than assign).
+ *   "Mixture of Kittens" teaching digest, Step 1, The Math: Expert_i(x) =
+ *     Down_i(SwiGLU(Up_i(x), Gate_i(x))).
+ *   MoonEP README: "Integration" and "Weight buffer" (one contiguous weight tensor per
+ *     projection, experts addressed by row index, cu_seqlens selects each expert's rows);
+ *     "API walkthrough" (bf16 hidden states, fp32 route weights, int32 expert ids and
+ *     counts); "Performance" (the maxvio formula).
+ *
+ * Conventions shared by every call:
+ *   - All tensors are dense, row-major, caller-allocated device memory. The library never
+ *     allocates, frees or keeps pointers across calls. bf16 tensors are passed as void*.
+ *   - S tokens, K experts per token (slots), E experts, H hidden size, Hp = H' (expert
+ *     intermediate size), M = S*K routed rows. Flat slot f = t*K + k.
+ *   - Every call is asynchronous on `cuda_stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronises the host. The returned status covers argument checks
+ *     and launch errors only; on any error nothing has been launched. Errors that depend
+ *     on device data are OR-ed into *d_status (a device int32 the caller zeroes and reads
+ *     when it chooses; may be NULL to skip reporting).
+ *   - Preconditions, checked on the host: pointers non-NULL and 16-byte aligned (unless
+ *     documented nullable), H and Hp multiples of 8 (of 128 for moe_grouped_ffn),
+ *     1 <= K <= E <= MOE_MAX_EXPERTS, S*K < 2^31. S = 0 is a legal no-op.
+ *   - Results are deterministic: no floating-point atomics; every sum has a fixed order.
+ */
+#ifndef MOE_B200_H_
+#define MOE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t moe_status;
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARGUMENT 1  /* null/misaligned pointer, negative size, K > E ... */
+#define MOE_ERR_UNSUPPORTED_SHAPE 2 /* legal but outside what the kernels handle       */
+#define MOE_ERR_CUDA 3              /* a CUDA runtime/driver call failed                 */
+#define MOE_ERR_BAD_ROUTING 4       /* device: an expert id outside [0, E)               */
+#define MOE_ERR_DEVICE_TIMEOUT 8    /* device: a bounded wait in a kernel ran out        */
+
+/* Largest E the kernels accept (per-expert tables live in shared memory). */
+#define MOE_MAX_EXPERTS 1024
+
+/* Static description of a status code. Never NULL. */
+const char* moe_status_string(moe_status s);
+
+/* Version of this ABI, (major << 16) | minor. */
+int32_t moe_abi_version(void);
+
+/*
+ * Bytes of device workspace moe_permute needs for (S, K, E): per-expert counts of every
+ * 512-slot chunk of the flat routing table, rounded up to 256 bytes. 0 when S == 0.
+ */
+size_t moe_permute_workspace_bytes(int64_t S, int32_t K, int32_t E);
+
+/*
+ * moe_permute - top-k route permutation into expert-contiguous order ("Distributed expert
+ * parallelism", "Token permutation and metadata"; MoonEP README, "dispatch fwd").
+ *
+ *   x          [S, H] bf16 token states. May be NULL together with x_perm, or when S == 0
+ *              (then topk_ids, row_id_map and perm_src may be NULL too).
+ *   topk_ids   [S, K] int32 expert of every slot; K distinct ids per token are not required
+ *              (a repeated id gives two rows that the combine adds).
+ *   x_perm     [S*K, H] bf16 out: row row_id_map[f] = x[f / K]. NULL: metadata only.
+ *   counts     [E] int32 out: rows per expert.
+ *   cu_seqlens [E+1] int32 out: cu[0] = 0, cu[e+1] = cu[e] + counts[e], cu[E] = S*K. Expert e
+ *              owns rows [cu[e], cu[e+1]). (MoonEP's end-offset array is cu_seqlens + 1.)
+ *   row_id_map [S*K] int32 out: flat slot -> row. Inside one expert rows follow increasing
+ *              f, i.e. (token, slot) order; the permutation is a bijection of [0, S*K).
+ *   perm_src   [S*K] int32 out, nullable: row -> flat slot (inverse of row_id_map).
+ *   maxvio     device double out, nullable: as moe_maxvio on the counts.
+ *   max_count  device int32 out, nullable: max_e counts[e].
+ *   workspace  device scratch of moe_permute_workspace_bytes(S, K, E) bytes (contents
+ *              ignored on entry, undefined on exit).
+ *   d_status   nullable device int32: MOE_ERR_BAD_ROUTING is OR-ed in if any id is outside
+ *              [0, E); such slots are dropped (row_id_map[f] = -1) and counts no longer sum
+ *              to S*K.
+ */
+moe_status moe_permute(const void* x, const int32_t* topk_ids, int64_t S, int64_t H, int32_t K,
+                       int32_t E, void* x_perm, int32_t* counts, int32_t* cu_seqlens,
+                       int32_t* row_id_map, int32_t* perm_src, double* maxvio, int32_t* max_count,
+                       void* workspace, size_t workspace_bytes, int32_t* d_status,
+                       void* cuda_stream);
+
+/*
+ * moe_grouped_ffn - grouped expert SwiGLU FFN over expert-contiguous rows ("Mixture of
+ * Kittens" digest, Step 1; MoonEP README, "Integration" and "Weight buffer"; "Distributed
+ * expert parallelism", "Grouped expert computation").
+ *
+ * For every expert e and row r in [cu_seqlens[e], cu_seqlens[e+1]):
+ *   g = x_perm[r] . W_gate[e],  u = x_perm[r] . W_up[e]     (fp32 accumulate)
+ *   h[r] = bf16(silu(g) * u),   silu(z) = z / (1 + exp(-z))
+ *   y[r] = bf16(h[r] . W_down[e])                            (fp32 accumulate)
+ *
+ *   x_perm      [M, H] bf16, e.g. from moe_permute.
+ *   w_gate      [E, H, Hp] bf16, w_up [E, H, Hp] bf16, w_down [E, Hp, H] bf16: one contiguous
+ *               tensor per projection; expert e is addressed by row index only.
+ *   cu_seqlens  device [E+1] int32 as produced by moe_permute (read on the device: the host
+ *               never learns the counts). Must be non-decreasing with cu[E] <= M; rows outside
+ *               [0, M) are never written.
+ *   h_scratch   [M, Hp] bf16 out: the SwiGLU activations (kept: the backward pass needs them).
+ *   y           [M, H] bf16 out: expert outputs, row-aligned with x_perm.
+ *   Requires H % 128 == 0, Hp % 128 == 0, 1 <= E <= MOE_MAX_EXPERTS, M < 2^31.
+ *   d_status    nullable: MOE_ERR_DEVICE_TIMEOUT is OR-ed in if a pipeline wait in the kernel
+ *               exceeded its bound (outputs are then incomplete).
+ */
+moe_status moe_grouped_ffn(const void* x_perm, const void* w_gate, const void* w_up,
+                           const void* w_down, const int32_t* cu_seqlens, int64_t M, int64_t H,
+                           int64_t Hp, int32_t E, void* h_scratch, void* y, int32_t* d_status,
+                           void* cuda_stream);
+
+/*
+ * The two passes of moe_grouped_ffn, callable on their own (same arguments, conventions and
+ * requirements; moe_grouped_ffn is exactly moe_grouped_ffn_up_gate then
+ * moe_grouped_ffn_down on the same stream):
+ *   moe_grouped_ffn_up_gate  h[r] = bf16(silu(x_perm[r] . W_gate[e]) * (x_perm[r] . W_up[e]))
+ *   moe_grouped_ffn_down     y[r] = bf16(h[r] . W_down[e])
+ */
+moe_status moe_grouped_ffn_up_gate(const void* x_perm, const void* w_gate, const void* w_up,
+                                   const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp,
+                                   int32_t E, void* h_scratch, int32_t* d_status,
+                                   void* cuda_stream);
+
+moe_status moe_grouped_ffn_down(const void* h_scratch, const void* w_down,
+                                const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp,
+                                int32_t E, void* y, int32_t* d_status, void* cuda_stream);
+
+/*
+ * moe_unpermute_combine - restore token order, scale by route weight, sum the K results
+ * ("Distributed expert parallelism", lifecycle step 8 and "Duplicate route accumulation";
+ * MoonEP README, "combine fwd").
+ *
+ *   out[t] = bf16( sum_{k=0..K-1} route_w[t,k] * float(y[row_id_map[t*K+k]]) )
+ *
+ * with an fp32 accumulator, k ascending. Slots whose row_id_map entry is negative are
+ * skipped.
+ *   y          [M, H] bf16, M = S*K.    row_id_map [S*K] int32 (from moe_permute).
+ *   route_w    [S, K] fp32.             out [S, H] bf16.
+ */
+moe_status moe_unpermute_combine(const void* y, const int32_t* row_id_map, const float* route_w,
+                                 int64_t S, int64_t H, int32_t K, void* out, void* cuda_stream);
+
+/*
+ * moe_maxvio - routing imbalance (MoonEP README, "Performance"):
+ *   maxvio = max_e(T_e / T_bar) - 1,  T_e = counts[e],  T_bar = S*K/E,
+ * evaluated in IEEE double as ((double)max_count * E) / ((double)S * K) - 1.
+ *   counts     device [E] int32.   maxvio device double out.   max_count device int32 out
+ *   (nullable). S*K must be > 0.
+ */
+moe_status moe_maxvio(const int32_t* counts, int32_t E, int64_t S, int32_t K, double* maxvio,
+                      int32_t* max_count, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H_ */

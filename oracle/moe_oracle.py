@@ -158,6 +158,11 @@ def expert_ffn_rows(x_rows_bits: np.ndarray, w_gate_e: np.ndarray, w_up_e: np.nd
     return h_bits, y_bits
 
 
+def expert_down_rows(h_rows_bits: np.ndarray, w_down_e: np.ndarray) -> np.ndarray:
+    """Second half of one expert on given activations: y = bf16(h Wd), float64 products."""
+    return f64_to_bf16_bits(bf16_bits_to_f64(h_rows_bits) @ bf16_bits_to_f64(w_down_e))
+
+
 def grouped_ffn(x_perm_bits: np.ndarray, cu_seqlens: np.ndarray, get_weights, Hp: int):
     """Grouped expert FFN over expert-contiguous rows.
 

@@ -1,0 +1,90 @@
+"""CPU-side checks of the C ABI: the library loads, exports every declared symbol, and
+rejects bad arguments on the host before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import grouped_ffn_moe_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("moe_permute", "moe_grouped_ffn", "moe_unpermute_combine", "moe_maxvio",
+              "moe_permute_workspace_bytes", "moe_status_string", "moe_abi_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = moe.lib()
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} not exported by {moe.LIB_PATH}"
+        assert getattr(lib, n) is not None
+
+
+def test_binding_names_match_abi():
+    for n in ("moe_permute", "moe_grouped_ffn", "moe_unpermute_combine", "moe_maxvio",
+              "moe_permute_workspace_bytes", "moe_status_string"):
+        assert callable(getattr(moe, n))
+
+
+def test_status_strings_and_version():
+    assert moe.moe_status_string(0) == "ok"
+    assert "argument" in moe.moe_status_string(moe.MOE_ERR_INVALID_ARGUMENT)
+    assert "timed out" in moe.moe_status_string(moe.MOE_ERR_DEVICE_TIMEOUT)
+    assert moe.lib().moe_abi_version() >> 16 == 1
+
+
+def test_workspace_bytes():
+    assert moe.moe_permute_workspace_bytes(0, 8, 384) == 0
+    # 65536 tokens x 8 slots = 1024 chunks of 512, times 384 experts, int32
+    assert moe.moe_permute_workspace_bytes(65536, 8, 384) == 1024 * 384 * 4
+    assert moe.moe_permute_workspace_bytes(3, 2, 8) % 256 == 0
+
+
+P = ctypes.c_void_p
+
+
+def fake(addr):
+    return P(addr)
+
+
+def test_host_validation_rejects_without_launch():
+    L = moe.lib()
+    a = fake(0x10000)  # never dereferenced: validation fails first
+    null = P(0)
+    # K > E
+    assert L.moe_permute(a, a, 4, 64, 9, 8, a, a, a, a, null, null, null, a, 1 << 20, null, null) == 1
+    # E beyond the supported maximum
+    assert L.moe_permute(a, a, 4, 64, 2, 5000, a, a, a, a, null, null, null, a, 1 << 20, null,
+                         null) == 2
+    # missing outputs
+    assert L.moe_permute(a, a, 4, 64, 2, 8, a, null, a, a, null, null, null, a, 1 << 20, null,
+                         null) == 1
+    # H not a multiple of 8 with a row copy
+    assert L.moe_permute(a, a, 4, 60, 2, 8, a, a, a, a, null, null, null, a, 1 << 20, null, null) == 2
+    # misaligned x_perm
+    assert L.moe_permute(a, a, 4, 64, 2, 8, fake(0x10008), a, a, a, null, null, null, a, 1 << 20,
+                         null, null) == 1
+    # workspace too small
+    assert L.moe_permute(a, a, 4096, 64, 8, 384, a, a, a, a, null, null, null, a, 16, null, null) == 1
+    # grouped FFN: H' not a multiple of 128, then a null weight
+    assert L.moe_grouped_ffn(a, a, a, a, a, 16, 256, 200, 4, a, a, null, null) == 2
+    assert L.moe_grouped_ffn(a, null, a, a, a, 16, 256, 256, 4, a, a, null, null) == 1
+    assert L.moe_grouped_ffn(a, a, a, a, a, 0, 256, 256, 4, a, a, null, null) == 0  # M = 0: no-op
+    # combine: H % 8, K < 1
+    assert L.moe_unpermute_combine(a, a, a, 4, 12, 2, a, null) == 2
+    assert L.moe_unpermute_combine(a, a, a, 4, 16, 0, a, null) == 1
+    assert L.moe_unpermute_combine(a, a, a, 0, 16, 2, a, null) == 0  # S = 0: no-op
+    # maxvio: S*K must be positive
+    assert L.moe_maxvio(a, 8, 0, 2, a, null, null) == 1

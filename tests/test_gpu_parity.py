@@ -1,0 +1,358 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Integer outputs (counts, cu_seqlens, row_id_map, perm_src, max count, maxvio, x_perm) must
+match bit for bit; bf16 outputs (h, y, out) must meet the acceptance bar in helpers.py.
+Small workloads are compared element by element in full; the full-size workloads on
+sampled rows and tokens that the oracle recomputes one by one.
+"""
+import json
+import os
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import grouped_ffn_moe_b200 as moe
+import synth
+from helpers import assert_close_bf16, bf16_ulp, bits, f64
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def gpu_permute(x, ids, E, with_rows=True):
+    S, K = ids.shape
+    dev = ids.device
+    H = x.shape[1]
+    M = S * K
+    i32 = dict(dtype=torch.int32, device=dev)
+    r = dict(
+        x_perm=torch.full((M, H), float("nan"), dtype=torch.bfloat16, device=dev) if with_rows else None,
+        counts=torch.full((E,), -7, **i32), cu=torch.full((E + 1,), -7, **i32),
+        rmap=torch.full((M,), -7, **i32), psrc=torch.full((M,), -7, **i32),
+        maxvio=torch.full((1,), -7.0, dtype=torch.float64, device=dev),
+        max_count=torch.full((1,), -7, **i32), status=torch.zeros(1, **i32))
+    moe.moe_permute(x, ids, E, r["x_perm"], r["counts"], r["cu"], r["rmap"], r["psrc"], r["maxvio"],
+                    r["max_count"], d_status=r["status"])
+    torch.cuda.synchronize()
+    return r
+
+
+def check_permute_exact(r, ids_np, E, x_bits=None, sample_rows=None):
+    S, K = ids_np.shape
+    counts, cu, rmap, psrc = O.permute_metadata(ids_np, E)
+    mv, mc = O.maxvio(counts, S, K)
+    assert np.array_equal(r["counts"].cpu().numpy(), counts)
+    assert np.array_equal(r["cu"].cpu().numpy(), cu)
+    assert np.array_equal(r["rmap"].cpu().numpy(), rmap)
+    assert np.array_equal(r["psrc"].cpu().numpy(), psrc)
+    assert int(r["max_count"].item()) == mc
+    assert r["maxvio"].item() == mv  # same IEEE expression: bit-exact
+    assert int(r["status"].item()) == 0
+    if x_bits is not None and r["x_perm"] is not None:
+        if sample_rows is None:
+            assert np.array_equal(bits(r["x_perm"]), O.permute_rows(x_bits, psrc, K))
+        else:
+            got = bits(r["x_perm"][torch.as_tensor(sample_rows, device=r["x_perm"].device)])
+            assert np.array_equal(got, x_bits[psrc[sample_rows] // K])
+    return counts, cu, rmap, psrc
+
+
+def layer_inputs(w, dev):
+    return synth.make_layer_inputs(w, device=str(dev))
+
+
+def weights_getter(inp):
+    cache = {}
+
+    def get(e):
+        if e not in cache:
+            cache.clear()
+            cache[e] = (bits(inp["w_gate"][e]), bits(inp["w_up"][e]), bits(inp["w_down"][e]))
+        return cache[e]
+    return get
+
+
+def run_layer(inp, w, dev):
+    buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev, with_ffn=not w.identity_ffn)
+    moe.moe_layer_forward(inp["x"], inp["topk_ids"], inp["route_w"], inp.get("w_gate"),
+                          inp.get("w_up"), inp.get("w_down"), buf)
+    torch.cuda.synchronize()
+    assert int(buf.d_status.item()) == 0
+    return buf
+
+
+# ----------------------------------------------------------------------------- permute
+
+def test_permute_four_rank_worked_example(cuda_device):
+    g = json.load(open(os.path.join(GOLDEN, "four_rank_example.json")))
+    ids = torch.tensor(g["topk_ids"], dtype=torch.int32, device=cuda_device)
+    x = torch.arange(3 * 8, dtype=torch.float32, device=cuda_device).reshape(3, 8).to(torch.bfloat16)
+    r = gpu_permute(x, ids, g["E"])
+    assert r["counts"].tolist() == g["counts"]
+    assert r["cu"].tolist() == g["cu_seqlens"]
+    assert r["psrc"].tolist() == g["perm_src"]
+    assert r["rmap"].tolist() == g["row_id_map"]
+    assert r["max_count"].item() == g["max_count"]
+    assert abs(r["maxvio"].item() - 5.0 / 3.0) <= 4e-16
+    xp = r["x_perm"].float().cpu().numpy()
+    for f, row in enumerate(g["row_id_map"]):
+        assert np.array_equal(xp[row], x.float().cpu().numpy()[f // 2])
+
+
+def _routing_case(name):
+    rng = np.random.default_rng(zlib.crc32(name.encode()))
+    if name == "one_expert_k1":
+        return np.zeros((777, 1), np.int32), 5
+    if name == "empty_experts":
+        return rng.choice([1, 4, 9], size=(300, 2)).astype(np.int32), 12
+    if name == "duplicates":
+        return rng.integers(0, 6, size=(513, 4)).astype(np.int32), 6
+    if name == "ragged":
+        return rng.integers(0, 7, size=(1001, 3)).astype(np.int32), 7
+    if name == "e_max":
+        return rng.integers(0, 1024, size=(3000, 8)).astype(np.int32), 1024
+    if name == "many_chunks":
+        return rng.integers(0, 384, size=(20000, 8)).astype(np.int32), 384
+    raise KeyError(name)
+
+
+@pytest.mark.parametrize("name", ["one_expert_k1", "empty_experts", "duplicates", "ragged", "e_max",
+                                  "many_chunks"])
+def test_permute_edge_cases(cuda_device, name):
+    ids_np, E = _routing_case(name)
+    S, K = ids_np.shape
+    H = 64
+    xb = synth.normal_bf16_bits(11, synth.TAG_X, S * H).reshape(S, H)
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(cuda_device)
+    r = gpu_permute(x, torch.from_numpy(ids_np).to(cuda_device), E)
+    check_permute_exact(r, ids_np, E, xb)
+
+
+@pytest.mark.parametrize("wname", ["tiny", "medium", "large", "skew20",
+                                   "permute_combine_S65536_mv20"])
+def test_permute_workloads(cuda_device, wname):
+    w = synth.WORKLOADS[wname]
+    ids_np, _ = synth.routing_for(w)
+    x = synth.normal_bf16_into(torch.empty(w.S, w.H, dtype=torch.bfloat16, device=cuda_device),
+                               w.seed, synth.TAG_X)
+    with_rows = w.S * w.K * w.H * 2 < 8e9
+    r = gpu_permute(x, torch.from_numpy(ids_np).to(cuda_device), w.E, with_rows=with_rows)
+    M = w.S * w.K
+    sample = None if M * w.H <= 64e6 else np.random.default_rng(0).choice(M, 4096, replace=False)
+    xb = bits(x) if with_rows else None
+    check_permute_exact(r, ids_np, w.E, xb, sample)
+
+
+def test_permute_metadata_only_and_zero_tokens(cuda_device):
+    ids_np, E = _routing_case("ragged")
+    ids = torch.from_numpy(ids_np).to(cuda_device)
+    x = torch.zeros(ids_np.shape[0], 64, dtype=torch.bfloat16, device=cuda_device)
+    r = gpu_permute(x, ids, E, with_rows=False)
+    check_permute_exact(r, ids_np, E)
+    # S = 0: counts and offsets are zero, maxvio NaN (T_bar = 0)
+    r0 = gpu_permute(x[:0], ids[:0], E, with_rows=False)
+    assert r0["counts"].abs().sum().item() == 0 and r0["cu"].abs().sum().item() == 0
+    assert np.isnan(r0["maxvio"].item())
+
+
+def test_bad_routing_is_flagged(cuda_device):
+    ids_np = np.array([[0, 1], [2, 7], [3, -1], [1, 2]], dtype=np.int32)
+    ids = torch.from_numpy(ids_np).to(cuda_device)
+    x = torch.ones(4, 64, dtype=torch.bfloat16, device=cuda_device)
+    r = gpu_permute(x, ids, 4)
+    assert int(r["status"].item()) & moe.MOE_ERR_BAD_ROUTING
+    rmap = r["rmap"].cpu().numpy()
+    assert rmap[3] == -1 and rmap[5] == -1
+    good = ids_np.reshape(-1)[[0, 1, 2, 4, 6, 7]]
+    assert r["counts"].tolist() == np.bincount(good, minlength=4).tolist()
+
+
+def test_maxvio_entry_point(cuda_device):
+    counts = torch.tensor([3584] + [161] * 383, dtype=torch.int32, device=cuda_device)
+    mv = torch.zeros(1, dtype=torch.float64, device=cuda_device)
+    mc = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    moe.moe_maxvio(counts, 8192, 8, mv, mc)
+    torch.cuda.synchronize()
+    assert mc.item() == 3584
+    assert mv.item() == O.maxvio(counts.cpu().numpy(), 8192, 8)[0] == 20.0
+
+
+# ----------------------------------------------------------------------------- combine
+
+@pytest.mark.parametrize("wname", ["permute_combine_S1024_mv0", "permute_combine_S4096_mv20"])
+def test_identity_expert_layer(cuda_device, wname):
+    w = synth.WORKLOADS[wname]
+    inp = layer_inputs(w, cuda_device)
+    buf = run_layer(inp, w, cuda_device)
+    ref = O.moe_layer(bits(inp["x"]), inp["topk_ids"].cpu().numpy(), inp["route_w"].cpu().numpy(),
+                      w.E, None, 0, identity_ffn=True)
+    assert np.array_equal(buf.cu_seqlens.cpu().numpy(), ref["cu_seqlens"])
+    assert np.array_equal(buf.row_id_map.cpu().numpy(), ref["row_id_map"])
+    assert buf.maxvio.item() == ref["maxvio"]
+    assert_close_bf16(bits(buf.out), ref["out"], "out")
+
+
+def test_combine_unit_weight_invariants(cuda_device):
+    S, K, E, H = 2000, 4, 16, 256
+    rng = np.random.default_rng(7)
+    ids = torch.from_numpy(np.stack([rng.permutation(E)[:K] for _ in range(S)]).astype(np.int32))
+    ids = ids.to(cuda_device)
+    x = synth.normal_bf16_into(torch.empty(S, H, dtype=torch.bfloat16, device=cuda_device), 3,
+                               synth.TAG_X)
+    buf = moe.LayerBuffers.allocate(S, H, 0, E, K, cuda_device, with_ffn=False)
+    ones = torch.ones(S, K, dtype=torch.float32, device=cuda_device)
+    moe.moe_layer_forward(x, ids, ones, None, None, None, buf)
+    torch.cuda.synchronize()
+    # unpermute o permute with identity experts and unit weights: exactly bf16(K * x)
+    assert torch.equal(buf.out, (x.float() * K).to(torch.bfloat16))
+    # K = 1, weight 1: exactly x
+    buf1 = moe.LayerBuffers.allocate(S, H, 0, E, 1, cuda_device, with_ffn=False)
+    moe.moe_layer_forward(x, ids[:, :1].contiguous(), ones[:, :1].contiguous(), None, None, None, buf1)
+    torch.cuda.synchronize()
+    assert torch.equal(buf1.out, x)
+
+
+# ----------------------------------------------------------------------------- grouped FFN
+
+def _check_full_layer(inp, w, buf):
+    ref = O.moe_layer(bits(inp["x"]), inp["topk_ids"].cpu().numpy(), inp["route_w"].cpu().numpy(),
+                      w.E, weights_getter(inp), w.Hp)
+    assert np.array_equal(buf.counts.cpu().numpy(), ref["counts"])
+    assert np.array_equal(buf.cu_seqlens.cpu().numpy(), ref["cu_seqlens"])
+    assert np.array_equal(buf.row_id_map.cpu().numpy(), ref["row_id_map"])
+    assert np.array_equal(bits(buf.x_perm), ref["x_perm"])
+    assert buf.maxvio.item() == ref["maxvio"]
+    # end to end: the GPU chain against the oracle chain
+    for name in ("h", "y"):
+        stats = assert_close_bf16(bits(getattr(buf, name)), ref[name], name)
+        print(f"[{w.name}] {name}: {stats}")
+    rw = inp["route_w"].cpu().numpy().astype(np.float64)
+    rmap = ref["row_id_map"].reshape(w.S, w.K)
+    inherited = sum(np.abs(rw[:, k:k + 1]) * bf16_ulp(ref["y"][rmap[:, k]]) for k in range(w.K))
+    stats = assert_close_bf16(bits(buf.out), ref["out"], "out", inherited=inherited)
+    print(f"[{w.name}] out (end to end): {stats}")
+    # stage by stage: each kernel against the oracle applied to the GPU's own inputs
+    get = weights_getter(inp)
+    h_gpu = bits(buf.h)
+    y_stage = np.zeros_like(ref["y"])
+    for e in range(w.E):
+        a, b = int(ref["cu_seqlens"][e]), int(ref["cu_seqlens"][e + 1])
+        if b > a:
+            y_stage[a:b] = O.expert_down_rows(h_gpu[a:b], get(e)[2])
+    print(f"[{w.name}] y (stage): {assert_close_bf16(bits(buf.y), y_stage, 'y stage')}")
+    out_stage = O.unpermute_combine(bits(buf.y), ref["row_id_map"], inp["route_w"].cpu().numpy(),
+                                    w.S, w.K)
+    print(f"[{w.name}] out (stage): {assert_close_bf16(bits(buf.out), out_stage, 'out stage')}")
+
+
+def test_layer_tiny_full(cuda_device):
+    w = synth.WORKLOADS["tiny"]
+    inp = layer_inputs(w, cuda_device)
+    _check_full_layer(inp, w, run_layer(inp, w, cuda_device))
+
+
+def test_layer_ragged_chunks_full(cuda_device):
+    """Experts of 0, 1, 15, 16, 17, 255, 256, 257, 600 and 1100 rows: every chunking
+    path of the tile scheduler (one chunk, balanced chunks, tails of 1 row)."""
+    sizes = [0, 1, 15, 16, 17, 255, 256, 257, 600, 1100]
+    E, K, H, Hp = len(sizes), 1, 256, 384
+    ids_np = np.concatenate([np.full(n, e, np.int32) for e, n in enumerate(sizes)])
+    ids_np = np.random.default_rng(9).permutation(ids_np).reshape(-1, 1)
+    S = ids_np.shape[0]
+    w = synth.Workload("ragged", S, H, Hp, E, K, 21)
+    inp = {"topk_ids": torch.from_numpy(ids_np).to(cuda_device),
+           "route_w": torch.ones(S, 1, dtype=torch.float32, device=cuda_device)}
+    inp["x"] = synth.normal_bf16_into(torch.empty(S, H, dtype=torch.bfloat16, device=cuda_device),
+                                      21, synth.TAG_X)
+    for name, tag, shape in (("w_gate", synth.TAG_W_GATE, (E, H, Hp)),
+                             ("w_up", synth.TAG_W_UP, (E, H, Hp)),
+                             ("w_down", synth.TAG_W_DOWN, (E, Hp, H))):
+        inp[name] = synth.normal_bf16_into(torch.empty(*shape, dtype=torch.bfloat16,
+                                                       device=cuda_device), 21, tag,
+                                           synth.weight_scale(w, name[2:]))
+    _check_full_layer(inp, w, run_layer(inp, w, cuda_device))
+
+
+def test_layer_medium_full(cuda_device):
+    w = synth.WORKLOADS["medium"]
+    inp = layer_inputs(w, cuda_device)
+    _check_full_layer(inp, w, run_layer(inp, w, cuda_device))
+
+
+def _sampled_rows(cu, hot, rng, per=6):
+    E = len(cu) - 1
+    experts = sorted({0, E - 1, hot, *rng.choice(E, 5, replace=False).tolist()})
+    rows = []
+    for e in experts:
+        a, b = int(cu[e]), int(cu[e + 1])
+        if b > a:
+            rows += sorted({a, b - 1, (a + b) // 2, *rng.integers(a, b, per).tolist()})
+    return np.array(rows, dtype=np.int64)
+
+
+@pytest.mark.parametrize("wname", ["large", "skew20"])
+def test_layer_full_size_sampled(cuda_device, wname):
+    w = synth.WORKLOADS[wname]
+    inp = layer_inputs(w, cuda_device)
+    buf = run_layer(inp, w, cuda_device)
+    ids_np = inp["topk_ids"].cpu().numpy()
+    counts, cu, rmap, psrc = check_permute_exact(
+        dict(counts=buf.counts, cu=buf.cu_seqlens, rmap=buf.row_id_map, psrc=buf.perm_src,
+             maxvio=buf.maxvio, max_count=buf.max_count, status=buf.d_status, x_perm=None),
+        ids_np, w.E)
+    rng = np.random.default_rng(1)
+    rows = _sampled_rows(cu, int(np.argmax(counts)), rng)
+    x_bits = bits(inp["x"])
+    get = weights_getter(inp)
+    experts = O.expert_of_rows(cu, rows)
+    h_ref = np.zeros((len(rows), w.Hp), np.uint16)
+    y_ref = np.zeros((len(rows), w.H), np.uint16)
+    for e in np.unique(experts):
+        sel = np.nonzero(experts == e)[0]
+        src = x_bits[psrc[rows[sel]] // w.K]
+        h_ref[sel], y_ref[sel] = O.expert_ffn_rows(src, *get(int(e)))
+    idx = torch.as_tensor(rows, device=cuda_device)
+    assert np.array_equal(bits(buf.x_perm[idx]), x_bits[psrc[rows] // w.K])
+    print(f"[{w.name}] h: {assert_close_bf16(bits(buf.h[idx]), h_ref, 'h (sampled rows)')}")
+    print(f"[{w.name}] y: {assert_close_bf16(bits(buf.y[idx]), y_ref, 'y (sampled rows)')}")
+    # whole-layer output for a few tokens, each through its K experts
+    toks = rng.choice(w.S, 3, replace=False)
+    rw = inp["route_w"].cpu().numpy()
+    out_ref = np.zeros((len(toks), w.H), np.uint16)
+    out_stage = np.zeros((len(toks), w.H), np.uint16)
+    inherited = np.zeros((len(toks), w.H))
+    for i, t in enumerate(toks):
+        ys = np.zeros((w.K, w.H), np.uint16)
+        for k in range(w.K):
+            _, ys[k] = O.expert_ffn_rows(x_bits[t:t + 1], *get(int(ids_np[t, k])))
+            inherited[i] += abs(float(rw[t, k])) * bf16_ulp(ys[k])
+        out_ref[i] = O.combine_token(ys, rw[t])
+        y_gpu = bits(buf.y[torch.as_tensor(rmap[t * w.K:(t + 1) * w.K], device=cuda_device)])
+        out_stage[i] = O.combine_token(y_gpu, rw[t])
+    out_gpu = bits(buf.out[torch.as_tensor(toks, device=cuda_device)])
+    print(f"[{w.name}] out: {assert_close_bf16(out_gpu, out_ref, 'out (sampled)', inherited)}")
+    print(f"[{w.name}] out (stage): {assert_close_bf16(out_gpu, out_stage, 'out stage (sampled)')}")
+
+
+def test_layer_is_deterministic(cuda_device):
+    w = synth.WORKLOADS["medium"]
+    inp = layer_inputs(w, cuda_device)
+    a = run_layer(inp, w, cuda_device)
+    b = run_layer(inp, w, cuda_device)
+    for name in ("x_perm", "h", "y", "out"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+
+
+def test_generator_twin_matches_host(cuda_device):
+    """The device twin of the input generator draws the same bf16 values as the host one."""
+    n = 1 << 20
+    for off in (0, 5_000_000_000):
+        t = synth.normal_bf16_into(torch.empty(n, dtype=torch.bfloat16, device=cuda_device), 2,
+                                   synth.TAG_W_GATE, 0.125, offset=off)
+        host = synth.normal_bf16_bits(2, synth.TAG_W_GATE, n, 0.125, offset=off)
+        assert (bits(t) != host).sum() <= 2

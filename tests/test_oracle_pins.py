@@ -305,3 +305,27 @@ def test_mis_addressed_expert_is_visible():
     bad = O.moe_layer(x, (ids + 1) % E, w, E, get, Hp)
     a, b = O.bf16_bits_to_f64(good["out"]), O.bf16_bits_to_f64(bad["out"])
     assert np.linalg.norm(a - b) > 0.3 * np.linalg.norm(a)
+
+
+# ----------------------------------------------------------------------------- acceptance bar
+
+def test_acceptance_bar_accepts_one_step_flips_only():
+    """The bf16 bar: rel-Frobenius and max-abs, where an element beyond the max-abs bar must
+    be exactly one bf16 step from the reference (a rounding-boundary flip)."""
+    from helpers import assert_close_bf16
+
+    rng = np.random.default_rng(12)
+    ref = O.f64_to_bf16_bits(rng.standard_normal(100000))
+    ref[7] = O.f64_to_bf16_bits(np.array([13.0]))[0]  # an outlier at ~13 rms
+    got = ref.copy()
+    got[7] += 1  # one step: 13.0 -> 13.0625, above 3e-2 * rms
+    stats = assert_close_bf16(got, ref, "flip")
+    assert stats["one_step_flips_over_bar"] == 1
+    bad = ref.copy()
+    bad[7] += 2  # two steps: rejected
+    with pytest.raises(AssertionError):
+        assert_close_bf16(bad, ref, "two steps")
+    wrong_row = ref.copy()
+    wrong_row[:100] = ref[100:200]  # mis-addressed rows: rejected
+    with pytest.raises(AssertionError):
+        assert_close_bf16(wrong_row, ref, "wrong rows")
