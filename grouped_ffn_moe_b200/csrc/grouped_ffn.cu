@@ -45,15 +45,16 @@ namespace {
 constexpr int kBM = 128;                       // output features per unit (UMMA M)
 constexpr int kBK = 64;                        // reduction elements per stage (128 bytes)
 constexpr int kNMax = 256;                     // tokens per unit (UMMA N max)
-constexpr int kRowsPerBox = 16;                // token rows per TMA box
-constexpr int kABytes = kBM * kBK * 2;         // 16 KB: two [64 k][64 f] boxes
-constexpr int kABoxBytes = 64 * kBK * 2;       // 8 KB
+constexpr int kABytes = kBM * kBK * 2;         // 16 KB: [2 halves][64 k][64 f], one TMA box
+constexpr int kAHalfBytes = 64 * kBK * 2;      // 8 KB: one 64-feature half (UMMA LBO)
 constexpr int kBBytes = kNMax * kBK * 2;       // 32 KB
-constexpr int kBBoxBytes = kRowsPerBox * kBK * 2;  // 2 KB
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kRowBytes = kBK * 2;             // one token row of a B stage (128 bytes)
+constexpr int kNumBoxHeights = 5;              // token boxes of 256, 128, 64, 32, 16 rows
+constexpr int kEpiGroups = 2;                  // epilogue warp groups, alternating chunks
+constexpr int kEpiThreads = 128 * kEpiGroups;
+constexpr int kThreads = 64 + kEpiThreads;     // TMA warp, MMA warp, epilogue warps
 constexpr int kOutChunk = 32;                  // tokens per epilogue chunk
-constexpr int kOutBytes = kOutChunk * kBM * 2;  // 8 KB staging buffer
+constexpr int kOutBytes = kOutChunk * kBM * 2;  // 8 KB staging buffer per group
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = 256;
 
@@ -65,7 +66,7 @@ struct Cfg {
   static constexpr int kStageBytes = kNumA * kABytes + kBBytes;
   static constexpr int kPipeBytes = kStages * kStageBytes;
   static constexpr int kOffOut = kPipeBytes;
-  static constexpr int kOffCu = kOffOut + 2 * kOutBytes;
+  static constexpr int kOffCu = kOffOut + kEpiGroups * kOutBytes;
   static constexpr int kOffUnits = kOffCu + 4 * (MOE_MAX_EXPERTS + 1);
   static constexpr int kOffBars = (kOffUnits + 4 * (MOE_MAX_EXPERTS + 1) + 7) & ~7;
   static constexpr int kNumBars = 2 * kStages + 2 * 2 + 1;
@@ -74,6 +75,13 @@ struct Cfg {
 };
 static_assert(Cfg<true>::kSmemBytes <= 232448, "shared memory budget (dual)");
 static_assert(Cfg<false>::kSmemBytes <= 232448, "shared memory budget (single)");
+
+// Token-row tensor maps of one activation matrix, box heights 256, 128, 64, 32, 16 rows: a
+// unit's N rows (a multiple of 16) load as the binary decomposition of N, i.e. at most five
+// boxes and no row beyond the 16-row rounding.
+struct RowMaps {
+  CUtensorMap m[kNumBoxHeights];
+};
 
 struct FfnArgs {
   const int32_t* cu;     // [E+1]
@@ -87,7 +95,7 @@ struct FfnArgs {
 };
 
 struct Unit {
-  int e, fb, row0, nrows;
+  int e, fb, row0, nrows, ntc;
 };
 
 // Unit u -> (expert, feature block, token rows). s_ustart[e] is the first unit of expert e.
@@ -103,6 +111,7 @@ __device__ __forceinline__ Unit decode_unit(int u, const int32_t* s_ustart, cons
   const int local = u - s_ustart[lo];
   const int cnt = s_cu[lo + 1] - s_cu[lo];
   const int ntc = (cnt + kNMax - 1) / kNMax;
+  U.ntc = ntc;
   U.fb = local / ntc;
   const int tc = local - U.fb * ntc;
   const int cs = (((cnt + ntc - 1) / ntc) + 15) & ~15;  // balanced chunks, multiple of 16
@@ -121,7 +130,7 @@ template <bool kDual>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_ffn_kernel(const __grid_constant__ CUtensorMap tmA0,
                        const __grid_constant__ CUtensorMap tmA1,
-                       const __grid_constant__ CUtensorMap tmB, const FfnArgs args) {
+                       const __grid_constant__ RowMaps tmB, const FfnArgs args) {
   using C = Cfg<kDual>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
@@ -151,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&tfull[s], 1);
-      mbar_init(&tempty[s], kEpiThreads / 32);
+      mbar_init(&tempty[s], kEpiThreads / 32);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -160,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&tmA0);
     if (kDual) tma_prefetch_map(&tmA1);
-    tma_prefetch_map(&tmB);
+    for (int i = 0; i < kNumBoxHeights; ++i) tma_prefetch_map(&tmB.m[i]);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, kTmemCols);
@@ -212,32 +221,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // TMA producer
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();  // weights: streamed once
-      const uint64_t pol_x = policy_evict_last();   // token rows: reused by all feature blocks
+      const uint64_t pol_stream = policy_evict_first();  // weights read by one unit only
+      const uint64_t pol_keep = policy_evict_last();     // token rows (all feature blocks) and
+                                                         // weights shared by an expert's chunks
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
       for (int u = blockIdx.x; u < total_units && !*s_abort; u += gridDim.x) {
         const Unit U = decode_unit(u, s_ustart, s_cu, E);
         if (U.nrows <= 0) continue;
-        const int nbox = (U.nrows + kRowsPerBox - 1) / kRowsPerBox;
-        const uint32_t bytes = C::kNumA * kABytes + nbox * kBBoxBytes;
-        const int fx = U.fb * kBM;
+        const int n = (U.nrows + 15) & ~15;
+        const uint32_t bytes = C::kNumA * kABytes + n * kRowBytes;
+        const uint64_t pol_w = U.ntc > 1 ? pol_keep : pol_stream;
+        const int fz = U.fb * 2;  // 64-feature half index of the unit's first feature
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, s_abort, args.budget_ns)) break;
           uint8_t* st = smem + stage * C::kStageBytes;
           const int ky = U.e * args.k_dim + kt * kBK;
           mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d_hint(st, &tmA0, &full[stage], fx, ky, pol_w);
-          tma_load_2d_hint(st + kABoxBytes, &tmA0, &full[stage], fx + 64, ky, pol_w);
-          if (kDual) {
-            tma_load_2d_hint(st + kABytes, &tmA1, &full[stage], fx, ky, pol_w);
-            tma_load_2d_hint(st + kABytes + kABoxBytes, &tmA1, &full[stage], fx + 64, ky, pol_w);
-          }
+          tma_load_3d_hint(st, &tmA0, &full[stage], 0, ky, fz, pol_w);
+          if (kDual) tma_load_3d_hint(st + kABytes, &tmA1, &full[stage], 0, ky, fz, pol_w);
           uint8_t* sb = st + C::kNumA * kABytes;
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d_hint(sb + b * kBBoxBytes, &tmB, &full[stage], kt * kBK,
-                             U.row0 + b * kRowsPerBox, pol_x);
+          int r = 0;
+#pragma unroll
+          for (int i = 0; i < kNumBoxHeights; ++i) {
+            const int h = kNMax >> i;
+            if (n & h) {
+              tma_load_2d_hint(sb + r * kRowBytes, &tmB.m[i], &full[stage], kt * kBK, U.row0 + r,
+                               pol_keep);
+              r += h;
+            }
+          }
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) {
@@ -285,9 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t bdesc = smem_desc_sw128(b0 + kk * 32, 16, 1024);
             const uint32_t acc = (kt | kk) != 0 ? 1u : 0u;
-            umma_f16(d0, smem_desc_sw128(a0 + kk * 2048, kABoxBytes, 1024), bdesc, idesc, acc);
+            umma_f16(d0, smem_desc_sw128(a0 + kk * 2048, kAHalfBytes, 1024), bdesc, idesc, acc);
             if (kDual)
-              umma_f16(d1, smem_desc_sw128(a1 + kk * 2048, kABoxBytes, 1024), bdesc, idesc, acc);
+              umma_f16(d1, smem_desc_sw128(a1 + kk * 2048, kAHalfBytes, 1024), bdesc, idesc, acc);
           }
           issued_any = true;
           umma_commit(&empty[stage]);  // frees the smem stage when these MMAs complete
@@ -310,36 +324,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // Epilogue: warps 2..5; warp w reads TMEM lanes 32*(w%4) .. +31 (its feature rows)
+    // Epilogue: warps 2..9 in two groups of four (warps 2-5 and 6-9); group g drains the
+    // 32-token chunks c with (c / 32) % 2 == g. Warp w reads TMEM lanes 32*(w%4) .. +31, i.e.
+    // 32 of the unit's 128 features, and within a group the four warps cover all 128.
     const int q = warp & 3;
+    const int grp = (warp - 2) >> 2;
     const int f_local = q * 32 + lane;
-    const int et = tid - 64;  // 0..127
+    const int gt = (tid - 64) & 127;  // thread index inside the group
+    const uint32_t bar_grp = 1 + grp, bar_all = 3;
+    uint8_t* so_bytes = s_out + grp * kOutBytes;
+    __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(so_bytes);
     int astage = 0;
     uint32_t aphase = 0;
-    uint32_t chunk_ctr = 0;
     for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
       const Unit U = decode_unit(u, s_ustart, s_cu, E);
       if (U.nrows <= 0) continue;
       mbar_wait_bounded(&tfull[astage], aphase, s_abort, args.budget_ns);
-      named_bar_sync(1, kEpiThreads);  // all four warps take the same abort decision
+      named_bar_sync(bar_all, kEpiThreads);  // every epilogue warp takes the same decision
       if (*s_abort) break;
       tc_fence_after();
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (kDual ? 0u : astage * kAccCols);
-      for (int c = 0; c < U.nrows; c += kOutChunk) {
+      for (int c = grp * kOutChunk; c < U.nrows; c += kEpiGroups * kOutChunk) {
         __syncwarp();  // tcgen05.ld is .sync.aligned: whole warp, converged
         uint32_t r0[32];
         tmem_ld_32x32b_x32(tbase + c, r0);
-        __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(s_out + (chunk_ctr & 1u) * kOutBytes);
         if (kDual) {
           uint32_t r1[32];
           tmem_ld_32x32b_x32(tbase + kAccCols + c, r1);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
+            // silu(g) * u = g / (1 + e^-g) * u (fast exp and divide; the result is rounded
+            // to bf16, whose step is 2^16 times coarser than their error)
             const float g = __uint_as_float(r0[j]);
-            const float v = __uint_as_float(r1[j]);
-            const float hval = (g / (1.0f + expf(-g))) * v;
+            const float hval = __fdividef(g, 1.0f + __expf(-g)) * __uint_as_float(r1[j]);
             so[j * kBM + f_local] = __float2bfloat16_rn(hval);
           }
         } else {
@@ -347,20 +366,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) so[j * kBM + f_local] = __float2bfloat16_rn(__uint_as_float(r0[j]));
         }
-        named_bar_sync(1, kEpiThreads);
-        const uint8_t* sob = reinterpret_cast<const uint8_t*>(so);
+        named_bar_sync(bar_grp, 128);
 #pragma unroll
-        for (int p = 0; p < (kOutChunk * kBM * 2 / 16) / kEpiThreads; ++p) {
-          const int vid = et + kEpiThreads * p;
+        for (int p = 0; p < (kOutChunk * kBM * 2 / 16) / 128; ++p) {
+          const int vid = gt + 128 * p;
           const int j = vid >> 4, c16 = vid & 15;
           if (c + j < U.nrows) {
-            const uint4 val = *reinterpret_cast<const uint4*>(sob + j * (kBM * 2) + c16 * 16);
+            const uint4 val = *reinterpret_cast<const uint4*>(so_bytes + j * (kBM * 2) + c16 * 16);
             __nv_bfloat16* dst = args.out + static_cast<int64_t>(U.row0 + c + j) * args.n_feat +
                                  U.fb * kBM + c16 * 8;
             *reinterpret_cast<uint4*>(dst) = val;
           }
         }
-        ++chunk_ctr;
+        named_bar_sync(bar_grp, 128);  // staging buffer free for the group's next chunk
       }
       tc_fence_before();
       __syncwarp();
@@ -398,19 +416,40 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix [outer, inner] with a (box_inner x box_outer) box, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
-              uint32_t box_outer) {
+// Token rows: row-major bf16 [rows, inner] with a (64 x box_rows) box, 128-byte swizzle.
+bool make_row_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows,
+                  uint32_t box_rows) {
   auto enc = get_encode_fn();
   if (enc == nullptr) return false;
-  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_row_maps(RowMaps* maps, const void* ptr, uint64_t inner, uint64_t rows) {
+  for (int i = 0; i < kNumBoxHeights; ++i)
+    if (!make_row_map(&maps->m[i], ptr, inner, rows, static_cast<uint32_t>(kNMax >> i)))
+      return false;
+  return true;
+}
+
+// Weights W[E * k_dim][n_feat] (bf16, features contiguous) viewed in three dimensions,
+// (64 features, E * k_dim rows, n_feat / 64 halves): one (64 x 64 x 2) box is the unit's
+// 128 features x 64 k, laid out as two 8 KB MN-major halves, 128-byte swizzle.
+bool make_weight_map(CUtensorMap* m, const void* ptr, uint64_t n_feat, uint64_t rows) {
+  auto enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {64, rows, n_feat / 64};
+  cuuint64_t strides[2] = {n_feat * 2, 128};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kBK), 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 uint64_t wait_budget_ns() {
@@ -443,18 +482,20 @@ moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const voi
                            void* out, int32_t* d_status, cudaStream_t stream) {
   const int grid = num_sms();
   if (dual) {
-    CUtensorMap m_wg, m_wu, m_x;
-    if (!make_map(&m_wg, w0, Hp, static_cast<uint64_t>(E) * H, 64, 64) ||
-        !make_map(&m_wu, w1, Hp, static_cast<uint64_t>(E) * H, 64, 64) ||
-        !make_map(&m_x, act, H, M, 64, kRowsPerBox) || !ensure_smem_attr<true>())
+    CUtensorMap m_wg, m_wu;
+    RowMaps m_x;
+    if (!make_weight_map(&m_wg, w0, Hp, static_cast<uint64_t>(E) * H) ||
+        !make_weight_map(&m_wu, w1, Hp, static_cast<uint64_t>(E) * H) ||
+        !make_row_maps(&m_x, act, H, M) || !ensure_smem_attr<true>())
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
                     static_cast<int32_t>(H), static_cast<int32_t>(Hp), wait_budget_ns()};
     grouped_ffn_kernel<true><<<grid, kThreads, Cfg<true>::kSmemBytes, stream>>>(m_wg, m_wu, m_x, a);
   } else {
-    CUtensorMap m_wd, m_h;
-    if (!make_map(&m_wd, w0, H, static_cast<uint64_t>(E) * Hp, 64, 64) ||
-        !make_map(&m_h, act, Hp, M, 64, kRowsPerBox) || !ensure_smem_attr<false>())
+    CUtensorMap m_wd;
+    RowMaps m_h;
+    if (!make_weight_map(&m_wd, w0, H, static_cast<uint64_t>(E) * Hp) ||
+        !make_row_maps(&m_h, act, Hp, M) || !ensure_smem_attr<false>())
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
                     static_cast<int32_t>(Hp), static_cast<int32_t>(H), wait_budget_ns()};

@@ -4,7 +4,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/moe_b200.h"
+#include "moe_b200.h"
 
 namespace moe {
 

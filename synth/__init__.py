@@ -247,6 +247,9 @@ WORKLOADS: dict[str, Workload] = {
         Workload("skew10", 8192, 7168, 2048, 384, 8, 4, "capped", 10.0),
         Workload("skew20", 8192, 7168, 2048, 384, 8, 5, "capped", 20.0),
         Workload("skew20_last", 8192, 7168, 2048, 384, 8, 5, "capped", 20.0, hot_e=383),
+        # per-expert shape of "large" (171 rows per expert) on 32 experts: 2.8 GB of weights,
+        # small enough for detailed profiler captures
+        Workload("large_slice", 684, 7168, 2048, 32, 8, 2, "capped", 0.2),
     ]
     + [_c5(S, mv) for S in (1024, 4096, 16384, 65536) for mv in (0, 1, 20)]
 }
