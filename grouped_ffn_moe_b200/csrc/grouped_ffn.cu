@@ -5,7 +5,7 @@
 // "Integration" and "Weight buffer": experts addressed by row index of one contiguous
 // [E, H, H'] tensor per projection, cu_seqlens selects the rows):
 //
-//   pass 1 (kDual):  h[r] = bf16( silu(x[r] . W_gate[e]) * (x[r] . W_up[e]) )
+//   pass 1 (SwiGLU): h[r] = bf16( silu(x[r] . W_gate[e]) * (x[r] . W_up[e]) )
 //   pass 2:          y[r] = bf16( h[r] . W_down[e] )
 //
 // Design ("swap AB"): the tensor-core M side (128) runs over output features and the N side
@@ -35,6 +35,7 @@
 #include <atomic>
 #include <cstdlib>
 #include <mutex>
+#include <string>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -58,11 +59,19 @@ constexpr int kOutBytes = kOutChunk * kBM * 2;  // 8 KB staging buffer per group
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = 256;
 
-template <bool kDual>
+// Kernel modes.
+//   kSwiGLU: A0 = W_gate, A1 = W_up on the same 128 features; h = silu(acc0) * acc1.
+//   kSingle: A0 = one 128-feature block; two TMEM accumulators double-buffered.
+//   kPair:   A0, A1 = two adjacent 128-feature blocks of one weight tensor sharing the token
+//            tile (half the token-row traffic per feature); y = acc0 | acc1.
+enum Mode : int { kSwiGLU = 0, kSingle = 1, kPair = 2 };
+
+template <int kMode>
 struct Cfg {
-  static constexpr int kNumA = kDual ? 2 : 1;
-  static constexpr int kStages = kDual ? 3 : 4;
-  static constexpr int kAccStages = kDual ? 1 : 2;
+  static constexpr int kNumA = kMode == kSingle ? 1 : 2;
+  static constexpr int kStages = kNumA == 2 ? 3 : 4;
+  static constexpr int kAccStages = kMode == kSingle ? 2 : 1;
+  static constexpr int kFeatPerUnit = kMode == kPair ? 2 * kBM : kBM;
   static constexpr int kStageBytes = kNumA * kABytes + kBBytes;
   static constexpr int kPipeBytes = kStages * kStageBytes;
   static constexpr int kOffOut = kPipeBytes;
@@ -73,8 +82,9 @@ struct Cfg {
   static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 };
-static_assert(Cfg<true>::kSmemBytes <= 232448, "shared memory budget (dual)");
-static_assert(Cfg<false>::kSmemBytes <= 232448, "shared memory budget (single)");
+static_assert(Cfg<kSwiGLU>::kSmemBytes <= 232448, "shared memory budget (SwiGLU)");
+static_assert(Cfg<kSingle>::kSmemBytes <= 232448, "shared memory budget (single)");
+static_assert(Cfg<kPair>::kSmemBytes <= 232448, "shared memory budget (pair)");
 
 // Token-row tensor maps of one activation matrix, box heights 256, 128, 64, 32, 16 rows: a
 // unit's N rows (a multiple of 16) load as the binary decomposition of N, i.e. at most five
@@ -98,7 +108,8 @@ struct Unit {
   int e, fb, row0, nrows, ntc;
 };
 
-// Unit u -> (expert, feature block, token rows). s_ustart[e] is the first unit of expert e.
+// Unit u -> (expert, feature block, token rows). s_ustart[e] is the first unit of expert e;
+// a feature block is 128 features (256 in kPair mode).
 __device__ __forceinline__ Unit decode_unit(int u, const int32_t* s_ustart, const int32_t* s_cu,
                                             int E) {
   int lo = 0, hi = E - 1;
@@ -126,12 +137,13 @@ __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
   return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-template <bool kDual>
+template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_ffn_kernel(const __grid_constant__ CUtensorMap tmA0,
                        const __grid_constant__ CUtensorMap tmA1,
                        const __grid_constant__ RowMaps tmB, const FfnArgs args) {
-  using C = Cfg<kDual>;
+  using C = Cfg<kMode>;
+  constexpr bool kDual = C::kNumA == 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint8_t* s_out = smem + C::kOffOut;
@@ -149,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = args.E;
-  const int nfb = args.n_feat / kBM;
+  const int nfb = (args.n_feat + C::kFeatPerUnit - 1) / C::kFeatPerUnit;
   const int KT = args.k_dim / kBK;
 
   // ------------------------------------------------------------------ prologue
@@ -168,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&tmA0);
-    if (kDual) tma_prefetch_map(&tmA1);
+    if (kMode == kSwiGLU) tma_prefetch_map(&tmA1);
     for (int i = 0; i < kNumBoxHeights; ++i) tma_prefetch_map(&tmB.m[i]);
   }
   if (warp == 1) {
@@ -233,14 +245,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = (U.nrows + 15) & ~15;
         const uint32_t bytes = C::kNumA * kABytes + n * kRowBytes;
         const uint64_t pol_w = U.ntc > 1 ? pol_keep : pol_stream;
-        const int fz = U.fb * 2;  // 64-feature half index of the unit's first feature
+        const int fz = U.fb * (C::kFeatPerUnit / 64);  // 64-feature index of the first feature
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, s_abort, args.budget_ns)) break;
           uint8_t* st = smem + stage * C::kStageBytes;
           const int ky = U.e * args.k_dim + kt * kBK;
           mbar_arrive_expect_tx(&full[stage], bytes);
           tma_load_3d_hint(st, &tmA0, &full[stage], 0, ky, fz, pol_w);
-          if (kDual) tma_load_3d_hint(st + kABytes, &tmA1, &full[stage], 0, ky, fz, pol_w);
+          if (kMode == kSwiGLU) tma_load_3d_hint(st + kABytes, &tmA1, &full[stage], 0, ky, fz, pol_w);
+          // second block of a pair; past the last feature the box is zero-filled (not stored)
+          if (kMode == kPair) tma_load_3d_hint(st + kABytes, &tmA0, &full[stage], 0, ky, fz + 2, pol_w);
           uint8_t* sb = st + C::kNumA * kABytes;
           int r = 0;
 #pragma unroll
@@ -346,39 +360,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (kDual ? 0u : astage * kAccCols);
       for (int c = grp * kOutChunk; c < U.nrows; c += kEpiGroups * kOutChunk) {
-        __syncwarp();  // tcgen05.ld is .sync.aligned: whole warp, converged
-        uint32_t r0[32];
-        tmem_ld_32x32b_x32(tbase + c, r0);
-        if (kDual) {
-          uint32_t r1[32];
-          tmem_ld_32x32b_x32(tbase + kAccCols + c, r1);
-          tmem_ld_wait();
+        // kPair: two 128-feature halves per chunk; otherwise one
+        for (int half = 0; half < (kMode == kPair ? 2 : 1); ++half) {
+          const int f0 = U.fb * C::kFeatPerUnit + half * kBM;
+          if (f0 >= args.n_feat) break;  // uniform across the group
+          __syncwarp();  // tcgen05.ld is .sync.aligned: whole warp, converged
+          uint32_t r0[32];
+          tmem_ld_32x32b_x32(tbase + half * kAccCols + c, r0);
+          if (kMode == kSwiGLU) {
+            uint32_t r1[32];
+            tmem_ld_32x32b_x32(tbase + kAccCols + c, r1);
+            tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            // silu(g) * u = g / (1 + e^-g) * u (fast exp and divide; the result is rounded
-            // to bf16, whose step is 2^16 times coarser than their error)
-            const float g = __uint_as_float(r0[j]);
-            const float hval = __fdividef(g, 1.0f + __expf(-g)) * __uint_as_float(r1[j]);
-            so[j * kBM + f_local] = __float2bfloat16_rn(hval);
+            for (int j = 0; j < 32; ++j) {
+              // silu(g) * u = g / (1 + e^-g) * u (fast exp and divide; the result is rounded
+              // to bf16, whose step is 2^16 times coarser than their error)
+              const float g = __uint_as_float(r0[j]);
+              const float hval = __fdividef(g, 1.0f + __expf(-g)) * __uint_as_float(r1[j]);
+              so[j * kBM + f_local] = __float2bfloat16_rn(hval);
+            }
+          } else {
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              so[j * kBM + f_local] = __float2bfloat16_rn(__uint_as_float(r0[j]));
           }
-        } else {
-          tmem_ld_wait();
+          named_bar_sync(bar_grp, 128);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) so[j * kBM + f_local] = __float2bfloat16_rn(__uint_as_float(r0[j]));
-        }
-        named_bar_sync(bar_grp, 128);
-#pragma unroll
-        for (int p = 0; p < (kOutChunk * kBM * 2 / 16) / 128; ++p) {
-          const int vid = gt + 128 * p;
-          const int j = vid >> 4, c16 = vid & 15;
-          if (c + j < U.nrows) {
-            const uint4 val = *reinterpret_cast<const uint4*>(so_bytes + j * (kBM * 2) + c16 * 16);
-            __nv_bfloat16* dst = args.out + static_cast<int64_t>(U.row0 + c + j) * args.n_feat +
-                                 U.fb * kBM + c16 * 8;
-            *reinterpret_cast<uint4*>(dst) = val;
+          for (int p = 0; p < (kOutChunk * kBM * 2 / 16) / 128; ++p) {
+            const int vid = gt + 128 * p;
+            const int j = vid >> 4, c16 = vid & 15;
+            if (c + j < U.nrows) {
+              const uint4 val =
+                  *reinterpret_cast<const uint4*>(so_bytes + j * (kBM * 2) + c16 * 16);
+              __nv_bfloat16* dst =
+                  args.out + static_cast<int64_t>(U.row0 + c + j) * args.n_feat + f0 + c16 * 8;
+              *reinterpret_cast<uint4*>(dst) = val;
+            }
           }
+          named_bar_sync(bar_grp, 128);  // staging buffer free for the group's next use
         }
-        named_bar_sync(bar_grp, 128);  // staging buffer free for the group's next chunk
       }
       tc_fence_before();
       __syncwarp();
@@ -461,18 +482,29 @@ uint64_t wait_budget_ns() {
   return budget;
 }
 
-template <bool kDual>
+template <int kMode>
 bool ensure_smem_attr() {
   static std::atomic<int> done_dev_mask{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   const int bit = 1 << (dev & 31);
   if (done_dev_mask.load() & bit) return true;
-  if (cudaFuncSetAttribute(grouped_ffn_kernel<kDual>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Cfg<kDual>::kSmemBytes) != cudaSuccess)
+  if (cudaFuncSetAttribute(grouped_ffn_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Cfg<kMode>::kSmemBytes) != cudaSuccess)
     return false;
   done_dev_mask.fetch_or(bit);
   return true;
+}
+
+// Down-projection kernel: "pair" (two 128-feature blocks per unit, default) or "single",
+// from MOE_DOWN_KERNEL; both give identical results.
+int down_mode() {
+  static int mode = [] {
+    const char* s = std::getenv("MOE_DOWN_KERNEL");
+    return (s != nullptr && std::string(s) == "single") ? static_cast<int>(kSingle)
+                                                        : static_cast<int>(kPair);
+  }();
+  return mode;
 }
 
 }  // namespace
@@ -486,21 +518,28 @@ moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const voi
     RowMaps m_x;
     if (!make_weight_map(&m_wg, w0, Hp, static_cast<uint64_t>(E) * H) ||
         !make_weight_map(&m_wu, w1, Hp, static_cast<uint64_t>(E) * H) ||
-        !make_row_maps(&m_x, act, H, M) || !ensure_smem_attr<true>())
+        !make_row_maps(&m_x, act, H, M) || !ensure_smem_attr<kSwiGLU>())
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
                     static_cast<int32_t>(H), static_cast<int32_t>(Hp), wait_budget_ns()};
-    grouped_ffn_kernel<true><<<grid, kThreads, Cfg<true>::kSmemBytes, stream>>>(m_wg, m_wu, m_x, a);
+    grouped_ffn_kernel<kSwiGLU><<<grid, kThreads, Cfg<kSwiGLU>::kSmemBytes, stream>>>(m_wg, m_wu,
+                                                                                    m_x, a);
   } else {
     CUtensorMap m_wd;
     RowMaps m_h;
+    const bool pair = down_mode() == kPair;
     if (!make_weight_map(&m_wd, w0, H, static_cast<uint64_t>(E) * Hp) ||
-        !make_row_maps(&m_h, act, Hp, M) || !ensure_smem_attr<false>())
+        !make_row_maps(&m_h, act, Hp, M) ||
+        !(pair ? ensure_smem_attr<kPair>() : ensure_smem_attr<kSingle>()))
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
                     static_cast<int32_t>(Hp), static_cast<int32_t>(H), wait_budget_ns()};
-    grouped_ffn_kernel<false><<<grid, kThreads, Cfg<false>::kSmemBytes, stream>>>(m_wd, m_wd, m_h,
-                                                                                  a);
+    if (pair)
+      grouped_ffn_kernel<kPair><<<grid, kThreads, Cfg<kPair>::kSmemBytes, stream>>>(m_wd, m_wd,
+                                                                                     m_h, a);
+    else
+      grouped_ffn_kernel<kSingle><<<grid, kThreads, Cfg<kSingle>::kSmemBytes, stream>>>(
+          m_wd, m_wd, m_h, a);
   }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

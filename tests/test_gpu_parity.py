@@ -256,11 +256,13 @@ def test_layer_tiny_full(cuda_device):
     _check_full_layer(inp, w, run_layer(inp, w, cuda_device))
 
 
-def test_layer_ragged_chunks_full(cuda_device):
+@pytest.mark.parametrize("H,Hp", [(256, 384), (384, 256)])
+def test_layer_ragged_chunks_full(cuda_device, H, Hp):
     """Experts of 0, 1, 15, 16, 17, 255, 256, 257, 600 and 1100 rows: every chunking
-    path of the tile scheduler (one chunk, balanced chunks, tails of 1 row)."""
+    path of the tile scheduler (one chunk, balanced chunks, tails of 1 row); H = 384 leaves
+    the down projection's last 256-feature pair half empty."""
     sizes = [0, 1, 15, 16, 17, 255, 256, 257, 600, 1100]
-    E, K, H, Hp = len(sizes), 1, 256, 384
+    E, K = len(sizes), 1
     ids_np = np.concatenate([np.full(n, e, np.int32) for e, n in enumerate(sizes)])
     ids_np = np.random.default_rng(9).permutation(ids_np).reshape(-1, 1)
     S = ids_np.shape[0]
@@ -356,3 +358,30 @@ def test_generator_twin_matches_host(cuda_device):
                                    synth.TAG_W_GATE, 0.125, offset=off)
         host = synth.normal_bf16_bits(2, synth.TAG_W_GATE, n, 0.125, offset=off)
         assert (bits(t) != host).sum() <= 2
+
+
+def test_down_kernel_variants_agree(cuda_device, tmp_path):
+    """The two down-projection kernels ("pair", default, and "single") give bit-identical y:
+    both accumulate every output in the same order. The variant is chosen per process."""
+    import subprocess
+    import sys
+
+    script = (
+        "import sys, torch, synth, grouped_ffn_moe_b200 as moe\n"
+        "w = synth.WORKLOADS['medium']\n"
+        "inp = synth.make_layer_inputs(w, device='cuda:0')\n"
+        "buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, torch.device('cuda:0'))\n"
+        "moe.moe_layer_forward(inp['x'], inp['topk_ids'], inp['route_w'], inp['w_gate'],"
+        " inp['w_up'], inp['w_down'], buf)\n"
+        "torch.cuda.synchronize()\n"
+        "assert int(buf.d_status.item()) == 0\n"
+        "torch.save(buf.y.cpu(), sys.argv[1])\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    outs = {}
+    for mode in ("pair", "single"):
+        env = dict(os.environ, MOE_DOWN_KERNEL=mode, PYTHONPATH=root)
+        path = str(tmp_path / f"y_{mode}.pt")
+        subprocess.run([sys.executable, "-c", script, path], check=True, env=env, cwd=root,
+                       timeout=600)
+        outs[mode] = torch.load(path)
+    assert torch.equal(outs["pair"], outs["single"])
