@@ -329,3 +329,16 @@ def test_acceptance_bar_accepts_one_step_flips_only():
     wrong_row[:100] = ref[100:200]  # mis-addressed rows: rejected
     with pytest.raises(AssertionError):
         assert_close_bf16(wrong_row, ref, "wrong rows")
+
+
+def test_expert_down_rows_against_torch():
+    """The stage-wise down projection (used to check the down kernel on its own inputs)
+    equals torch's fp64 matmul rounded to bf16 (torch rounds via float32: allow 1 step)."""
+    rng = np.random.default_rng(13)
+    h = O.f64_to_bf16_bits(rng.standard_normal((40, 24)))
+    wd = O.f64_to_bf16_bits(rng.standard_normal((24, 16)) / math.sqrt(24))
+    got = O.bf16_bits_to_f64(O.expert_down_rows(h, wd))
+    T = lambda b: torch_bf16_of(b).to(torch.float64)
+    ref = (T(h) @ T(wd)).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert (got == ref).mean() > 0.99
+    np.testing.assert_allclose(got, ref, rtol=2.0 ** -7, atol=1e-30)
