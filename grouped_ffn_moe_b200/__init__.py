@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.moe_permute_workspace_bytes.argtypes = [i64, i32, i32]
         L.moe_permute.restype = i32
         L.moe_permute.argtypes = [p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p, sz, p, p]
+        L.moe_permute_no_alloc.restype = i32
+        L.moe_permute_no_alloc.argtypes = [p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p, p]
         L.moe_grouped_ffn.restype = i32
         L.moe_grouped_ffn.argtypes = [p, p, p, p, p, i64, i64, i64, i32, p, p, p, p]
         L.moe_grouped_ffn_up_gate.restype = i32
@@ -139,6 +141,31 @@ def moe_permute(x, topk_ids, E, x_perm, counts, cu_seqlens, row_id_map, perm_src
                            _ptr(max_count), _ptr(workspace), wbytes, _ptr(d_status),
                            _stream(stream, dev))
     _check("moe_permute", st)
+
+
+MOE_NO_ALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def moe_permute_no_alloc(x, topk_ids, E, x_perm, counts, cu_seqlens, row_id_map, perm_src=None,
+                         maxvio=None, max_count=None, d_status=None, stream=None):
+    """moe_permute without a workspace argument, for callers that may not allocate device
+    memory: the scratch is a fixed 4 MiB array inside the library (see include/moe_b200.h
+    for the size limit and the sharing rules). Allocates nothing."""
+    S, K = topk_ids.shape
+    dev = topk_ids.device
+    _need(topk_ids, "topk_ids", torch.int32, dev, 2)
+    _need(x, "x", torch.bfloat16, dev, 2)
+    _need(x_perm, "x_perm", torch.bfloat16, dev, 2)
+    for t, n in ((counts, "counts"), (cu_seqlens, "cu_seqlens"), (row_id_map, "row_id_map"),
+                 (perm_src, "perm_src"), (max_count, "max_count"), (d_status, "d_status")):
+        _need(t, n, torch.int32, dev)
+    _need(maxvio, "maxvio", torch.float64, dev)
+    H = x.shape[1] if x is not None else 0
+    st = lib().moe_permute_no_alloc(_ptr(x), _ptr(topk_ids), S, H, K, E, _ptr(x_perm),
+                                    _ptr(counts), _ptr(cu_seqlens), _ptr(row_id_map),
+                                    _ptr(perm_src), _ptr(maxvio), _ptr(max_count),
+                                    _ptr(d_status), _stream(stream, dev))
+    _check("moe_permute_no_alloc", st)
 
 
 def moe_grouped_ffn(x_perm, w_gate, w_up, w_down, cu_seqlens, h_scratch, y, d_status=None,

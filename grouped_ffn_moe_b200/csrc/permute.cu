@@ -13,6 +13,7 @@
 //               replays its chunk with per-expert cursors -> row_id_map, perm_src
 //   permute_rows one warp per token: read the row once (16-byte vectors), write K copies
 #include <algorithm>
+#include <mutex>
 
 #include "internal.h"
 
@@ -271,4 +272,52 @@ moe_status launch_maxvio(const int32_t* counts, int32_t E, int64_t S, int32_t K,
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// ----------------------------------------------------------------------------- no-alloc entry
+
+// Scratch of moe_permute_no_alloc, in the library's own device memory: every GPU that loads
+// the library holds MOE_NO_ALLOC_SCRATCH_BYTES of it until the process exits. All calls on a
+// device share it.
+static __device__ __align__(256) int32_t g_permute_scratch[MOE_NO_ALLOC_SCRATCH_BYTES / 4];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_permute_scratch on the current device. The host-side name is only a
+// stand-in, so the address is looked up once per device (with that device current) and kept.
+moe_status scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr)
+      return MOE_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
 }  // namespace moe
+
+extern "C" moe_status moe_permute_no_alloc(const void* x, const int32_t* topk_ids, int64_t S,
+                                           int64_t H, int32_t K, int32_t E, void* x_perm,
+                                           int32_t* counts, int32_t* cu_seqlens,
+                                           int32_t* row_id_map, int32_t* perm_src, double* maxvio,
+                                           int32_t* max_count, int32_t* d_status,
+                                           void* cuda_stream) {
+  if (S < 0 || K < 1 || E < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (moe_permute_workspace_bytes(S, K, E) > MOE_NO_ALLOC_SCRATCH_BYTES)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  void* scratch = nullptr;
+  const moe_status st = moe::scratch_address(&scratch);
+  if (st != MOE_OK) return st;
+  // The kernels write every scratch entry they later read, so nothing is cleared first.
+  return moe_permute(x, topk_ids, S, H, K, E, x_perm, counts, cu_seqlens, row_id_map, perm_src,
+                     maxvio, max_count, scratch, MOE_NO_ALLOC_SCRATCH_BYTES, d_status,
+                     cuda_stream);
+}

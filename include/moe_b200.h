@@ -100,6 +100,36 @@ moe_status moe_permute(const void* x, const int32_t* topk_ids, int64_t S, int64_
                        void* cuda_stream);
 
 /*
+ * moe_permute_no_alloc - moe_permute for callers that cannot allocate device memory.
+ *
+ * This entry point has no counterpart in the pages this library follows; it exists for
+ * callers that cannot hand moe_permute a workspace because they may not allocate device
+ * memory at the point of the call: for example a plugin inside an inference engine whose
+ * memory was planned up front, or a host framework that owns the whole device memory pool
+ * and forbids cudaMalloc while it runs. It behaves exactly like moe_permute (same arguments
+ * without workspace/workspace_bytes, same outputs bit for bit) but takes its scratch from
+ * a fixed array inside this library's own device memory instead of from the caller.
+ *
+ *   - Limit: moe_permute_workspace_bytes(S, K, E) must be at most MOE_NO_ALLOC_SCRATCH_BYTES
+ *     (4 MiB: e.g. S*K up to 524288 routed slots with E up to 1024); larger problems return
+ *     MOE_ERR_UNSUPPORTED_SHAPE and launch nothing. Use moe_permute with a workspace then.
+ *   - Every GPU that loads the library holds this array until the process exits.
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current) and keeps it; make that first call before any stream capture.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - All calls on a device share the one array, and it keeps the last call's contents.
+ *     Nothing in it has to start at zero (each call writes every entry it reads), but calls
+ *     whose work overlaps on the GPU (e.g. on two streams at once) race on it: order them.
+ */
+#define MOE_NO_ALLOC_SCRATCH_BYTES (4u << 20)
+
+moe_status moe_permute_no_alloc(const void* x, const int32_t* topk_ids, int64_t S, int64_t H,
+                                int32_t K, int32_t E, void* x_perm, int32_t* counts,
+                                int32_t* cu_seqlens, int32_t* row_id_map, int32_t* perm_src,
+                                double* maxvio, int32_t* max_count, int32_t* d_status,
+                                void* cuda_stream);
+
+/*
  * moe_grouped_ffn - grouped expert SwiGLU FFN over expert-contiguous rows ("Mixture of
  * Kittens" digest, Step 1; MoonEP README, "Integration" and "Weight buffer"; "Distributed
  * expert parallelism", "Grouped expert computation").
