@@ -48,6 +48,25 @@ def parse_args():
     return p.parse_args()
 
 
+def profiled_traffic(kernel_key: str):
+    """DRAM bytes per launch of a kernel from the ncu summary in profiles/, if it was taken
+    on the current kernel source (the summary records the source's sha256); else None."""
+    import hashlib
+    import re
+
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "grouped_ffn_moe_b200", "csrc", "grouped_ffn.cu")
+    if not os.path.exists(path) or not os.path.exists(src):
+        return None
+    rec = json.load(open(path)).get(kernel_key)
+    if not rec:
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if rec.get("source_sha256") != digest:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -308,7 +327,8 @@ def run_ours(args):
                     "peak": peaks["hbm_gbs"], "unit": "GB/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["peak_source"] = f"{peak_src} (burst)"
-        roof["traffic"] = None
+        roof["traffic"] = (profiled_traffic(f"up_gate/{w.name}") if not w.identity_ffn
+                           else None)
         line = {
             "metric": METRIC, "value": world * w.S / (ms_step / 1e3), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
