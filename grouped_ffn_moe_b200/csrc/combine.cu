@@ -7,13 +7,21 @@
 //
 //   out[t] = bf16( sum_{k ascending} w[t,k] * float(y[row_id_map[t*K+k]]) )
 //
-// One warp per token. Each lane owns U 16-byte vectors (8 bf16) per pass and keeps their
-// fp32 sums in registers; the K source rows of a pass are loaded four slots at a time so
-// that several loads are in flight before the fixed-order FMAs consume them.
+// One warp per token. Each lane owns U = 4 16-byte vectors (8 bf16 each) per pass and keeps
+// their fp32 sums in registers; the K source rows of a pass are loaded four slots at a time
+// (16 loads in flight per lane) before the fixed-order FMAs consume them.
 #include <algorithm>
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "ptx.cuh"
+
+#ifndef MOE_COMBINE_U
+#define MOE_COMBINE_U 4      // 16-byte vectors per lane per pass
+#endif
+#ifndef MOE_COMBINE_SLOTS
+#define MOE_COMBINE_SLOTS 4  // route slots whose loads are issued together
+#endif
 
 namespace moe {
 namespace {
@@ -40,14 +48,15 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float (&acc)[8]) {
   return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
-template <int U>
+template <int U, int kSlots>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y,
                                                       const int32_t* __restrict__ row_id_map,
                                                       const float* __restrict__ route_w, int64_t S,
                                                       int64_t nvec, int32_t K,
                                                       uint4* __restrict__ out) {
-  constexpr int kSlots = 4;  // slots loaded together
   const int lane = threadIdx.x & 31;
+  griddep_wait();  // y and row_id_map come from earlier kernels in the stream
+  griddep_launch_dependents();
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        t < S; t += nwarps) {
@@ -104,9 +113,11 @@ moe_status launch_combine(const void* y, const int32_t* row_id_map, const float*
                           int64_t S, int64_t H, int32_t K, void* out, cudaStream_t stream) {
   const int64_t nvec = H / 8;
   const int64_t blocks = std::min<int64_t>(ceil_div(S, 8), static_cast<int64_t>(num_sms()) * 8);
-  combine_kernel<2><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      static_cast<const uint4*>(y), row_id_map, route_w, S, nvec, K, static_cast<uint4*>(out));
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  const cudaError_t err = launch_dependent(
+      combine_kernel<MOE_COMBINE_U, MOE_COMBINE_SLOTS>, dim3(static_cast<unsigned>(blocks)),
+      dim3(256), 0, stream, static_cast<const uint4*>(y), row_id_map, route_w, S, nvec, K,
+      static_cast<uint4*>(out));
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace moe

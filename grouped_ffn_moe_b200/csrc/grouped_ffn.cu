@@ -187,6 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(s_tmem, kTmemCols);
     tmem_relinquish();
   }
+  // everything above overlaps the previous kernel's tail (programmatic dependent launch);
+  // cu_seqlens and the activations come from earlier kernels in the stream
+  griddep_wait();
+  griddep_launch_dependents();
   // cu_seqlens, clamped to [0, M] so that no row outside [0, M) is ever addressed
   for (int e = tid; e <= E; e += kThreads) {
     int64_t v = args.cu[e];
@@ -522,8 +526,9 @@ moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const voi
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
                     static_cast<int32_t>(H), static_cast<int32_t>(Hp), wait_budget_ns()};
-    grouped_ffn_kernel<kSwiGLU><<<grid, kThreads, Cfg<kSwiGLU>::kSmemBytes, stream>>>(m_wg, m_wu,
-                                                                                    m_x, a);
+    if (launch_dependent(grouped_ffn_kernel<kSwiGLU>, dim3(grid), dim3(kThreads),
+                         Cfg<kSwiGLU>::kSmemBytes, stream, m_wg, m_wu, m_x, a) != cudaSuccess)
+      return MOE_ERR_CUDA;
   } else {
     CUtensorMap m_wd;
     RowMaps m_h;
@@ -534,12 +539,12 @@ moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const voi
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
                     static_cast<int32_t>(Hp), static_cast<int32_t>(H), wait_budget_ns()};
-    if (pair)
-      grouped_ffn_kernel<kPair><<<grid, kThreads, Cfg<kPair>::kSmemBytes, stream>>>(m_wd, m_wd,
-                                                                                     m_h, a);
-    else
-      grouped_ffn_kernel<kSingle><<<grid, kThreads, Cfg<kSingle>::kSmemBytes, stream>>>(
-          m_wd, m_wd, m_h, a);
+    const cudaError_t err =
+        pair ? launch_dependent(grouped_ffn_kernel<kPair>, dim3(grid), dim3(kThreads),
+                                Cfg<kPair>::kSmemBytes, stream, m_wd, m_wd, m_h, a)
+             : launch_dependent(grouped_ffn_kernel<kSingle>, dim3(grid), dim3(kThreads),
+                                Cfg<kSingle>::kSmemBytes, stream, m_wd, m_wd, m_h, a);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -2,6 +2,8 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <utility>
+
 #include <cuda_runtime.h>
 
 #include "moe_b200.h"
@@ -19,6 +21,31 @@ inline int64_t permute_num_chunks(int64_t F) { return ceil_div(F, kChunk); }
 
 // Number of SMs of the current device (cached per device).
 int num_sms();
+
+// Launch `kernel` as a programmatic dependent launch: it may be scheduled while the previous
+// kernel in the stream finishes, and waits for it (griddepcontrol.wait) before touching data
+// that kernel produces. Falls back to an ordinary launch if the attribute is refused.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (err != cudaSuccess) {
+    (void)cudaGetLastError();
+    cfg.numAttrs = 0;
+    err = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  }
+  return err;
+}
 
 moe_status launch_permute(const void* x, const int32_t* topk_ids, int64_t S, int64_t H, int32_t K,
                           int32_t E, void* x_perm, int32_t* counts, int32_t* cu_seqlens,

@@ -6,16 +6,25 @@
 // reverses them). The order inside an expert is the flat slot order f = t*K + k, which
 // makes the permutation a stable counting sort and the output independent of scheduling.
 //
-// Four launches, no host synchronisation, no atomics on data:
-//   route_hist  per 512-slot chunk (one warp), per-expert counts via __match_any_sync
-//   route_scan  per expert (one warp), exclusive scan over chunks -> chunk bases + counts
-//   route_rank  exclusive scan of counts -> cu_seqlens (+ max count, maxvio); every warp
-//               replays its chunk with per-expert cursors -> row_id_map, perm_src
-//   permute_rows one warp per token: read the row once (16-byte vectors), write K copies
+// Two launches, no host synchronisation, no atomics on data. The metadata kernel is one
+// cooperative launch (all CTAs co-resident, grid-wide syncs between its phases):
+//   A  per 512-slot chunk (one warp; the chunk's ids prefetched into registers): per-expert
+//      counts with __match_any_sync
+//   B  per expert (one warp): exclusive scan over chunks -> chunk bases, counts
+//   C  exclusive scan of counts -> cu_seqlens (+ max count, maxvio); every warp replays its
+//      chunk with per-expert cursors -> row_id_map, perm_src
+// then permute_rows (one warp per token: the row is read once in 16-byte vectors and written
+// to its K rows) runs as a programmatic dependent launch. The metadata phases also exist as
+// three ordinary launches ("staged", MOE_PERMUTE_KERNEL=staged); both give identical results.
+#include <cooperative_groups.h>
+
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace moe {
 namespace {
@@ -193,6 +202,8 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint4* __restri
                                                            const int32_t* __restrict__ row_id_map,
                                                            uint4* __restrict__ x_perm) {
   const int lane = threadIdx.x & 31;
+  griddep_wait();  // row_id_map comes from the metadata kernel
+  griddep_launch_dependents();
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        t < S; t += nwarps) {
@@ -236,6 +247,180 @@ __global__ void maxvio_kernel(const int32_t* __restrict__ counts, int32_t E, int
   }
 }
 
+// ----------------------------------------------------------------------------- fused kernel
+
+struct PermuteArgs {
+  const int32_t* ids;
+  int64_t S, F, nchunk;
+  int32_t K, E;
+  int32_t* chunk_counts;
+  int32_t* counts;
+  int32_t* cu_seqlens;
+  int32_t* row_id_map;
+  int32_t* perm_src;
+  double* maxvio;
+  int32_t* max_count;
+  int32_t* d_status;
+};
+
+__device__ __forceinline__ void load_chunk_ids(const PermuteArgs& a, int64_t c, int lane,
+                                               int32_t (&idr)[kChunk / 32]) {
+#pragma unroll
+  for (int j = 0; j < kChunk / 32; ++j) {
+    const int64_t f = c * kChunk + j * 32 + lane;
+    idr[j] = f < a.F ? __ldg(a.ids + f) : -1;
+  }
+}
+
+__global__ void __launch_bounds__(256) permute_fused_kernel(const PermuteArgs a) {
+  namespace cg = cooperative_groups;
+  cg::grid_group grid = cg::this_grid();
+  extern __shared__ __align__(128) uint8_t fsmem[];
+  int32_t* s_tab = reinterpret_cast<int32_t*>(fsmem);  // [8][E]
+  int32_t* s_cu = s_tab + kWarpsPerTile * a.E;         // [E+1]
+  __shared__ int32_t s_tmp[16];
+  __shared__ int32_t s_max;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = a.E;
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * kWarpsPerTile;
+
+  griddep_wait();  // the routing table may come from the previous kernel in the stream
+
+  // A: chunk histograms -> chunk_counts[e][c]
+  for (int64_t cb = static_cast<int64_t>(blockIdx.x) * kWarpsPerTile; cb < a.nchunk; cb += wstride) {
+    int32_t* hist = s_tab + warp * E;
+    for (int i = lane; i < E; i += 32) hist[i] = 0;
+    __syncwarp();
+    const int64_t c = cb + warp;
+    if (c < a.nchunk) {
+      int32_t idr[kChunk / 32];
+      load_chunk_ids(a, c, lane, idr);
+      bool bad = false;
+#pragma unroll
+      for (int j = 0; j < kChunk / 32; ++j) {
+        const int64_t f = c * kChunk + j * 32 + lane;
+        const int32_t e = idr[j];
+        const bool ok = f < a.F && e >= 0 && e < E;
+        bad |= (f < a.F) && !ok;
+        const unsigned peers = __match_any_sync(kFull, ok ? e : -1);
+        if (ok && lane == __ffs(peers) - 1) hist[e] += __popc(peers);
+        __syncwarp();
+      }
+      if (__any_sync(kFull, bad) && lane == 0) flag_status(a.d_status, MOE_ERR_BAD_ROUTING);
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < kWarpsPerTile * E; j += blockDim.x) {
+      const int e = j / kWarpsPerTile, w = j % kWarpsPerTile;
+      if (cb + w < a.nchunk)
+        a.chunk_counts[static_cast<int64_t>(e) * a.nchunk + cb + w] = s_tab[w * E + e];
+    }
+    __syncthreads();
+  }
+  grid.sync();
+
+  // B: per-expert exclusive scan over chunks
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * kWarpsPerTile + warp; e < E; e += wstride) {
+    int32_t* row = a.chunk_counts + e * a.nchunk;
+    int32_t carry = 0;
+    for (int64_t base = 0; base < a.nchunk; base += 32) {
+      const int64_t i = base + lane;
+      const int32_t v = (i < a.nchunk) ? row[i] : 0;
+      int32_t incl = v;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int32_t n = __shfl_up_sync(kFull, incl, d);
+        if (lane >= d) incl += n;
+      }
+      if (i < a.nchunk) row[i] = carry + incl - v;
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) a.counts[e] = carry;
+  }
+  grid.sync();
+
+  // C: cu_seqlens, maxvio; stable ranks
+  block_scan_counts(a.counts, E, s_cu, s_tmp, &s_max);
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) a.cu_seqlens[e] = s_cu[e];
+    if (threadIdx.x == 0) {
+      if (a.max_count != nullptr) *a.max_count = s_max;
+      if (a.maxvio != nullptr) *a.maxvio = maxvio_expr(s_max, E, a.S, a.K);
+    }
+  }
+  for (int64_t cb = static_cast<int64_t>(blockIdx.x) * kWarpsPerTile; cb < a.nchunk; cb += wstride) {
+    for (int j = threadIdx.x; j < kWarpsPerTile * E; j += blockDim.x) {
+      const int e = j / kWarpsPerTile, w = j % kWarpsPerTile;
+      if (cb + w < a.nchunk)
+        s_tab[w * E + e] = s_cu[e] + a.chunk_counts[static_cast<int64_t>(e) * a.nchunk + cb + w];
+    }
+    __syncthreads();
+    const int64_t c = cb + warp;
+    if (c < a.nchunk) {
+      int32_t* cur = s_tab + warp * E;
+      int32_t idr[kChunk / 32];
+      load_chunk_ids(a, c, lane, idr);
+#pragma unroll
+      for (int j = 0; j < kChunk / 32; ++j) {
+        const int64_t f = c * kChunk + j * 32 + lane;
+        const int32_t e = idr[j];
+        const bool ok = f < a.F && e >= 0 && e < E;
+        const unsigned peers = __match_any_sync(kFull, ok ? e : -1);
+        int32_t row = -1;
+        if (ok) row = cur[e] + __popc(peers & ((1u << lane) - 1u));
+        __syncwarp();
+        if (ok && lane == __ffs(peers) - 1) cur[e] += __popc(peers);
+        __syncwarp();
+        if (f < a.F) {
+          a.row_id_map[f] = row;
+          if (a.perm_src != nullptr && ok) a.perm_src[row] = static_cast<int32_t>(f);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  // rows are copied by permute_rows_kernel, launched right after as a dependent grid
+  griddep_launch_dependents();
+}
+
+size_t fused_smem_bytes(int32_t E) {
+  return sizeof(int32_t) * (static_cast<size_t>(kWarpsPerTile) * E + E + 1);
+}
+
+// Co-resident CTAs per SM of the fused kernel at the largest shared-memory size (cached).
+int fused_blocks_per_sm() {
+  static std::once_flag once;
+  static int blocks = 0;
+  std::call_once(once, [] {
+    const size_t smem = fused_smem_bytes(MOE_MAX_EXPERTS);
+    if (cudaFuncSetAttribute(permute_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, permute_fused_kernel, 256, smem) ==
+        cudaSuccess)
+      blocks = n;
+  });
+  return blocks;
+}
+
+bool use_staged_permute() {
+  static const bool staged = [] {
+    const char* s = std::getenv("MOE_PERMUTE_KERNEL");
+    return s != nullptr && std::strcmp(s, "staged") == 0;
+  }();
+  return staged;
+}
+
+// Row copy as a programmatic dependent launch of the metadata kernel before it.
+cudaError_t launch_rows(const void* x, int64_t S, int64_t H, int32_t K, const int32_t* row_id_map,
+                        void* x_perm, cudaStream_t stream) {
+  const int64_t nvec = H / 8;
+  const int64_t blocks = std::min<int64_t>(ceil_div(S, 8), static_cast<int64_t>(num_sms()) * 8);
+  return launch_dependent(permute_rows_kernel<4>, dim3(static_cast<unsigned>(blocks)), dim3(256),
+                          0, stream, static_cast<const uint4*>(x), S, nvec, K, row_id_map,
+                          static_cast<uint4*>(x_perm));
+}
+
 }  // namespace
 
 moe_status launch_permute(const void* x, const int32_t* topk_ids, int64_t S, int64_t H, int32_t K,
@@ -246,10 +431,36 @@ moe_status launch_permute(const void* x, const int32_t* topk_ids, int64_t S, int
   const int64_t F = S * K;
   const int64_t nchunk = permute_num_chunks(F);
   const int64_t tiles = ceil_div(nchunk, kWarpsPerTile);
+  const int per_sm = use_staged_permute() ? 0 : fused_blocks_per_sm();
+  if (per_sm > 0) {
+    const int64_t want = std::max<int64_t>({tiles, ceil_div(E, kWarpsPerTile), 1});
+    const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(per_sm) * num_sms()));
+    PermuteArgs pa{topk_ids, S, F, nchunk, K, E, chunk_counts, counts, cu_seqlens, row_id_map,
+                   perm_src, maxvio, max_count, d_status};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = fused_smem_bytes(E);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, permute_fused_kernel, pa) != cudaSuccess) {
+      (void)cudaGetLastError();  // refused as a dependent launch: cooperative only
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, permute_fused_kernel, pa) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if (x_perm != nullptr && launch_rows(x, S, H, K, row_id_map, x_perm, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
+  // staged: three ordinary launches (E <= 1024: at most 32 KB and 37 KB of shared memory)
   const size_t hist_smem = sizeof(int32_t) * kWarpsPerTile * E;
   const size_t rank_smem = sizeof(int32_t) * (E + 1 + kWarpsPerTile * E);
-  // E <= 1024: at most 32 KB (hist) and 37 KB (rank), under the 48 KB default limit.
-
   route_hist_kernel<<<static_cast<unsigned>(tiles), 256, hist_smem, stream>>>(
       topk_ids, F, E, nchunk, chunk_counts, d_status);
   route_scan_kernel<<<static_cast<unsigned>(ceil_div(E, 8)), 256, 0, stream>>>(chunk_counts,
@@ -257,12 +468,8 @@ moe_status launch_permute(const void* x, const int32_t* topk_ids, int64_t S, int
   route_rank_kernel<<<static_cast<unsigned>(tiles), 256, rank_smem, stream>>>(
       topk_ids, F, S, K, E, nchunk, chunk_counts, counts, cu_seqlens, row_id_map, perm_src,
       maxvio, max_count);
-  if (x_perm != nullptr) {
-    const int64_t nvec = H / 8;
-    const int64_t blocks = std::min<int64_t>(ceil_div(S, 8), static_cast<int64_t>(num_sms()) * 8);
-    permute_rows_kernel<4><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        static_cast<const uint4*>(x), S, nvec, K, row_id_map, static_cast<uint4*>(x_perm));
-  }
+  if (x_perm != nullptr && launch_rows(x, S, H, K, row_id_map, x_perm, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

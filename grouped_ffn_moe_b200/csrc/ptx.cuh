@@ -116,6 +116,19 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   return p;
 }
 
+// ----------------------------------------------------------------------------- dependent launch
+
+// Wait until the grids this one depends on (programmatic dependent launch) have completed
+// and their memory is visible; a no-op for a normally launched grid.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the dependent grid to be scheduled (it still waits in griddep_wait for this grid).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------------------- tcgen05
 
 // Whole warp. Writes the TMEM base address of `ncols` columns to *dst (shared).

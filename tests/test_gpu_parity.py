@@ -385,3 +385,35 @@ def test_down_kernel_variants_agree(cuda_device, tmp_path):
                        timeout=600)
         outs[mode] = torch.load(path)
     assert torch.equal(outs["pair"], outs["single"])
+
+
+def test_permute_variants_agree(cuda_device, tmp_path):
+    """The fused cooperative permutation (default) and the four-launch staged one
+    (MOE_PERMUTE_KERNEL=staged) give bit-identical metadata and rows."""
+    import subprocess
+    import sys
+
+    script = (
+        "import sys, torch, synth, grouped_ffn_moe_b200 as moe\n"
+        "w = synth.WORKLOADS['permute_combine_S4096_mv20']\n"
+        "inp = synth.make_layer_inputs(w, device='cuda:0')\n"
+        "buf = moe.LayerBuffers.allocate(w.S, w.H, 0, w.E, w.K, torch.device('cuda:0'),"
+        " with_ffn=False)\n"
+        "moe.moe_layer_forward(inp['x'], inp['topk_ids'], inp['route_w'], None, None, None, buf)\n"
+        "torch.cuda.synchronize()\n"
+        "assert int(buf.d_status.item()) == 0\n"
+        "torch.save({k: getattr(buf, k).cpu() for k in ('x_perm', 'counts', 'cu_seqlens',"
+        " 'row_id_map', 'perm_src', 'maxvio', 'max_count', 'out')}, sys.argv[1])\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    outs = {}
+    for mode in ("fused", "staged"):
+        env = dict(os.environ, MOE_PERMUTE_KERNEL=mode, PYTHONPATH=root)
+        path = str(tmp_path / f"p_{mode}.pt")
+        subprocess.run([sys.executable, "-c", script, path], check=True, env=env, cwd=root,
+                       timeout=600)
+        outs[mode] = torch.load(path)
+    for k, v in outs["fused"].items():
+        a, b = v, outs["staged"][k]
+        if a.dtype == torch.bfloat16:
+            a, b = a.view(torch.int16), b.view(torch.int16)
+        assert torch.equal(a, b), k
