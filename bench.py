@@ -67,6 +67,23 @@ def profiled_traffic(kernel_key: str):
     return rec.get("dram_bytes_per_launch")
 
 
+def reduce_step_time(ms_local: float, world: int, device=None) -> float:
+    """Step time of the whole job: the maximum over ranks (replicas run in lock step)."""
+    if world <= 1:
+        return ms_local
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([ms_local], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_step: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batch (weak scaling)."""
+    return world * tokens_per_rank / (ms_step / 1e3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -236,11 +253,7 @@ def run_ours(args):
         dist.barrier()
     t1 = time.time()
     step_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    ms_step = sum(step_ms) / len(step_ms)
-    if world > 1:
-        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = reduce_step_time(sum(step_ms) / len(step_ms), world, dev)
 
     # stage breakdown (separate loop: events between the stages of every step)
     sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
@@ -291,12 +304,8 @@ def run_ours(args):
             b.record()
             e_ms.append((a, b))
         torch.cuda.synchronize()
-        e2e_ms = sum(a.elapsed_time(b) for a, b in e_ms) / len(e_ms)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * w.S / (e2e_ms / 1e3), "unit": UNIT,
+        e2e_ms = reduce_step_time(sum(a.elapsed_time(b) for a, b in e_ms) / len(e_ms), world, dev)
+        e2e = {"value": job_throughput(w.S, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": hx.numel() * 2 + hids.numel() * 4 + hw.numel() * 4,
                "d2h_bytes_per_step": hout.numel() * 2, "ms_per_step": e2e_ms}
         if not torch.equal(hout.to(dev), buf.out):
@@ -341,7 +350,7 @@ def run_ours(args):
         roof["traffic"] = (profiled_traffic(f"up_gate/{w.name}") if not w.identity_ffn
                            else None)
         line = {
-            "metric": METRIC, "value": world * w.S / (ms_step / 1e3), "unit": UNIT,
+            "metric": METRIC, "value": job_throughput(w.S, world, ms_step), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded SplitMix64/Box-Muller inputs, random-init expert weights)",

@@ -57,6 +57,9 @@ constexpr int kThreads = 64 + kEpiThreads;     // TMA warp, MMA warp, epilogue w
 constexpr int kOutChunk = 32;                  // tokens per epilogue chunk
 constexpr int kOutBytes = kOutChunk * kBM * 2;  // 8 KB staging buffer per group
 constexpr uint32_t kTmemCols = 512;
+// After a time-out, waits for this CTA's own copies and MMAs to land use this fixed bound
+// (not the caller's budget, which may be tiny), so that nothing is in flight at exit.
+constexpr uint64_t kDrainBudgetNs = 200000000ull;
 constexpr uint32_t kAccCols = 256;
 
 // Kernel modes.
@@ -283,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         volatile int dummy = 0;
         for (int s = 0; s < C::kStages; ++s)
           if (issued_mask & (1u << s))
-            mbar_wait_bounded(&full[s], (issued_phase >> s) & 1u, &dummy, args.budget_ns);
+            mbar_wait_bounded(&full[s], (issued_phase >> s) & 1u, &dummy, kDrainBudgetNs);
       }
     }
   } else if (warp == 1) {
@@ -338,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*s_abort && issued_any) {
         umma_commit(drain);
         volatile int dummy = 0;
-        mbar_wait_bounded(drain, 0, &dummy, args.budget_ns);
+        mbar_wait_bounded(drain, 0, &dummy, kDrainBudgetNs);
       }
     }
   } else {

@@ -417,3 +417,36 @@ def test_permute_variants_agree(cuda_device, tmp_path):
         if a.dtype == torch.bfloat16:
             a, b = a.view(torch.int16), b.view(torch.int16)
         assert torch.equal(a, b), k
+
+
+def test_device_wait_timeout_reports_status_and_keeps_context(cuda_device, tmp_path):
+    """Failure detection without a fault: with a 1 ns wait budget every pipeline wait of the
+    grouped FFN runs out; the kernels record MOE_ERR_DEVICE_TIMEOUT in d_status, drain their
+    own copies and MMAs, free TMEM and return, and the CUDA context stays usable."""
+    import subprocess
+    import sys
+
+    script = (
+        "import torch, synth, grouped_ffn_moe_b200 as moe\n"
+        "w = synth.WORKLOADS['tiny']\n"
+        "inp = synth.make_layer_inputs(w, device='cuda:0')\n"
+        "buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, torch.device('cuda:0'))\n"
+        "moe.moe_layer_forward(inp['x'], inp['topk_ids'], inp['route_w'], inp['w_gate'],"
+        " inp['w_up'], inp['w_down'], buf)\n"
+        "torch.cuda.synchronize()\n"
+        "st = int(buf.d_status.item())\n"
+        "assert st & moe.MOE_ERR_DEVICE_TIMEOUT, st\n"
+        "z = torch.arange(1000, device='cuda:0').sum().item()\n"
+        "assert z == 499500\n"
+        "print('timeout status', st)\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, PYTHONPATH=root, MOE_WAIT_BUDGET_NS="1")
+    r = subprocess.run([sys.executable, "-c", script], env=env, cwd=root, timeout=600,
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "timeout status" in r.stdout
+    # this process (normal budget) still runs the layer correctly
+    w = synth.WORKLOADS["tiny"]
+    inp = layer_inputs(w, cuda_device)
+    buf = run_layer(inp, w, cuda_device)
+    assert int(buf.d_status.item()) == 0
