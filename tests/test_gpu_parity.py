@@ -450,3 +450,33 @@ def test_device_wait_timeout_reports_status_and_keeps_context(cuda_device, tmp_p
     inp = layer_inputs(w, cuda_device)
     buf = run_layer(inp, w, cuda_device)
     assert int(buf.d_status.item()) == 0
+
+
+def test_swiglu_kernel_variants_agree(cuda_device, tmp_path):
+    """The one-CTA SwiGLU kernel (default) and the CTA-pair kernel (MOE_SWIGLU_KERNEL=pair,
+    tcgen05 cta_group::2) give bit-identical h (and therefore y and out)."""
+    import subprocess
+    import sys
+
+    script = (
+        "import sys, torch, synth, grouped_ffn_moe_b200 as moe\n"
+        "w = synth.WORKLOADS[sys.argv[2]]\n"
+        "inp = synth.make_layer_inputs(w, device='cuda:0')\n"
+        "buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, torch.device('cuda:0'))\n"
+        "moe.moe_layer_forward(inp['x'], inp['topk_ids'], inp['route_w'], inp['w_gate'],"
+        " inp['w_up'], inp['w_down'], buf)\n"
+        "torch.cuda.synchronize()\n"
+        "assert int(buf.d_status.item()) == 0\n"
+        "torch.save({k: getattr(buf, k).cpu() for k in ('h', 'y', 'out')}, sys.argv[1])\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for wl in ("tiny", "medium"):
+        outs = {}
+        for mode in ("pair", "single"):
+            env = dict(os.environ, MOE_SWIGLU_KERNEL=mode, PYTHONPATH=root)
+            path = str(tmp_path / f"s_{wl}_{mode}.pt")
+            subprocess.run([sys.executable, "-c", script, path, wl], check=True, env=env,
+                           cwd=root, timeout=600)
+            outs[mode] = torch.load(path)
+        for k in outs["pair"]:
+            assert torch.equal(outs["pair"][k].view(torch.int16),
+                               outs["single"][k].view(torch.int16)), (wl, k)
