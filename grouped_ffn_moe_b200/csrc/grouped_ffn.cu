@@ -46,9 +46,11 @@ namespace {
 constexpr int kBM = 128;                       // output features per unit (UMMA M)
 constexpr int kBK = 64;                        // reduction elements per stage (128 bytes)
 constexpr int kNMax = 256;                     // tokens per unit (UMMA N max)
+#ifndef MOE_SWIGLU_NMAX
+#define MOE_SWIGLU_NMAX 256                    // tokens per SwiGLU unit (128: two TMEM stages)
+#endif
 constexpr int kABytes = kBM * kBK * 2;         // 16 KB: [2 halves][64 k][64 f], one TMA box
 constexpr int kAHalfBytes = 64 * kBK * 2;      // 8 KB: one 64-feature half (UMMA LBO)
-constexpr int kBBytes = kNMax * kBK * 2;       // 32 KB
 constexpr int kRowBytes = kBK * 2;             // one token row of a B stage (128 bytes)
 constexpr int kNumBoxHeights = 5;              // token boxes of 256, 128, 64, 32, 16 rows
 constexpr int kEpiGroups = 2;                  // epilogue warp groups, alternating chunks
@@ -72,10 +74,13 @@ enum Mode : int { kSwiGLU = 0, kSingle = 1, kPair = 2 };
 template <int kMode>
 struct Cfg {
   static constexpr int kNumA = kMode == kSingle ? 1 : 2;
-  static constexpr int kStages = kNumA == 2 ? 3 : 4;
-  static constexpr int kAccStages = kMode == kSingle ? 2 : 1;
+  static constexpr int kNMaxMode = kMode == kSwiGLU ? MOE_SWIGLU_NMAX : kNMax;
+  // accumulator stages: two when they fit in TMEM (kSingle; kSwiGLU with N <= 128)
+  static constexpr int kAccStages = (kMode == kSingle || kNMaxMode <= 128) ? 2 : 1;
+  static constexpr int kUpOff = kAccStages == 2 ? kNMaxMode : 256;  // up accumulator column
   static constexpr int kFeatPerUnit = kMode == kPair ? 2 * kBM : kBM;
-  static constexpr int kStageBytes = kNumA * kABytes + kBBytes;
+  static constexpr int kStageBytes = kNumA * kABytes + kNMaxMode * kBK * 2;
+  static constexpr int kStages = (192 * 1024) / kStageBytes;
   static constexpr int kPipeBytes = kStages * kStageBytes;
   static constexpr int kOffOut = kPipeBytes;
   static constexpr int kOffCu = kOffOut + kEpiGroups * kOutBytes;
@@ -113,6 +118,7 @@ struct Unit {
 
 // Unit u -> (expert, feature block, token rows). s_ustart[e] is the first unit of expert e;
 // a feature block is 128 features (256 in kPair mode).
+template <int kNMaxU = kNMax>
 __device__ __forceinline__ Unit decode_unit(int u, const int32_t* s_ustart, const int32_t* s_cu,
                                             int E) {
   int lo = 0, hi = E - 1;
@@ -124,7 +130,7 @@ __device__ __forceinline__ Unit decode_unit(int u, const int32_t* s_ustart, cons
   U.e = lo;
   const int local = u - s_ustart[lo];
   const int cnt = s_cu[lo + 1] - s_cu[lo];
-  const int ntc = (cnt + kNMax - 1) / kNMax;
+  const int ntc = (cnt + kNMaxU - 1) / kNMaxU;
   U.ntc = ntc;
   U.fb = local / ntc;
   const int tc = local - U.fb * ntc;
@@ -208,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int local = 0;
     for (int e = beg; e < end; ++e) {
       const int cnt = s_cu[e + 1] - s_cu[e];
-      const int units = cnt > 0 ? ((cnt + kNMax - 1) / kNMax) * nfb : 0;
+      const int units = cnt > 0 ? ((cnt + C::kNMaxMode - 1) / C::kNMaxMode) * nfb : 0;
       s_ustart[e] = units;
       local += units;
     }
@@ -247,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
       for (int u = blockIdx.x; u < total_units && !*s_abort; u += gridDim.x) {
-        const Unit U = decode_unit(u, s_ustart, s_cu, E);
+        const Unit U = decode_unit<C::kNMaxMode>(u, s_ustart, s_cu, E);
         if (U.nrows <= 0) continue;
         const int n = (U.nrows + 15) & ~15;
         const uint32_t bytes = C::kNumA * kABytes + n * kRowBytes;
@@ -298,14 +304,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t aphase = 0;
       bool issued_any = false;
       for (int u = blockIdx.x; u < total_units && !*s_abort; u += gridDim.x) {
-        const Unit U = decode_unit(u, s_ustart, s_cu, E);
+        const Unit U = decode_unit<C::kNMaxMode>(u, s_ustart, s_cu, E);
         if (U.nrows <= 0) continue;
         const uint32_t n = static_cast<uint32_t>((U.nrows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_m128_amn_bk(n);
         if (!mbar_wait_bounded(&tempty[astage], aphase ^ 1u, s_abort, args.budget_ns)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + (kDual ? 0u : astage * kAccCols);
-        const uint32_t d1 = tmem_base + kAccCols;
+        const uint32_t d0 = tmem_base + astage * kAccCols;  // astage is 0 with one stage
+        const uint32_t d1 = d0 + (kMode == kSwiGLU ? C::kUpOff : kAccCols);
         bool ok = true;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait_bounded(&full[stage], phase, s_abort, args.budget_ns)) {
@@ -358,14 +364,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int astage = 0;
     uint32_t aphase = 0;
     for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
-      const Unit U = decode_unit(u, s_ustart, s_cu, E);
+      const Unit U = decode_unit<C::kNMaxMode>(u, s_ustart, s_cu, E);
       if (U.nrows <= 0) continue;
       mbar_wait_bounded(&tfull[astage], aphase, s_abort, args.budget_ns);
       named_bar_sync(bar_all, kEpiThreads);  // every epilogue warp takes the same decision
       if (*s_abort) break;
       tc_fence_after();
       const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (kDual ? 0u : astage * kAccCols);
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + astage * kAccCols;
       for (int c = grp * kOutChunk; c < U.nrows; c += kEpiGroups * kOutChunk) {
         // kPair: two 128-feature halves per chunk; otherwise one
         for (int half = 0; half < (kMode == kPair ? 2 : 1); ++half) {
@@ -376,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_32x32b_x32(tbase + half * kAccCols + c, r0);
           if (kMode == kSwiGLU) {
             uint32_t r1[32];
-            tmem_ld_32x32b_x32(tbase + kAccCols + c, r1);
+            tmem_ld_32x32b_x32(tbase + C::kUpOff + c, r1);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
