@@ -30,8 +30,9 @@ MOE_ERR_DEVICE_TIMEOUT = 8
 MOE_MAX_EXPERTS = 1024
 
 # Kernels launched by one call of each entry point (permute with a row copy).
-LAUNCHES = {"moe_permute": 4, "moe_grouped_ffn": 2, "moe_grouped_ffn_up_gate": 1,
-            "moe_grouped_ffn_down": 1, "moe_unpermute_combine": 1, "moe_maxvio": 1}
+LAUNCHES = {"moe_permute": 2, "moe_grouped_ffn": 2, "moe_grouped_ffn_up_gate": 1,
+            "moe_grouped_ffn_down": 1, "moe_unpermute_combine": 1, "moe_maxvio": 1,
+            "moe_combine_backward": 1, "moe_permute_backward": 1}
 
 
 class MoeError(RuntimeError):
@@ -69,6 +70,10 @@ def lib() -> ctypes.CDLL:
         L.moe_grouped_ffn_down.argtypes = [p, p, p, i64, i64, i64, i32, p, p, p]
         L.moe_unpermute_combine.restype = i32
         L.moe_unpermute_combine.argtypes = [p, p, p, i64, i64, i32, p, p]
+        L.moe_combine_backward.restype = i32
+        L.moe_combine_backward.argtypes = [p, p, p, p, i64, i64, i32, p, p, p]
+        L.moe_permute_backward.restype = i32
+        L.moe_permute_backward.argtypes = [p, p, i64, i64, i32, p, p]
         L.moe_maxvio.restype = i32
         L.moe_maxvio.argtypes = [p, i32, i64, i32, p, p, p]
         _lib = L
@@ -256,6 +261,40 @@ def moe_unpermute_combine(y, row_id_map, route_w, out, stream=None):
     st = lib().moe_unpermute_combine(_ptr(y), _ptr(row_id_map), _ptr(route_w), S, H, K, _ptr(out),
                                      _stream(stream, dev))
     _check("moe_unpermute_combine", st)
+
+
+def moe_combine_backward(grad_out, y, row_id_map, route_w, grad_y, grad_w=None, stream=None):
+    """grad_y[r(t,k)] = w[t,k] * grad_out[t]; grad_w[t,k] = <grad_out[t], y[r(t,k)]>."""
+    S, K = route_w.shape
+    dev = grad_out.device
+    _need(grad_out, "grad_out", torch.bfloat16, dev, 2)
+    _need(y, "y", torch.bfloat16, dev, 2)
+    _need(grad_y, "grad_y", torch.bfloat16, dev, 2)
+    _need(row_id_map, "row_id_map", torch.int32, dev)
+    _need(route_w, "route_w", torch.float32, dev, 2)
+    _need(grad_w, "grad_w", torch.float32, dev)
+    H = grad_out.shape[1]
+    if tuple(grad_out.shape) != (S, H) or grad_y.shape[1] != H or row_id_map.numel() != S * K:
+        raise ValueError("grad_out [S,H], grad_y [M,H], row_id_map [S*K] expected")
+    if grad_w is not None and (y is None or grad_w.numel() != S * K):
+        raise ValueError("grad_w needs y and S*K entries")
+    st = lib().moe_combine_backward(_ptr(grad_out), _ptr(y), _ptr(row_id_map), _ptr(route_w), S,
+                                    H, K, _ptr(grad_y), _ptr(grad_w), _stream(stream, dev))
+    _check("moe_combine_backward", st)
+
+
+def moe_permute_backward(grad_x_perm, row_id_map, grad_x, K, stream=None):
+    """grad_x[t] = sum_k grad_x_perm[row_id_map[t*K+k]] (dispatch backward)."""
+    S, H = grad_x.shape
+    dev = grad_x.device
+    _need(grad_x_perm, "grad_x_perm", torch.bfloat16, dev, 2)
+    _need(grad_x, "grad_x", torch.bfloat16, dev, 2)
+    _need(row_id_map, "row_id_map", torch.int32, dev)
+    if grad_x_perm.shape[1] != H or row_id_map.numel() != S * K:
+        raise ValueError("grad_x_perm [M,H] and row_id_map [S*K] expected")
+    st = lib().moe_permute_backward(_ptr(grad_x_perm), _ptr(row_id_map), S, H, K, _ptr(grad_x),
+                                    _stream(stream, dev))
+    _check("moe_permute_backward", st)
 
 
 def moe_maxvio(counts, S, K, maxvio, max_count=None, stream=None):

@@ -170,6 +170,34 @@ moe_status moe_unpermute_combine(const void* y, const int32_t* row_id_map, const
                              static_cast<cudaStream_t>(cuda_stream));
 }
 
+moe_status moe_combine_backward(const void* grad_out, const void* y, const int32_t* row_id_map,
+                                const float* route_w, int64_t S, int64_t H, int32_t K,
+                                void* grad_y, float* grad_w, void* cuda_stream) {
+  if (S < 0 || H <= 0 || K < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (H % 8 != 0 || S * K > moe::kMaxRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (S == 0) return MOE_OK;
+  if (!grad_out || !row_id_map || !route_w || !grad_y || (grad_w && !y))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned(grad_out, 16) || !aligned(grad_y, 16) || !aligned(y, 16) ||
+      !aligned(row_id_map, 4) || !aligned(route_w, 4) || !aligned(grad_w, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  return moe::launch_combine_backward(grad_out, grad_w != nullptr ? y : nullptr, row_id_map,
+                                      route_w, S, H, K, grad_y, grad_w,
+                                      static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_permute_backward(const void* grad_x_perm, const int32_t* row_id_map, int64_t S,
+                                int64_t H, int32_t K, void* grad_x, void* cuda_stream) {
+  if (S < 0 || H <= 0 || K < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (H % 8 != 0 || S * K > moe::kMaxRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (S == 0) return MOE_OK;
+  if (!grad_x_perm || !row_id_map || !grad_x) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned(grad_x_perm, 16) || !aligned(grad_x, 16) || !aligned(row_id_map, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  return moe::launch_combine(grad_x_perm, row_id_map, nullptr, S, H, K, grad_x,
+                             static_cast<cudaStream_t>(cuda_stream));
+}
+
 moe_status moe_maxvio(const int32_t* counts, int32_t E, int64_t S, int32_t K, double* maxvio,
                       int32_t* max_count, void* cuda_stream) {
   if (E < 1 || S < 1 || K < 1) return MOE_ERR_INVALID_ARGUMENT;

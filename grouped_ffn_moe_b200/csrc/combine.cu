@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        t < S; t += nwarps) {
     const int32_t my_row = (lane < K) ? row_id_map[t * K + lane] : -1;
-    const float my_w = (lane < K) ? route_w[t * K + lane] : 0.0f;
+    const float my_w = (lane < K) ? (route_w != nullptr ? route_w[t * K + lane] : 1.0f) : 0.0f;
     for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
       float acc[U][8];
 #pragma unroll
@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
             ws[s] = __shfl_sync(kFull, my_w, k & 31);
           } else {
             rows[s] = (k < K) ? row_id_map[t * K + k] : -1;
-            ws[s] = (k < K) ? route_w[t * K + k] : 0.0f;
+            ws[s] = (k < K) ? (route_w != nullptr ? route_w[t * K + k] : 1.0f) : 0.0f;
           }
           if (k >= K) rows[s] = -1;
 #pragma unroll
@@ -107,7 +107,88 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
   }
 }
 
+// w * g rounded once to bf16, as the exact product would be: the fp32 product is taken
+// rounded toward zero and its last bit set when inexact (rounding to odd, Boldo and
+// Melquiond, "Emulation of FMA and correctly rounded sums: proved algorithms using rounding
+// to odd"); with 24 >= 8 + 2 significand bits the bf16 round-to-nearest of that value equals
+// the round-to-nearest of the exact product. The residual fmaf(w, g, -p) is exact.
+__device__ __forceinline__ float mul_round_odd(float w, float g) {
+  const float p = __fmul_rz(w, g);
+  const float e = fmaf(w, g, -p);
+  return (e != 0.0f) ? __uint_as_float(__float_as_uint(p) | 1u) : p;
+}
+
+// Backward of the combine (MoonEP README, "combine bwd": the output gradient goes back to the
+// expert-grouped rows along the saved plan), one warp per token, for each slot k in order:
+//   grad_y[r(t,k)] = bf16(w[t,k] * grad_out[t])   (one rounding of the exact product)
+//   grad_w[t,k]    = <grad_out[t], y[r(t,k)]>  (fp32; per-lane partial sums in vector order,
+//                    then a fixed butterfly reduction: deterministic)
+// The token's gradient row is re-read per slot from L1/L2; HBM traffic stays grad_out once,
+// grad_y and y once each.
+__global__ void __launch_bounds__(256) combine_backward_kernel(
+    const uint4* __restrict__ grad_out, const uint4* __restrict__ y,
+    const int32_t* __restrict__ row_id_map, const float* __restrict__ route_w, int64_t S,
+    int64_t nvec, int32_t K, uint4* __restrict__ grad_y, float* __restrict__ grad_w) {
+  const int lane = threadIdx.x & 31;
+  griddep_wait();
+  griddep_launch_dependents();
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       t < S; t += nwarps) {
+    const uint4* g = grad_out + t * nvec;
+    for (int k = 0; k < K; ++k) {
+      const int32_t r = row_id_map[t * K + k];
+      const float wk = route_w[t * K + k];
+      float dot = 0.0f;
+      if (r >= 0) {
+        uint4* dst = grad_y + static_cast<int64_t>(r) * nvec;
+        const uint4* src = y != nullptr ? y + static_cast<int64_t>(r) * nvec : nullptr;
+        for (int64_t v = lane; v < nvec; v += 32) {
+          const uint4 gv = __ldg(g + v);
+          float gf[8];
+          const uint32_t gu[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            gf[2 * i] = __uint_as_float(gu[i] << 16);
+            gf[2 * i + 1] = __uint_as_float(gu[i] & 0xFFFF0000u);
+          }
+          float sc[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) sc[i] = mul_round_odd(wk, gf[i]);
+          dst[v] = pack_bf16x8(sc);
+          if (src != nullptr) {
+            const uint4 yv = __ldg(src + v);
+            const uint32_t yu[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              dot = fmaf(gf[2 * i], __uint_as_float(yu[i] << 16), dot);
+              dot = fmaf(gf[2 * i + 1], __uint_as_float(yu[i] & 0xFFFF0000u), dot);
+            }
+          }
+        }
+      }
+      if (grad_w != nullptr) {
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) dot += __shfl_xor_sync(kFull, dot, d);
+        if (lane == 0) grad_w[t * K + k] = dot;
+      }
+    }
+  }
+}
+
 }  // namespace
+
+moe_status launch_combine_backward(const void* grad_out, const void* y, const int32_t* row_id_map,
+                                   const float* route_w, int64_t S, int64_t H, int32_t K,
+                                   void* grad_y, float* grad_w, cudaStream_t stream) {
+  const int64_t nvec = H / 8;
+  const int64_t blocks = std::min<int64_t>(ceil_div(S, 8), static_cast<int64_t>(num_sms()) * 8);
+  const cudaError_t err = launch_dependent(
+      combine_backward_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+      static_cast<const uint4*>(grad_out), static_cast<const uint4*>(y), row_id_map, route_w, S,
+      nvec, K, static_cast<uint4*>(grad_y), grad_w);
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
 
 moe_status launch_combine(const void* y, const int32_t* row_id_map, const float* route_w,
                           int64_t S, int64_t H, int32_t K, void* out, cudaStream_t stream) {

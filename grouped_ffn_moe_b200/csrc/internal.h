@@ -56,8 +56,13 @@ moe_status launch_permute(const void* x, const int32_t* topk_ids, int64_t S, int
 moe_status launch_maxvio(const int32_t* counts, int32_t E, int64_t S, int32_t K, double* maxvio,
                          int32_t* max_count, cudaStream_t stream);
 
+// route_w == nullptr: unit weights (the permutation's backward).
 moe_status launch_combine(const void* y, const int32_t* row_id_map, const float* route_w,
                           int64_t S, int64_t H, int32_t K, void* out, cudaStream_t stream);
+
+moe_status launch_combine_backward(const void* grad_out, const void* y, const int32_t* row_id_map,
+                                   const float* route_w, int64_t S, int64_t H, int32_t K,
+                                   void* grad_y, float* grad_w, cudaStream_t stream);
 
 // One pass of the grouped FFN. dual: h = SwiGLU pass (w0 = gate, w1 = up, act = x_perm,
 // out = h); otherwise the down pass (w0 = down, act = h, out = y).

@@ -188,6 +188,30 @@ moe_status moe_unpermute_combine(const void* y, const int32_t* row_id_map, const
                                  int64_t S, int64_t H, int32_t K, void* out, void* cuda_stream);
 
 /*
+ * moe_combine_backward - backward of moe_unpermute_combine (MoonEP README, "combine bwd":
+ * the output gradient is scattered back to the expert-grouped rows by re-dispatching with the
+ * saved plan; "Distributed expert parallelism", lifecycle step 8). For every slot f = t*K+k
+ * with r = row_id_map[f] >= 0:
+ *   grad_y[r]    = bf16(route_w[t,k] * grad_out[t])                 (fp32 product, one rounding)
+ *   grad_w[t,k]  = sum_n grad_out[t,n] * y[r,n]                      (fp32, fixed order)
+ *   grad_out [S, H] bf16; y [M, H] bf16 (the expert outputs of the forward; may be NULL when
+ *   grad_w is NULL); row_id_map [S*K] int32; route_w [S, K] fp32; grad_y [M, H] bf16 out (rows
+ *   no slot maps to are not written); grad_w [S, K] fp32 out, nullable.
+ */
+moe_status moe_combine_backward(const void* grad_out, const void* y, const int32_t* row_id_map,
+                                const float* route_w, int64_t S, int64_t H, int32_t K,
+                                void* grad_y, float* grad_w, void* cuda_stream);
+
+/*
+ * moe_permute_backward - backward of moe_permute's row copy (MoonEP README, "dispatch bwd":
+ * each token's K dispatched gradient copies are summed back to token-major, i.e. a combine):
+ *   grad_x[t] = bf16( sum_{k ascending} grad_x_perm[row_id_map[t*K+k]] )   (fp32 accumulate)
+ *   grad_x_perm [M, H] bf16; row_id_map [S*K] int32; grad_x [S, H] bf16 out.
+ */
+moe_status moe_permute_backward(const void* grad_x_perm, const int32_t* row_id_map, int64_t S,
+                                int64_t H, int32_t K, void* grad_x, void* cuda_stream);
+
+/*
  * moe_maxvio - routing imbalance (MoonEP README, "Performance"):
  *   maxvio = max_e(T_e / T_bar) - 1,  T_e = counts[e],  T_bar = S*K/E,
  * evaluated in IEEE double as ((double)max_count * E) / ((double)S * K) - 1.

@@ -214,6 +214,41 @@ def combine_token(y_rows_bits: np.ndarray, w_row: np.ndarray) -> np.ndarray:
     return f64_to_bf16_bits(acc)
 
 
+# ----------------------------------------------------------------------------- backward
+#
+# MoonEP README, "dispatch bwd" (sum each token's K dispatched gradient copies back to
+# token-major: a combine) and "combine bwd" (scatter the output gradient back to the
+# expert-grouped order by re-dispatching with the saved plan). With the layer's combine
+# out[t] = sum_k w[t,k] * y[r(t,k)], r = row_id_map, the gradients are
+#   grad_y[r(t,k)] = w[t,k] * grad_out[t]          (combine bwd, a weighted re-dispatch)
+#   grad_w[t,k]    = <grad_out[t], y[r(t,k)]>      (route-weight gradient)
+#   grad_x[t]      = sum_k grad_x_perm[r(t,k)]     (dispatch bwd, an unweighted combine)
+
+
+def combine_backward(grad_out_bits: np.ndarray, y_bits: np.ndarray, row_id_map: np.ndarray,
+                     route_w: np.ndarray, S: int, K: int):
+    """Returns (grad_y bits [M,H], grad_w float64 [S,K]); rows that no slot maps to stay 0."""
+    rmap = np.asarray(row_id_map, dtype=np.int64).reshape(S, K)
+    w = np.asarray(route_w, dtype=np.float32).astype(np.float64).reshape(S, K)
+    g = bf16_bits_to_f64(grad_out_bits)
+    M, H = y_bits.shape
+    grad_y = np.zeros((M, H), dtype=np.uint16)
+    grad_w = np.zeros((S, K), dtype=np.float64)
+    for k in range(K):
+        grad_y[rmap[:, k]] = f64_to_bf16_bits(w[:, k:k + 1] * g)
+        grad_w[:, k] = np.sum(g * bf16_bits_to_f64(y_bits[rmap[:, k]]), axis=1)
+    return grad_y, grad_w
+
+
+def permute_backward(grad_x_perm_bits: np.ndarray, row_id_map: np.ndarray, S: int, K: int):
+    """grad_x[t] = bf16(sum over k ascending of grad_x_perm[r(t,k)]), float64 sum."""
+    rmap = np.asarray(row_id_map, dtype=np.int64).reshape(S, K)
+    acc = np.zeros((S, grad_x_perm_bits.shape[1]), dtype=np.float64)
+    for k in range(K):
+        acc += bf16_bits_to_f64(grad_x_perm_bits[rmap[:, k]])
+    return f64_to_bf16_bits(acc)
+
+
 # ----------------------------------------------------------------------------- whole layer
 
 

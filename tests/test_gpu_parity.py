@@ -480,3 +480,78 @@ def test_swiglu_kernel_variants_agree(cuda_device, tmp_path):
         for k in outs["pair"]:
             assert torch.equal(outs["pair"][k].view(torch.int16),
                                outs["single"][k].view(torch.int16)), (wl, k)
+
+
+# ----------------------------------------------------------------------------- backward
+
+@pytest.mark.parametrize("wname,sample", [("medium", None), ("permute_combine_S65536_mv20", 4096)])
+def test_combine_and_permute_backward(cuda_device, wname, sample):
+    """moe_combine_backward (grad_y, grad_w) and moe_permute_backward (grad_x) against the
+    oracle, on the forward's own routing and expert outputs. grad_y is one rounding of the
+    exact product w * g on both sides and must match bit for bit."""
+    w = synth.WORKLOADS[wname]
+    inp = layer_inputs(w, cuda_device)
+    buf = run_layer(inp, w, cuda_device)
+    y = buf.y if buf.y is not None else buf.x_perm
+    M = w.S * w.K
+    g = synth.normal_bf16_into(torch.empty(w.S, w.H, dtype=torch.bfloat16, device=cuda_device),
+                               w.seed, synth.TAG_GRAD)
+    gxp = synth.normal_bf16_into(torch.empty(M, w.H, dtype=torch.bfloat16, device=cuda_device),
+                                 w.seed + 100, synth.TAG_GRAD)
+    grad_y = torch.empty(M, w.H, dtype=torch.bfloat16, device=cuda_device)
+    grad_w = torch.empty(w.S, w.K, dtype=torch.float32, device=cuda_device)
+    grad_x = torch.empty(w.S, w.H, dtype=torch.bfloat16, device=cuda_device)
+    moe.moe_combine_backward(g, y, buf.row_id_map, inp["route_w"], grad_y, grad_w)
+    moe.moe_permute_backward(gxp, buf.row_id_map, grad_x, w.K)
+    torch.cuda.synchronize()
+    rmap = buf.row_id_map.cpu().numpy()
+    rw = inp["route_w"].cpu().numpy()
+    g_bits = bits(g)
+    if sample is None:
+        ref_gy, ref_gw = O.combine_backward(g_bits, bits(y), rmap, rw, w.S, w.K)
+        print(f"[{wname}] grad_y: {assert_close_bf16(bits(grad_y), ref_gy, 'grad_y')}")
+        # one rounding of an exact product on both sides: bit-exact
+        np.testing.assert_array_equal(bits(grad_y), ref_gy)
+        ref_gx = O.permute_backward(bits(gxp), rmap, w.S, w.K)
+        print(f"[{wname}] grad_x: {assert_close_bf16(bits(grad_x), ref_gx, 'grad_x')}")
+    else:
+        toks = np.random.default_rng(2).choice(w.S, sample // w.K, replace=False)
+        slots = (toks[:, None] * w.K + np.arange(w.K)[None, :]).reshape(-1)
+        rows = rmap[slots]
+        ref_rows = O.f64_to_bf16_bits(rw.reshape(-1)[slots, None].astype(np.float64) *
+                                      O.bf16_bits_to_f64(g_bits[slots // w.K]))
+        got_rows = bits(grad_y[torch.as_tensor(rows, device=cuda_device)])
+        print(f"[{wname}] grad_y (sampled): {assert_close_bf16(got_rows, ref_rows, 'grad_y')}")
+        np.testing.assert_array_equal(got_rows, ref_rows)
+        _, ref_gw = O.combine_backward(g_bits, bits(y), rmap, rw, w.S, w.K)
+        gxp_bits = bits(gxp)
+        ref_gx = np.stack([O.combine_token(gxp_bits[rmap[t * w.K:(t + 1) * w.K]],
+                                           np.ones(w.K, np.float32)) for t in toks])
+        got_gx = bits(grad_x[torch.as_tensor(toks, device=cuda_device)])
+        print(f"[{wname}] grad_x (sampled): {assert_close_bf16(got_gx, ref_gx, 'grad_x')}")
+    gw = grad_w.cpu().numpy().astype(np.float64)
+    scale = np.abs(ref_gw).max()
+    err = np.abs(gw - ref_gw).max()
+    print(f"[{wname}] grad_w max |err| / max |ref| = {err / scale:.2e}")
+    assert err <= 1e-4 * scale
+
+
+def test_backward_unit_weight_and_adjoint_exactness(cuda_device):
+    """With unit route weights, grad_y rows are exact copies of grad_out; the permutation's
+    backward of K identical copies is exactly bf16(K * x) (every partial sum is exact)."""
+    S, K, E, H = 1500, 4, 16, 256
+    rng = np.random.default_rng(31)
+    ids = torch.from_numpy(np.stack([rng.permutation(E)[:K] for _ in range(S)]).astype(np.int32))
+    ids = ids.to(cuda_device)
+    x = synth.normal_bf16_into(torch.empty(S, H, dtype=torch.bfloat16, device=cuda_device), 4,
+                               synth.TAG_X)
+    buf = moe.LayerBuffers.allocate(S, H, 0, E, K, cuda_device, with_ffn=False)
+    ones = torch.ones(S, K, dtype=torch.float32, device=cuda_device)
+    moe.moe_layer_forward(x, ids, ones, None, None, None, buf)
+    grad_y = torch.empty(S * K, H, dtype=torch.bfloat16, device=cuda_device)
+    moe.moe_combine_backward(x, None, buf.row_id_map, ones, grad_y)
+    grad_x = torch.empty(S, H, dtype=torch.bfloat16, device=cuda_device)
+    moe.moe_permute_backward(buf.x_perm, buf.row_id_map, grad_x, K)
+    torch.cuda.synchronize()
+    assert torch.equal(grad_y, buf.x_perm)  # w = 1: the backward re-dispatch is the permutation
+    assert torch.equal(grad_x, (x.float() * K).to(torch.bfloat16))

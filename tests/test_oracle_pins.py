@@ -342,3 +342,62 @@ def test_expert_down_rows_against_torch():
     ref = (T(h) @ T(wd)).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
     assert (got == ref).mean() > 0.99
     np.testing.assert_allclose(got, ref, rtol=2.0 ** -7, atol=1e-30)
+
+
+# ----------------------------------------------------------------------------- backward
+
+def _autograd_combine(g, y, rmap, w, S, K):
+    """torch fp64 autograd of out[t] = sum_k w[t,k] * y[rmap[t,k]]."""
+    yt = torch.tensor(y, dtype=torch.float64, requires_grad=True)
+    wt = torch.tensor(w, dtype=torch.float64, requires_grad=True)
+    idx = torch.tensor(rmap.reshape(S, K), dtype=torch.long)
+    out = (wt.unsqueeze(-1) * yt[idx]).sum(dim=1)
+    out.backward(torch.tensor(g, dtype=torch.float64))
+    return yt.grad.numpy(), wt.grad.numpy()
+
+
+def test_combine_backward_against_autograd():
+    rng = np.random.default_rng(21)
+    S, K, E, H = 37, 3, 5, 24
+    ids = rng.integers(0, E, size=(S, K)).astype(np.int32)  # duplicates included
+    counts, cu, rmap, psrc = O.permute_metadata(ids, E)
+    y = O.f64_to_bf16_bits(rng.standard_normal((S * K, H)))
+    g = O.f64_to_bf16_bits(rng.standard_normal((S, H)))
+    w = rng.random((S, K)).astype(np.float32)
+    gy, gw = O.combine_backward(g, y, rmap, w, S, K)
+    ref_gy, ref_gw = _autograd_combine(O.bf16_bits_to_f64(g), O.bf16_bits_to_f64(y), rmap,
+                                       w.astype(np.float64), S, K)
+    # grad_y: every row is hit by exactly one slot, so the gradient is w * g rounded once
+    np.testing.assert_array_equal(gy, O.f64_to_bf16_bits(ref_gy))
+    np.testing.assert_allclose(gw, ref_gw, rtol=1e-12, atol=1e-12)
+
+
+def test_permute_backward_against_autograd():
+    rng = np.random.default_rng(22)
+    S, K, E, H = 29, 4, 6, 16
+    ids = rng.integers(0, E, size=(S, K)).astype(np.int32)
+    counts, cu, rmap, psrc = O.permute_metadata(ids, E)
+    gxp = O.f64_to_bf16_bits(rng.standard_normal((S * K, H)))
+    got = O.permute_backward(gxp, rmap, S, K)
+    xt = torch.zeros((S, H), dtype=torch.float64, requires_grad=True)
+    xperm = xt[torch.tensor(psrc.astype(np.int64) // K)]  # the permutation's forward gather
+    xperm.backward(torch.tensor(O.bf16_bits_to_f64(gxp)))
+    np.testing.assert_array_equal(got, O.f64_to_bf16_bits(xt.grad.numpy()))
+
+
+def test_backward_adjoint_identity():
+    """<grad_out, combine(y)> = <grad_y, y> (before rounding): the combine's backward is its
+    transpose; checked with exact small-integer data where every value is representable."""
+    rng = np.random.default_rng(23)
+    S, K, E, H = 11, 2, 3, 8
+    ids = rng.integers(0, E, size=(S, K)).astype(np.int32)
+    counts, cu, rmap, psrc = O.permute_metadata(ids, E)
+    y = O.f64_to_bf16_bits(rng.integers(-4, 5, size=(S * K, H)).astype(np.float64))
+    g = O.f64_to_bf16_bits(rng.integers(-4, 5, size=(S, H)).astype(np.float64))
+    w = (rng.integers(1, 5, size=(S, K)) / 4.0).astype(np.float32)
+    out = O.bf16_bits_to_f64(O.unpermute_combine(y, rmap, w, S, K))
+    gy, gw = O.combine_backward(g, y, rmap, w, S, K)
+    lhs = np.sum(O.bf16_bits_to_f64(g) * out)
+    rhs = np.sum(O.bf16_bits_to_f64(gy) * O.bf16_bits_to_f64(y))
+    assert lhs == rhs
+    assert np.sum(gw * w) == lhs  # sum_k w * <g, y_k> = <g, out>
