@@ -249,6 +249,98 @@ def permute_backward(grad_x_perm_bits: np.ndarray, row_id_map: np.ndarray, S: in
     return f64_to_bf16_bits(acc)
 
 
+# ----------------------------------------------------------------------------- expert FFN backward
+#
+# The pages give the forward of an expert, Down(SwiGLU(Up x, Gate x)) ("Mixture of Kittens"
+# digest, Step 1), and say that training keeps one fp32 gradient buffer per projection laid
+# out like the weights (MoonEP README, "Gradient buffers"). The backward below is the chain
+# rule of that forward. Readings: the training forward stores the gate and up
+# pre-activations g = x Wg and u = x Wu as bf16 tensors (like every stored activation),
+# and the backward starts from those; grad_h is not stored (it stays exact up to d_g and
+# d_u); d_g, d_u and grad_x_perm are stored bf16; weight gradients are stored fp32.
+# With s = sigmoid(g): silu(g) = g s, silu'(g) = s (1 + g (1 - s)), and for h = silu(g) u
+#   grad_h = grad_y Wd^T
+#   d_u    = grad_h * silu(g)              d_g = grad_h * u * silu'(g)
+#   grad_x = d_g Wg^T + d_u Wu^T
+#   dWg    = x^T d_g    dWu = x^T d_u    dWd = h^T grad_y     (sums over the expert's rows)
+
+
+def expert_preact_rows(x_rows_bits: np.ndarray, w_gate_e: np.ndarray, w_up_e: np.ndarray):
+    """Pre-activations saved by the training forward: (bf16(x Wg), bf16(x Wu)) bits."""
+    x = bf16_bits_to_f64(x_rows_bits)
+    return (f64_to_bf16_bits(x @ bf16_bits_to_f64(w_gate_e)),
+            f64_to_bf16_bits(x @ bf16_bits_to_f64(w_up_e)))
+
+
+def swiglu_backward(grad_h: np.ndarray, g_bits: np.ndarray, u_bits: np.ndarray):
+    """(d_g bits, d_u bits) of h = silu(g) * u for a float64 grad_h and saved bf16 g, u."""
+    g = bf16_bits_to_f64(g_bits)
+    u = bf16_bits_to_f64(u_bits)
+    s = 1.0 / (1.0 + np.exp(-g))
+    return (f64_to_bf16_bits(grad_h * u * (s * (1.0 + g * (1.0 - s)))),
+            f64_to_bf16_bits(grad_h * (g * s)))
+
+
+def expert_ffn_backward_rows(x_rows_bits, g_bits, u_bits, h_bits, grad_y_bits, w_gate_e, w_up_e,
+                             w_down_e):
+    """Backward of one expert on a block of rows.
+
+    Returns (d_g bits, d_u bits, grad_x bits, dWg, dWu, dWd), the weight gradients as
+    float64 sums of the block's rows (the caller stores them as fp32).
+    """
+    gy = bf16_bits_to_f64(grad_y_bits)
+    grad_h = gy @ bf16_bits_to_f64(w_down_e).T
+    dg_bits, du_bits = swiglu_backward(grad_h, g_bits, u_bits)
+    dg, du = bf16_bits_to_f64(dg_bits), bf16_bits_to_f64(du_bits)
+    grad_x = f64_to_bf16_bits(dg @ bf16_bits_to_f64(w_gate_e).T + du @ bf16_bits_to_f64(w_up_e).T)
+    x = bf16_bits_to_f64(x_rows_bits)
+    h = bf16_bits_to_f64(h_bits)
+    return dg_bits, du_bits, grad_x, x.T @ dg, x.T @ du, h.T @ gy
+
+
+def grouped_ffn_preact(x_perm_bits: np.ndarray, cu_seqlens: np.ndarray, get_weights, Hp: int):
+    """Saved pre-activations of the whole grouped FFN: (g bits [M,H'], u bits [M,H'])."""
+    M = x_perm_bits.shape[0]
+    g = np.zeros((M, Hp), dtype=np.uint16)
+    u = np.zeros((M, Hp), dtype=np.uint16)
+    for e in range(len(cu_seqlens) - 1):
+        r0, r1 = int(cu_seqlens[e]), int(cu_seqlens[e + 1])
+        if r1 > r0:
+            wg, wu, _ = get_weights(e)
+            g[r0:r1], u[r0:r1] = expert_preact_rows(x_perm_bits[r0:r1], wg, wu)
+    return g, u
+
+
+def grouped_ffn_backward(x_perm_bits, g_bits, u_bits, h_bits, grad_y_bits, cu_seqlens,
+                         get_weights, dw_prior=None):
+    """Backward of the grouped FFN over expert-contiguous rows.
+
+    Returns a dict: d_g, d_u, grad_x_perm (bf16 bits) and dWg [E,H,H'], dWu [E,H,H'],
+    dWd [E,H',H] as float32. An expert with no rows gets zero weight gradients. With
+    dw_prior = (Pg, Pu, Pd) the weight gradients are added to those fp32 buffers, each
+    element rounded once (fp64 sum of the prior value and the exact product sum).
+    """
+    M, H = x_perm_bits.shape
+    Hp = g_bits.shape[1]
+    E = len(cu_seqlens) - 1
+    out = dict(d_g=np.zeros((M, Hp), np.uint16), d_u=np.zeros((M, Hp), np.uint16),
+               grad_x_perm=np.zeros((M, H), np.uint16))
+    dw = [np.zeros((E, H, Hp)), np.zeros((E, H, Hp)), np.zeros((E, Hp, H))]
+    if dw_prior is not None:
+        dw = [np.asarray(p, dtype=np.float32).astype(np.float64) for p in dw_prior]
+    for e in range(E):
+        r0, r1 = int(cu_seqlens[e]), int(cu_seqlens[e + 1])
+        if r1 == r0:
+            continue
+        res = expert_ffn_backward_rows(x_perm_bits[r0:r1], g_bits[r0:r1], u_bits[r0:r1],
+                                       h_bits[r0:r1], grad_y_bits[r0:r1], *get_weights(e))
+        out["d_g"][r0:r1], out["d_u"][r0:r1], out["grad_x_perm"][r0:r1] = res[:3]
+        for i in range(3):
+            dw[i][e] += res[3 + i]
+    out["dWg"], out["dWu"], out["dWd"] = (d.astype(np.float32) for d in dw)
+    return out
+
+
 # ----------------------------------------------------------------------------- whole layer
 
 

@@ -401,3 +401,144 @@ def test_backward_adjoint_identity():
     rhs = np.sum(O.bf16_bits_to_f64(gy) * O.bf16_bits_to_f64(y))
     assert lhs == rhs
     assert np.sum(gw * w) == lhs  # sum_k w * <g, y_k> = <g, out>
+
+
+# ----------------------------------------------------------------------------- FFN backward
+
+
+def _ffn_bwd_case(seed, rows_per_expert, H, Hp):
+    rng = np.random.default_rng(seed)
+    E = len(rows_per_expert)
+    cu = np.concatenate([[0], np.cumsum(rows_per_expert)]).astype(np.int32)
+    M = int(cu[-1])
+    x = O.f64_to_bf16_bits(rng.standard_normal((M, H)))
+    wg = O.f64_to_bf16_bits(rng.standard_normal((E, H, Hp)) / math.sqrt(H))
+    wu = O.f64_to_bf16_bits(rng.standard_normal((E, H, Hp)) / math.sqrt(H))
+    wd = O.f64_to_bf16_bits(rng.standard_normal((E, Hp, H)) / math.sqrt(Hp))
+    get = _weights_getter(wg, wu, wd)
+    h, _ = O.grouped_ffn(x, cu, get, Hp)
+    g, u = O.grouped_ffn_preact(x, cu, get, Hp)
+    gy = O.f64_to_bf16_bits(rng.standard_normal((M, H)))
+    return dict(E=E, cu=cu, M=M, x=x, wg=wg, wu=wu, wd=wd, get=get, h=h, g=g, u=u, gy=gy)
+
+
+def _within_one_bf16_step(got_bits, ref_f64, min_exact=0.99):
+    ref_bits = O.f64_to_bf16_bits(ref_f64)
+    diff = np.abs(got_bits.astype(np.int32) - ref_bits.astype(np.int32))
+    assert diff.max() <= 1, diff.max()
+    assert np.mean(diff == 0) >= min_exact
+
+
+def test_ffn_backward_against_autograd():
+    """Each stage of the oracle's backward against torch autograd (float64) of the forward
+    definition, evaluated at the oracle's own stored tensors."""
+    c = _ffn_bwd_case(41, [5, 0, 9, 3], H=16, Hp=24)
+    res = O.grouped_ffn_backward(c["x"], c["g"], c["u"], c["h"], c["gy"], c["cu"], c["get"])
+    f = lambda b: torch.tensor(O.bf16_bits_to_f64(b))
+    for e in range(c["E"]):
+        r0, r1 = int(c["cu"][e]), int(c["cu"][e + 1])
+        if r1 == r0:
+            for k in ("dWg", "dWu", "dWd"):
+                assert not res[k][e].any()
+            continue
+        sl = slice(r0, r1)
+        # down projection: grad_h and dWd
+        hl = f(c["h"][sl]).requires_grad_()
+        wd = f(c["wd"][e]).requires_grad_()
+        (hl @ wd).backward(f(c["gy"][sl]))
+        np.testing.assert_allclose(res["dWd"][e], wd.grad.numpy().astype(np.float32), rtol=1e-6,
+                                   atol=1e-6)
+        # SwiGLU at the saved pre-activations
+        G = f(c["g"][sl]).requires_grad_()
+        U = f(c["u"][sl]).requires_grad_()
+        (torch.nn.functional.silu(G) * U).backward(hl.grad)
+        _within_one_bf16_step(res["d_g"][sl], G.grad.numpy())
+        _within_one_bf16_step(res["d_u"][sl], U.grad.numpy())
+        # up and gate projections, driven by the stored d_g, d_u
+        xl = f(c["x"][sl]).requires_grad_()
+        wg = f(c["wg"][e]).requires_grad_()
+        wu = f(c["wu"][e]).requires_grad_()
+        torch.autograd.backward([xl @ wg, xl @ wu], [f(res["d_g"][sl]), f(res["d_u"][sl])])
+        _within_one_bf16_step(res["grad_x_perm"][sl], xl.grad.numpy())
+        np.testing.assert_allclose(res["dWg"][e], wg.grad.numpy().astype(np.float32), rtol=1e-6,
+                                   atol=1e-6)
+        np.testing.assert_allclose(res["dWu"][e], wu.grad.numpy().astype(np.float32), rtol=1e-6,
+                                   atol=1e-6)
+
+
+def test_ffn_backward_brute_force_rows():
+    """Row by row with scalar loops: each row uses its own expert's weights, weight
+    gradients are sums of per-row outer products, empty experts get zeros."""
+    c = _ffn_bwd_case(42, [2, 3, 0, 1], H=4, Hp=6)
+    res = O.grouped_ffn_backward(c["x"], c["g"], c["u"], c["h"], c["gy"], c["cu"], c["get"])
+    f = O.bf16_bits_to_f64
+    H, Hp, E = 4, 6, c["E"]
+    dWg = np.zeros((E, H, Hp)); dWu = np.zeros((E, H, Hp)); dWd = np.zeros((E, Hp, H))
+    for r in range(c["M"]):
+        e = int(np.searchsorted(c["cu"], r, side="right") - 1)
+        wg, wu, wd = f(c["wg"][e]), f(c["wu"][e]), f(c["wd"][e])
+        gy, x, hrow = f(c["gy"][r]), f(c["x"][r]), f(c["h"][r])
+        dg = np.zeros(Hp); du = np.zeros(Hp)
+        for j in range(Hp):
+            gh = sum(gy[n] * wd[j, n] for n in range(H))
+            gj, uj = f(c["g"][r, j]), f(c["u"][r, j])
+            sg = 1.0 / (1.0 + math.exp(-gj))
+            dg[j] = f(O.f64_to_bf16_bits(np.array(gh * uj * sg * (1 + gj * (1 - sg)))))
+            du[j] = f(O.f64_to_bf16_bits(np.array(gh * gj * sg)))
+        assert np.array_equal(f(res["d_g"][r]), dg) and np.array_equal(f(res["d_u"][r]), du)
+        gx = [sum(dg[j] * wg[n, j] + du[j] * wu[n, j] for j in range(Hp)) for n in range(H)]
+        assert np.array_equal(res["grad_x_perm"][r], O.f64_to_bf16_bits(np.array(gx)))
+        dWg[e] += np.outer(x, dg); dWu[e] += np.outer(x, du); dWd[e] += np.outer(hrow, gy)
+    np.testing.assert_allclose(res["dWg"], dWg.astype(np.float32), rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(res["dWu"], dWu.astype(np.float32), rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(res["dWd"], dWd.astype(np.float32), rtol=1e-6, atol=1e-7)
+    assert not res["dWg"][2].any() and not res["dWd"][2].any()
+
+
+def test_swiglu_backward_closed_forms():
+    gh = np.array([[1.5, -2.0, 0.75, 3.0]])
+    u_bits = O.f64_to_bf16_bits(np.array([[2.0, 0.5, -1.25, 4.0]]))
+    u = O.bf16_bits_to_f64(u_bits)
+    # g = 0: silu(0) = 0, silu'(0) = 1/2
+    dg, du = O.swiglu_backward(gh, O.f64_to_bf16_bits(np.zeros((1, 4))), u_bits)
+    assert not O.bf16_bits_to_f64(du).any()
+    np.testing.assert_array_equal(dg, O.f64_to_bf16_bits(gh * u / 2))
+    # g = +-128: sigmoid is 1 or below bf16's range, so silu(g) -> g or 0 and
+    # silu'(g) -> 1 or 0 after rounding (compared as values: the zeros carry a sign)
+    for gv, sil, dsil in ((128.0, 128.0, 1.0), (-128.0, 0.0, 0.0)):
+        dg, du = O.swiglu_backward(gh, O.f64_to_bf16_bits(np.full((1, 4), gv)), u_bits)
+        np.testing.assert_array_equal(O.bf16_bits_to_f64(du), gh * sil)
+        np.testing.assert_array_equal(O.bf16_bits_to_f64(dg),
+                                      O.bf16_bits_to_f64(O.f64_to_bf16_bits(gh * u * dsil)))
+    # silu'(g) against a central difference of silu
+    gs = O.f64_to_bf16_bits(np.linspace(-6, 6, 25)[None, :])
+    gv = O.bf16_bits_to_f64(gs)
+    ones = O.f64_to_bf16_bits(np.ones_like(gv))
+    dg, _ = O.swiglu_backward(np.ones_like(gv), gs, ones)
+    eps = 1e-6
+    fd = (O.silu(gv + eps) - O.silu(gv - eps)) / (2 * eps)
+    _within_one_bf16_step(dg, fd, min_exact=0.9)
+
+
+def test_ffn_backward_accumulates_into_fp32_buffers():
+    c = _ffn_bwd_case(43, [4, 2], H=8, Hp=8)
+    fresh = O.grouped_ffn_backward(c["x"], c["g"], c["u"], c["h"], c["gy"], c["cu"], c["get"])
+    rng = np.random.default_rng(44)
+    prior = [rng.standard_normal(fresh[k].shape).astype(np.float32) for k in ("dWg", "dWu", "dWd")]
+    acc = O.grouped_ffn_backward(c["x"], c["g"], c["u"], c["h"], c["gy"], c["cu"], c["get"],
+                                 dw_prior=prior)
+    for k, p in zip(("dWg", "dWu", "dWd"), prior):
+        e1 = fresh[k].astype(np.float64)  # fresh is already fp32-rounded: allow that step
+        np.testing.assert_allclose(acc[k], p.astype(np.float64) + e1, rtol=1e-6, atol=1e-6)
+    np.testing.assert_array_equal(acc["d_g"], fresh["d_g"])
+
+
+def test_preactivations_against_torch():
+    rng = np.random.default_rng(45)
+    x = O.f64_to_bf16_bits(rng.standard_normal((7, 16)))
+    wg = O.f64_to_bf16_bits(rng.standard_normal((16, 8)))
+    wu = O.f64_to_bf16_bits(rng.standard_normal((16, 8)))
+    g, u = O.expert_preact_rows(x, wg, wu)
+    tx = torch_bf16_of(x).double()
+    np.testing.assert_array_equal(g, bits_of((tx @ torch_bf16_of(wg).double()).to(torch.bfloat16)))
+    np.testing.assert_array_equal(u, bits_of((tx @ torch_bf16_of(wu).double()).to(torch.bfloat16)))
