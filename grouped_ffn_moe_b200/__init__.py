@@ -32,7 +32,10 @@ MOE_MAX_EXPERTS = 1024
 # Kernels launched by one call of each entry point (permute with a row copy).
 LAUNCHES = {"moe_permute": 2, "moe_grouped_ffn": 2, "moe_grouped_ffn_up_gate": 1,
             "moe_grouped_ffn_down": 1, "moe_unpermute_combine": 1, "moe_maxvio": 1,
-            "moe_combine_backward": 1, "moe_permute_backward": 1}
+            "moe_combine_backward": 1, "moe_permute_backward": 1,
+            "moe_grouped_ffn_up_gate_train": 1, "moe_grouped_ffn_down_backward": 1,
+            "moe_grouped_ffn_up_gate_backward": 1, "moe_grouped_ffn_weight_grad": 1,
+            "moe_grouped_ffn_backward": 3}
 
 
 class MoeError(RuntimeError):
@@ -76,6 +79,18 @@ def lib() -> ctypes.CDLL:
         L.moe_permute_backward.argtypes = [p, p, i64, i64, i32, p, p]
         L.moe_maxvio.restype = i32
         L.moe_maxvio.argtypes = [p, i32, i64, i32, p, p, p]
+        L.moe_grouped_ffn_up_gate_train.restype = i32
+        L.moe_grouped_ffn_up_gate_train.argtypes = [p, p, p, p, i64, i64, i64, i32, p, p, p, p, p]
+        L.moe_grouped_ffn_down_backward.restype = i32
+        L.moe_grouped_ffn_down_backward.argtypes = [p, p, p, p, p, i64, i64, i64, i32, p, p, p, p]
+        L.moe_grouped_ffn_up_gate_backward.restype = i32
+        L.moe_grouped_ffn_up_gate_backward.argtypes = [p, p, p, p, p, i64, i64, i64, i32, p, p, p]
+        L.moe_grouped_ffn_weight_grad.restype = i32
+        L.moe_grouped_ffn_weight_grad.argtypes = [p, p, p, p, p, p, i64, i64, i64, i32, p, p, p,
+                                                  i32, p, p]
+        L.moe_grouped_ffn_backward.restype = i32
+        L.moe_grouped_ffn_backward.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i32, p, p,
+                                               p, p, p, p, p, i32, p, p]
         _lib = L
     return _lib
 
@@ -247,6 +262,124 @@ def moe_grouped_ffn_down(h_scratch, w_down, cu_seqlens, y, d_status=None, stream
     _check("moe_grouped_ffn_down", st)
 
 
+def moe_grouped_ffn_up_gate_train(x_perm, w_gate, w_up, cu_seqlens, h_scratch, gate_pre, up_pre,
+                                  d_status=None, stream=None):
+    """moe_grouped_ffn_up_gate that also stores the bf16 pre-activations x W_gate, x W_up."""
+    M, H, Hp, E, dev = _ffn_check(x_perm, w_gate, w_up, None, cu_seqlens, h_scratch, None, d_status)
+    for t, n in ((gate_pre, "gate_pre"), (up_pre, "up_pre")):
+        _need(t, n, torch.bfloat16, dev, 2)
+        if tuple(t.shape) != (M, Hp):
+            raise ValueError(f"{n} must be [M,H'] = {(M, Hp)}")
+    st = lib().moe_grouped_ffn_up_gate_train(_ptr(x_perm), _ptr(w_gate), _ptr(w_up),
+                                             _ptr(cu_seqlens), M, H, Hp, E, _ptr(h_scratch),
+                                             _ptr(gate_pre), _ptr(up_pre), _ptr(d_status),
+                                             _stream(stream, dev))
+    _check("moe_grouped_ffn_up_gate_train", st)
+
+
+def _bwd_shapes(grad_y, gate_pre, cu_seqlens):
+    M, H = grad_y.shape
+    Hp = gate_pre.shape[1]
+    return M, H, Hp, cu_seqlens.numel() - 1, grad_y.device
+
+
+def _need_shape(t, name, shape, dtype, dev):
+    _need(t, name, dtype, dev)
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def moe_grouped_ffn_down_backward(grad_y, w_down, gate_pre, up_pre, cu_seqlens, d_gate, d_up,
+                                  d_status=None, stream=None):
+    """d_gate, d_up = SwiGLU backward of grad_y W_down[e]^T at the saved pre-activations."""
+    M, H, Hp, E, dev = _bwd_shapes(grad_y, gate_pre, cu_seqlens)
+    _need_shape(grad_y, "grad_y", (M, H), torch.bfloat16, dev)
+    _need_shape(w_down, "w_down", (E, Hp, H), torch.bfloat16, dev)
+    for t, n in ((gate_pre, "gate_pre"), (up_pre, "up_pre"), (d_gate, "d_gate"), (d_up, "d_up")):
+        _need_shape(t, n, (M, Hp), torch.bfloat16, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(d_status, "d_status", torch.int32, dev)
+    st = lib().moe_grouped_ffn_down_backward(_ptr(grad_y), _ptr(w_down), _ptr(gate_pre),
+                                             _ptr(up_pre), _ptr(cu_seqlens), M, H, Hp, E,
+                                             _ptr(d_gate), _ptr(d_up), _ptr(d_status),
+                                             _stream(stream, dev))
+    _check("moe_grouped_ffn_down_backward", st)
+
+
+def moe_grouped_ffn_up_gate_backward(d_gate, d_up, w_gate, w_up, cu_seqlens, grad_x_perm,
+                                     d_status=None, stream=None):
+    """grad_x_perm = d_gate W_gate[e]^T + d_up W_up[e]^T."""
+    M, H = grad_x_perm.shape
+    Hp = d_gate.shape[1]
+    E = cu_seqlens.numel() - 1
+    dev = grad_x_perm.device
+    _need_shape(grad_x_perm, "grad_x_perm", (M, H), torch.bfloat16, dev)
+    for t, n in ((d_gate, "d_gate"), (d_up, "d_up")):
+        _need_shape(t, n, (M, Hp), torch.bfloat16, dev)
+    for t, n in ((w_gate, "w_gate"), (w_up, "w_up")):
+        _need_shape(t, n, (E, H, Hp), torch.bfloat16, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(d_status, "d_status", torch.int32, dev)
+    st = lib().moe_grouped_ffn_up_gate_backward(_ptr(d_gate), _ptr(d_up), _ptr(w_gate),
+                                                _ptr(w_up), _ptr(cu_seqlens), M, H, Hp, E,
+                                                _ptr(grad_x_perm), _ptr(d_status),
+                                                _stream(stream, dev))
+    _check("moe_grouped_ffn_up_gate_backward", st)
+
+
+def moe_grouped_ffn_weight_grad(x_perm, h, d_gate, d_up, grad_y, cu_seqlens, grad_w_gate,
+                                grad_w_up, grad_w_down, accumulate=False, d_status=None,
+                                stream=None):
+    """fp32 weight gradients x^T d_gate, x^T d_up, h^T grad_y per expert (written or added)."""
+    M, H = x_perm.shape
+    Hp = h.shape[1]
+    E = cu_seqlens.numel() - 1
+    dev = x_perm.device
+    _need_shape(x_perm, "x_perm", (M, H), torch.bfloat16, dev)
+    _need_shape(grad_y, "grad_y", (M, H), torch.bfloat16, dev)
+    for t, n in ((h, "h"), (d_gate, "d_gate"), (d_up, "d_up")):
+        _need_shape(t, n, (M, Hp), torch.bfloat16, dev)
+    _need_shape(grad_w_gate, "grad_w_gate", (E, H, Hp), torch.float32, dev)
+    _need_shape(grad_w_up, "grad_w_up", (E, H, Hp), torch.float32, dev)
+    _need_shape(grad_w_down, "grad_w_down", (E, Hp, H), torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(d_status, "d_status", torch.int32, dev)
+    st = lib().moe_grouped_ffn_weight_grad(_ptr(x_perm), _ptr(h), _ptr(d_gate), _ptr(d_up),
+                                           _ptr(grad_y), _ptr(cu_seqlens), M, H, Hp, E,
+                                           _ptr(grad_w_gate), _ptr(grad_w_up), _ptr(grad_w_down),
+                                           1 if accumulate else 0, _ptr(d_status),
+                                           _stream(stream, dev))
+    _check("moe_grouped_ffn_weight_grad", st)
+
+
+def moe_grouped_ffn_backward(x_perm, h, gate_pre, up_pre, w_gate, w_up, w_down, cu_seqlens, grad_y,
+                             d_gate, d_up, grad_x_perm, grad_w_gate, grad_w_up, grad_w_down,
+                             accumulate=False, d_status=None, stream=None):
+    """Backward of the grouped expert FFN (see include/moe_b200.h): d_gate, d_up, grad_x_perm
+    and the fp32 weight gradients, in three launches on one stream."""
+    M, H, Hp, E, dev = _bwd_shapes(grad_y, gate_pre, cu_seqlens)
+    for t, n in ((x_perm, "x_perm"), (grad_y, "grad_y"), (grad_x_perm, "grad_x_perm")):
+        _need_shape(t, n, (M, H), torch.bfloat16, dev)
+    for t, n in ((h, "h"), (gate_pre, "gate_pre"), (up_pre, "up_pre"), (d_gate, "d_gate"),
+                 (d_up, "d_up")):
+        _need_shape(t, n, (M, Hp), torch.bfloat16, dev)
+    for t, n in ((w_gate, "w_gate"), (w_up, "w_up")):
+        _need_shape(t, n, (E, H, Hp), torch.bfloat16, dev)
+    _need_shape(w_down, "w_down", (E, Hp, H), torch.bfloat16, dev)
+    _need_shape(grad_w_gate, "grad_w_gate", (E, H, Hp), torch.float32, dev)
+    _need_shape(grad_w_up, "grad_w_up", (E, H, Hp), torch.float32, dev)
+    _need_shape(grad_w_down, "grad_w_down", (E, Hp, H), torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(d_status, "d_status", torch.int32, dev)
+    st = lib().moe_grouped_ffn_backward(_ptr(x_perm), _ptr(h), _ptr(gate_pre), _ptr(up_pre),
+                                        _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(cu_seqlens),
+                                        M, H, Hp, E, _ptr(grad_y), _ptr(d_gate), _ptr(d_up),
+                                        _ptr(grad_x_perm), _ptr(grad_w_gate), _ptr(grad_w_up),
+                                        _ptr(grad_w_down), 1 if accumulate else 0,
+                                        _ptr(d_status), _stream(stream, dev))
+    _check("moe_grouped_ffn_backward", st)
+
+
 def moe_unpermute_combine(y, row_id_map, route_w, out, stream=None):
     """out[t] = sum_k route_w[t,k] * y[row_id_map[t*K+k]] (see include/moe_b200.h)."""
     S, K = route_w.shape
@@ -324,12 +457,16 @@ class LayerBuffers:
     y: torch.Tensor | None
     out: torch.Tensor
     d_status: torch.Tensor
+    gate_pre: torch.Tensor | None = None  # training: saved bf16 pre-activations [M,H']
+    up_pre: torch.Tensor | None = None
 
     @staticmethod
-    def allocate(S: int, H: int, Hp: int, E: int, K: int, device, with_ffn: bool = True):
+    def allocate(S: int, H: int, Hp: int, E: int, K: int, device, with_ffn: bool = True,
+                 train: bool = False):
         M = S * K
         i32 = dict(dtype=torch.int32, device=device)
         bf = dict(dtype=torch.bfloat16, device=device)
+        train = train and with_ffn
         return LayerBuffers(
             x_perm=torch.empty(M, H, **bf), counts=torch.empty(E, **i32),
             cu_seqlens=torch.empty(E + 1, **i32), row_id_map=torch.empty(M, **i32),
@@ -340,7 +477,9 @@ class LayerBuffers:
                                   device=device),
             h=torch.empty(M, Hp, **bf) if with_ffn else None,
             y=torch.empty(M, H, **bf) if with_ffn else None,
-            out=torch.empty(S, H, **bf), d_status=torch.zeros(1, **i32))
+            out=torch.empty(S, H, **bf), d_status=torch.zeros(1, **i32),
+            gate_pre=torch.empty(M, Hp, **bf) if train else None,
+            up_pre=torch.empty(M, Hp, **bf) if train else None)
 
 
 def moe_layer_forward(x, topk_ids, route_w, w_gate, w_up, w_down, buf: LayerBuffers, stream=None):
@@ -353,8 +492,60 @@ def moe_layer_forward(x, topk_ids, route_w, w_gate, w_up, w_down, buf: LayerBuff
                 buf.perm_src, buf.maxvio, buf.max_count, buf.workspace, buf.d_status, stream)
     y = buf.x_perm
     if w_gate is not None:
-        moe_grouped_ffn(buf.x_perm, w_gate, w_up, w_down, buf.cu_seqlens, buf.h, buf.y,
-                        buf.d_status, stream)
+        if buf.gate_pre is not None:
+            # training: keep the pre-activations for the backward
+            moe_grouped_ffn_up_gate_train(buf.x_perm, w_gate, w_up, buf.cu_seqlens, buf.h,
+                                          buf.gate_pre, buf.up_pre, buf.d_status, stream)
+            moe_grouped_ffn_down(buf.h, w_down, buf.cu_seqlens, buf.y, buf.d_status, stream)
+        else:
+            moe_grouped_ffn(buf.x_perm, w_gate, w_up, w_down, buf.cu_seqlens, buf.h, buf.y,
+                            buf.d_status, stream)
         y = buf.y
     moe_unpermute_combine(y, buf.row_id_map, route_w, buf.out, stream)
     return buf.out
+
+
+@dataclass
+class LayerGrads:
+    """Gradient buffers of one layer's backward (fp32 weight gradients laid out like the
+    weights, as the training buffers of the MoonEP README's "Gradient buffers")."""
+
+    grad_y: torch.Tensor        # [M,H] bf16
+    d_gate: torch.Tensor        # [M,H'] bf16
+    d_up: torch.Tensor          # [M,H'] bf16
+    grad_x_perm: torch.Tensor   # [M,H] bf16
+    grad_x: torch.Tensor        # [S,H] bf16
+    grad_route_w: torch.Tensor  # [S,K] fp32
+    grad_w_gate: torch.Tensor   # [E,H,H'] fp32
+    grad_w_up: torch.Tensor     # [E,H,H'] fp32
+    grad_w_down: torch.Tensor   # [E,H',H] fp32
+
+    @staticmethod
+    def allocate(S: int, H: int, Hp: int, E: int, K: int, device):
+        M = S * K
+        bf = dict(dtype=torch.bfloat16, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
+        return LayerGrads(
+            grad_y=torch.empty(M, H, **bf), d_gate=torch.empty(M, Hp, **bf),
+            d_up=torch.empty(M, Hp, **bf), grad_x_perm=torch.empty(M, H, **bf),
+            grad_x=torch.empty(S, H, **bf), grad_route_w=torch.empty(S, K, **f32),
+            grad_w_gate=torch.empty(E, H, Hp, **f32), grad_w_up=torch.empty(E, H, Hp, **f32),
+            grad_w_down=torch.empty(E, Hp, H, **f32))
+
+
+def moe_layer_backward(grad_out, route_w, w_gate, w_up, w_down, buf: LayerBuffers,
+                       grads: LayerGrads, accumulate: bool = False, stream=None):
+    """Backward of moe_layer_forward (run with LayerBuffers.allocate(..., train=True)):
+    combine backward -> grouped FFN backward -> permutation backward, on one stream.
+    Fills grads (grad_x, grad_route_w and the weight gradients, written or added into)."""
+    if buf.gate_pre is None:
+        raise ValueError("the forward did not keep pre-activations: allocate with train=True")
+    K = route_w.shape[1]
+    moe_combine_backward(grad_out, buf.y, buf.row_id_map, route_w, grads.grad_y,
+                         grads.grad_route_w, stream)
+    moe_grouped_ffn_backward(buf.x_perm, buf.h, buf.gate_pre, buf.up_pre, w_gate, w_up, w_down,
+                             buf.cu_seqlens, grads.grad_y, grads.d_gate, grads.d_up,
+                             grads.grad_x_perm, grads.grad_w_gate, grads.grad_w_up,
+                             grads.grad_w_down, accumulate, buf.d_status, stream)
+    moe_permute_backward(grads.grad_x_perm, buf.row_id_map, grads.grad_x, K, stream)
+    return grads

@@ -51,7 +51,7 @@ const char* moe_status_string(moe_status s) {
   }
 }
 
-int32_t moe_abi_version(void) { return (1 << 16) | 0; }
+int32_t moe_abi_version(void) { return (1 << 16) | 1; }
 
 size_t moe_permute_workspace_bytes(int64_t S, int32_t K, int32_t E) {
   if (S <= 0 || K <= 0 || E <= 0) return 0;
@@ -123,7 +123,7 @@ moe_status moe_grouped_ffn_up_gate(const void* x_perm, const void* w_gate, const
     return MOE_ERR_INVALID_ARGUMENT;
   if (M == 0) return MOE_OK;
   return moe::launch_ffn_pass(true, x_perm, w_gate, w_up, cu_seqlens, M, H, Hp, E, h_scratch,
-                              d_status, static_cast<cudaStream_t>(cuda_stream));
+                              nullptr, nullptr, d_status, static_cast<cudaStream_t>(cuda_stream));
 }
 
 moe_status moe_grouped_ffn_down(const void* h_scratch, const void* w_down,
@@ -136,7 +136,7 @@ moe_status moe_grouped_ffn_down(const void* h_scratch, const void* w_down,
     return MOE_ERR_INVALID_ARGUMENT;
   if (M == 0) return MOE_OK;
   return moe::launch_ffn_pass(false, h_scratch, w_down, nullptr, cu_seqlens, M, H, Hp, E, y,
-                              d_status, static_cast<cudaStream_t>(cuda_stream));
+                              nullptr, nullptr, d_status, static_cast<cudaStream_t>(cuda_stream));
 }
 
 moe_status moe_grouped_ffn(const void* x_perm, const void* w_gate, const void* w_up,
@@ -156,6 +156,119 @@ moe_status moe_grouped_ffn(const void* x_perm, const void* w_gate, const void* w
   if (s1 != MOE_OK) return s1;
   return moe_grouped_ffn_down(h_scratch, w_down, cu_seqlens, M, H, Hp, E, y, d_status,
                               cuda_stream);
+}
+
+moe_status moe_grouped_ffn_up_gate_train(const void* x_perm, const void* w_gate,
+                                         const void* w_up, const int32_t* cu_seqlens, int64_t M,
+                                         int64_t H, int64_t Hp, int32_t E, void* h_scratch,
+                                         void* gate_pre, void* up_pre, int32_t* d_status,
+                                         void* cuda_stream) {
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  if (!ok_ptr16(x_perm) || !ok_ptr16(w_gate) || !ok_ptr16(w_up) || !ok_ptr16(h_scratch) ||
+      !ok_ptr16(gate_pre) || !ok_ptr16(up_pre) || cu_seqlens == nullptr ||
+      !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M == 0) return MOE_OK;
+  return moe::launch_ffn_pass(true, x_perm, w_gate, w_up, cu_seqlens, M, H, Hp, E, h_scratch,
+                              gate_pre, up_pre, d_status, static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_grouped_ffn_down_backward(const void* grad_y, const void* w_down,
+                                         const void* gate_pre, const void* up_pre,
+                                         const int32_t* cu_seqlens, int64_t M, int64_t H,
+                                         int64_t Hp, int32_t E, void* d_gate, void* d_up,
+                                         int32_t* d_status, void* cuda_stream) {
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  if (!ok_ptr16(grad_y) || !ok_ptr16(w_down) || !ok_ptr16(gate_pre) || !ok_ptr16(up_pre) ||
+      !ok_ptr16(d_gate) || !ok_ptr16(d_up) || cu_seqlens == nullptr || !aligned(cu_seqlens, 4) ||
+      !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M == 0) return MOE_OK;
+  return moe::launch_ffn_down_backward(grad_y, w_down, gate_pre, up_pre, cu_seqlens, M, H, Hp, E,
+                                       d_gate, d_up, d_status,
+                                       static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_grouped_ffn_up_gate_backward(const void* d_gate, const void* d_up,
+                                            const void* w_gate, const void* w_up,
+                                            const int32_t* cu_seqlens, int64_t M, int64_t H,
+                                            int64_t Hp, int32_t E, void* grad_x_perm,
+                                            int32_t* d_status, void* cuda_stream) {
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  if (!ok_ptr16(d_gate) || !ok_ptr16(d_up) || !ok_ptr16(w_gate) || !ok_ptr16(w_up) ||
+      !ok_ptr16(grad_x_perm) || cu_seqlens == nullptr || !aligned(cu_seqlens, 4) ||
+      !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M == 0) return MOE_OK;
+  return moe::launch_ffn_up_gate_backward(d_gate, d_up, w_gate, w_up, cu_seqlens, M, H, Hp, E,
+                                          grad_x_perm, d_status,
+                                          static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_grouped_ffn_weight_grad(const void* x_perm, const void* h, const void* d_gate,
+                                       const void* d_up, const void* grad_y,
+                                       const int32_t* cu_seqlens, int64_t M, int64_t H,
+                                       int64_t Hp, int32_t E, float* grad_w_gate,
+                                       float* grad_w_up, float* grad_w_down, int32_t accumulate,
+                                       int32_t* d_status, void* cuda_stream) {
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  if (accumulate != 0 && accumulate != 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (!ok_ptr16(grad_w_gate) || !ok_ptr16(grad_w_up) || !ok_ptr16(grad_w_down) ||
+      cu_seqlens == nullptr || !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  if (M == 0) {
+    // no rows: every expert's gradient is zero
+    if (accumulate) return MOE_OK;
+    const size_t n = static_cast<size_t>(E) * H * Hp * sizeof(float);
+    if (cudaMemsetAsync(grad_w_gate, 0, n, stream) != cudaSuccess ||
+        cudaMemsetAsync(grad_w_up, 0, n, stream) != cudaSuccess ||
+        cudaMemsetAsync(grad_w_down, 0, n, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  if (!ok_ptr16(x_perm) || !ok_ptr16(h) || !ok_ptr16(d_gate) || !ok_ptr16(d_up) ||
+      !ok_ptr16(grad_y))
+    return MOE_ERR_INVALID_ARGUMENT;
+  return moe::launch_ffn_weight_grad(x_perm, h, d_gate, d_up, grad_y, cu_seqlens, M, H, Hp, E,
+                                     grad_w_gate, grad_w_up, grad_w_down, accumulate != 0,
+                                     d_status, stream);
+}
+
+moe_status moe_grouped_ffn_backward(const void* x_perm, const void* h, const void* gate_pre,
+                                    const void* up_pre, const void* w_gate, const void* w_up,
+                                    const void* w_down, const int32_t* cu_seqlens, int64_t M,
+                                    int64_t H, int64_t Hp, int32_t E, const void* grad_y,
+                                    void* d_gate, void* d_up, void* grad_x_perm,
+                                    float* grad_w_gate, float* grad_w_up, float* grad_w_down,
+                                    int32_t accumulate, int32_t* d_status, void* cuda_stream) {
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  // validate all three passes before launching any
+  if (accumulate != 0 && accumulate != 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (!ok_ptr16(grad_w_gate) || !ok_ptr16(grad_w_up) || !ok_ptr16(grad_w_down) ||
+      cu_seqlens == nullptr || !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M > 0 && (!ok_ptr16(x_perm) || !ok_ptr16(h) || !ok_ptr16(gate_pre) || !ok_ptr16(up_pre) ||
+                !ok_ptr16(w_gate) || !ok_ptr16(w_up) || !ok_ptr16(w_down) ||
+                !ok_ptr16(grad_y) || !ok_ptr16(d_gate) || !ok_ptr16(d_up) ||
+                !ok_ptr16(grad_x_perm)))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M > 0) {
+    moe_status s = moe_grouped_ffn_down_backward(grad_y, w_down, gate_pre, up_pre, cu_seqlens, M,
+                                                 H, Hp, E, d_gate, d_up, d_status, cuda_stream);
+    if (s != MOE_OK) return s;
+    s = moe_grouped_ffn_up_gate_backward(d_gate, d_up, w_gate, w_up, cu_seqlens, M, H, Hp, E,
+                                         grad_x_perm, d_status, cuda_stream);
+    if (s != MOE_OK) return s;
+  }
+  return moe_grouped_ffn_weight_grad(x_perm, h, d_gate, d_up, grad_y, cu_seqlens, M, H, Hp, E,
+                                     grad_w_gate, grad_w_up, grad_w_down, accumulate, d_status,
+                                     cuda_stream);
 }
 
 moe_status moe_unpermute_combine(const void* y, const int32_t* row_id_map, const float* route_w,

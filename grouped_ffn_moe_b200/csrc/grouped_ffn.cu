@@ -22,47 +22,26 @@
 // (and, for an expert split into chunks, its weight tile) through L2, so each weight byte
 // crosses HBM about once, and a hot expert's chunks spread over all SMs.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads into a kStages-deep shared-memory ring;
-// warp 1 owns TMEM (alloc/dealloc) and issues the MMAs from one thread; warps 2-5 drain the
-// fp32 accumulators with tcgen05.ld, apply SiLU*up (pass 1) and rounding, transpose through
-// shared memory and store whole 16-byte vectors of the expert's rows only.
+// Warp roles (320 threads): warp 0 issues TMA loads into a kStages-deep shared-memory ring;
+// warp 1 owns TMEM (alloc/dealloc) and issues the MMAs from one thread; warps 2-9 (two groups
+// of four, alternating 32-token chunks) drain the fp32 accumulators with tcgen05.ld, apply
+// SiLU*up (pass 1) and rounding, transpose through shared memory and store whole 16-byte
+// vectors of the expert's rows only. For training, pass 1 also stores the pre-activations
+// bf16(x.W_gate) and bf16(x.W_up) that the backward differentiates SwiGLU at.
 // Every wait is bounded (globaltimer); on expiry the CTA records MOE_ERR_DEVICE_TIMEOUT,
 // drains its own copies and MMAs with bounded waits, frees TMEM and exits.
-#include <cuda.h>
-#include <cuda_bf16.h>
-#include <cudaTypedefs.h>
-
 #include <atomic>
 #include <cstdlib>
-#include <mutex>
 #include <string>
 
-#include "internal.h"
-#include "ptx.cuh"
+#include "gemm_common.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kBM = 128;                       // output features per unit (UMMA M)
-constexpr int kBK = 64;                        // reduction elements per stage (128 bytes)
-constexpr int kNMax = 256;                     // tokens per unit (UMMA N max)
 #ifndef MOE_SWIGLU_NMAX
 #define MOE_SWIGLU_NMAX 256                    // tokens per SwiGLU unit (128: two TMEM stages)
 #endif
-constexpr int kABytes = kBM * kBK * 2;         // 16 KB: [2 halves][64 k][64 f], one TMA box
-constexpr int kAHalfBytes = 64 * kBK * 2;      // 8 KB: one 64-feature half (UMMA LBO)
-constexpr int kRowBytes = kBK * 2;             // one token row of a B stage (128 bytes)
-constexpr int kNumBoxHeights = 5;              // token boxes of 256, 128, 64, 32, 16 rows
-constexpr int kEpiGroups = 2;                  // epilogue warp groups, alternating chunks
-constexpr int kEpiThreads = 128 * kEpiGroups;
-constexpr int kThreads = 64 + kEpiThreads;     // TMA warp, MMA warp, epilogue warps
-constexpr int kOutChunk = 32;                  // tokens per epilogue chunk
-constexpr int kOutBytes = kOutChunk * kBM * 2;  // 8 KB staging buffer per group
-constexpr uint32_t kTmemCols = 512;
-// After a time-out, waits for this CTA's own copies and MMAs to land use this fixed bound
-// (not the caller's budget, which may be tiny), so that nothing is in flight at exit.
-constexpr uint64_t kDrainBudgetNs = 200000000ull;
-constexpr uint32_t kAccCols = 256;
 
 // Kernel modes.
 //   kSwiGLU: A0 = W_gate, A1 = W_up on the same 128 features; h = silu(acc0) * acc1.
@@ -94,13 +73,6 @@ static_assert(Cfg<kSwiGLU>::kSmemBytes <= 232448, "shared memory budget (SwiGLU)
 static_assert(Cfg<kSingle>::kSmemBytes <= 232448, "shared memory budget (single)");
 static_assert(Cfg<kPair>::kSmemBytes <= 232448, "shared memory budget (pair)");
 
-// Token-row tensor maps of one activation matrix, box heights 256, 128, 64, 32, 16 rows: a
-// unit's N rows (a multiple of 16) load as the binary decomposition of N, i.e. at most five
-// boxes and no row beyond the 16-row rounding.
-struct RowMaps {
-  CUtensorMap m[kNumBoxHeights + 1];  // + an 8-row box for the CTA-pair kernel's half tiles
-};
-
 struct FfnArgs {
   const int32_t* cu;     // [E+1]
   __nv_bfloat16* out;    // [M, n_feat]
@@ -110,41 +82,9 @@ struct FfnArgs {
   int32_t k_dim;         // reduction length: H (pass 1) or H' (pass 2)
   int32_t n_feat;        // output features: H' (pass 1) or H (pass 2)
   uint64_t budget_ns;
+  __nv_bfloat16* gate_pre;  // [M, H'] bf16(x.W_gate), pass 1 when training; else null
+  __nv_bfloat16* up_pre;    // [M, H'] bf16(x.W_up), with gate_pre
 };
-
-struct Unit {
-  int e, fb, row0, nrows, ntc;
-};
-
-// Unit u -> (expert, feature block, token rows). s_ustart[e] is the first unit of expert e;
-// a feature block is 128 features (256 in kPair mode).
-template <int kNMaxU = kNMax>
-__device__ __forceinline__ Unit decode_unit(int u, const int32_t* s_ustart, const int32_t* s_cu,
-                                            int E) {
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (s_ustart[mid] <= u) lo = mid; else hi = mid - 1;
-  }
-  Unit U;
-  U.e = lo;
-  const int local = u - s_ustart[lo];
-  const int cnt = s_cu[lo + 1] - s_cu[lo];
-  const int ntc = (cnt + kNMaxU - 1) / kNMaxU;
-  U.ntc = ntc;
-  U.fb = local / ntc;
-  const int tc = local - U.fb * ntc;
-  const int cs = (((cnt + ntc - 1) / ntc) + 15) & ~15;  // balanced chunks, multiple of 16
-  const int r0 = tc * cs;
-  U.row0 = s_cu[lo] + r0;
-  U.nrows = min(cnt - r0, cs);
-  return U;
-}
-
-__device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
-  const uint32_t a = smem_u32(p);
-  return p + ((1024u - (a & 1023u)) & 1023u);
-}
 
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -166,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
-  int32_t* s_scan = reinterpret_cast<int32_t*>(smem + C::kOffMisc + 8);  // [8]
+  int32_t* s_scan = reinterpret_cast<int32_t*>(smem + C::kOffMisc + 8);  // [10]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = args.E;
@@ -200,42 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // cu_seqlens and the activations come from earlier kernels in the stream
   griddep_wait();
   griddep_launch_dependents();
-  // cu_seqlens, clamped to [0, M] so that no row outside [0, M) is ever addressed
-  for (int e = tid; e <= E; e += kThreads) {
-    int64_t v = args.cu[e];
-    v = v < 0 ? 0 : (v > args.M ? args.M : v);
-    s_cu[e] = static_cast<int32_t>(v);
-  }
-  __syncthreads();
-  // units per expert, then an exclusive scan into s_ustart[0..E]
-  {
-    const int per = (E + kThreads - 1) / kThreads;  // <= 6 for E <= 1024
-    const int beg = min(tid * per, E), end = min(beg + per, E);
-    int local = 0;
-    for (int e = beg; e < end; ++e) {
-      const int cnt = s_cu[e + 1] - s_cu[e];
-      const int units = cnt > 0 ? ((cnt + C::kNMaxMode - 1) / C::kNMaxMode) * nfb : 0;
-      s_ustart[e] = units;
-      local += units;
-    }
-    int incl = local;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, incl, d);
-      if (lane >= d) incl += n;
-    }
-    if (lane == 31) s_scan[warp] = incl;
-    __syncthreads();
-    int off = 0;
-    for (int w = 0; w < warp; ++w) off += s_scan[w];
-    int run = off + incl - local;
-    for (int e = beg; e < end; ++e) {
-      const int units = s_ustart[e];
-      s_ustart[e] = run;
-      run += units;
-    }
-    if (tid == kThreads - 1) s_ustart[E] = off + incl;
-  }
+  unit_starts(args.cu, args.M, E, nfb, C::kNMaxMode, s_cu, s_ustart, s_scan);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -367,8 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit U = decode_unit<C::kNMaxMode>(u, s_ustart, s_cu, E);
       if (U.nrows <= 0) continue;
       mbar_wait_bounded(&tfull[astage], aphase, s_abort, args.budget_ns);
-      named_bar_sync(bar_all, kEpiThreads);  // every epilogue warp takes the same decision
-      if (*s_abort) break;
+      // every epilogue warp takes the same decision
+      if (named_bar_red_or(bar_all, kEpiThreads, *s_abort != 0)) break;
       tc_fence_after();
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + astage * kAccCols;
@@ -378,10 +283,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int f0 = U.fb * C::kFeatPerUnit + half * kBM;
           if (f0 >= args.n_feat) break;  // uniform across the group
           __syncwarp();  // tcgen05.ld is .sync.aligned: whole warp, converged
-          uint32_t r0[32];
+          // staged chunk [32 tokens][128 features] -> rows of dst (row stride n_feat)
+          auto store_chunk = [&](__nv_bfloat16* dst_base) {
+            named_bar_sync(bar_grp, 128);
+#pragma unroll
+            for (int p = 0; p < (kOutChunk * kBM * 2 / 16) / 128; ++p) {
+              const int vid = gt + 128 * p;
+              const int j = vid >> 4, c16 = vid & 15;
+              if (c + j < U.nrows) {
+                const uint4 val =
+                    *reinterpret_cast<const uint4*>(so_bytes + j * (kBM * 2) + c16 * 16);
+                __nv_bfloat16* dst = dst_base +
+                                     static_cast<int64_t>(U.row0 + c + j) * args.n_feat + f0 +
+                                     c16 * 8;
+                *reinterpret_cast<uint4*>(dst) = val;
+              }
+            }
+            named_bar_sync(bar_grp, 128);  // staging buffer free for the group's next use
+          };
+          uint32_t r0[32], r1[32];
           tmem_ld_32x32b_x32(tbase + half * kAccCols + c, r0);
           if (kMode == kSwiGLU) {
-            uint32_t r1[32];
             tmem_ld_32x32b_x32(tbase + C::kUpOff + c, r1);
             tmem_ld_wait();
 #pragma unroll
@@ -398,20 +320,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j)
               so[j * kBM + f_local] = __float2bfloat16_rn(__uint_as_float(r0[j]));
           }
-          named_bar_sync(bar_grp, 128);
+          store_chunk(args.out);
+          if (kMode == kSwiGLU && args.gate_pre != nullptr) {
+            // training: the pre-activations, each rounded once from the fp32 accumulator
 #pragma unroll
-          for (int p = 0; p < (kOutChunk * kBM * 2 / 16) / 128; ++p) {
-            const int vid = gt + 128 * p;
-            const int j = vid >> 4, c16 = vid & 15;
-            if (c + j < U.nrows) {
-              const uint4 val =
-                  *reinterpret_cast<const uint4*>(so_bytes + j * (kBM * 2) + c16 * 16);
-              __nv_bfloat16* dst =
-                  args.out + static_cast<int64_t>(U.row0 + c + j) * args.n_feat + f0 + c16 * 8;
-              *reinterpret_cast<uint4*>(dst) = val;
-            }
+            for (int j = 0; j < 32; ++j)
+              so[j * kBM + f_local] = __float2bfloat16_rn(__uint_as_float(r0[j]));
+            store_chunk(args.gate_pre);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              so[j * kBM + f_local] = __float2bfloat16_rn(__uint_as_float(r1[j]));
+            store_chunk(args.up_pre);
           }
-          named_bar_sync(bar_grp, 128);  // staging buffer free for the group's next use
         }
       }
       tc_fence_before();
@@ -520,40 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();  // both CTAs' barriers exist before either signals the other
   griddep_wait();
   griddep_launch_dependents();
-  for (int e = tid; e <= E; e += kThreads) {
-    int64_t v = args.cu[e];
-    v = v < 0 ? 0 : (v > args.M ? args.M : v);
-    s_cu[e] = static_cast<int32_t>(v);
-  }
-  __syncthreads();
-  {
-    const int per = (E + kThreads - 1) / kThreads;
-    const int beg = min(tid * per, E), end = min(beg + per, E);
-    int local = 0;
-    for (int e = beg; e < end; ++e) {
-      const int cnt = s_cu[e + 1] - s_cu[e];
-      const int units = cnt > 0 ? ((cnt + 255) / 256) * nfb : 0;
-      s_ustart[e] = units;
-      local += units;
-    }
-    int incl = local;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, incl, d);
-      if (lane >= d) incl += n;
-    }
-    if (lane == 31) s_scan[warp] = incl;
-    __syncthreads();
-    int off = 0;
-    for (int w = 0; w < warp; ++w) off += s_scan[w];
-    int run = off + incl - local;
-    for (int e = beg; e < end; ++e) {
-      const int units = s_ustart[e];
-      s_ustart[e] = run;
-      run += units;
-    }
-    if (tid == kThreads - 1) s_ustart[E] = off + incl;
-  }
+  unit_starts(args.cu, args.M, E, nfb, 256, s_cu, s_ustart, s_scan);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -678,8 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit U = decode_unit(u, s_ustart, s_cu, E);
       if (U.nrows <= 0) continue;
       mbar_wait_bounded(&tfull[astage], aphase, s_abort, args.budget_ns);
-      named_bar_sync(bar_all, kEpiThreads);
-      if (*s_abort) break;
+      // every epilogue warp takes the same decision
+      if (named_bar_red_or(bar_all, kEpiThreads, *s_abort != 0)) break;
       tc_fence_after();
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + astage * kAccCols;
@@ -743,67 +630,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------------- host side
-
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// Token rows: row-major bf16 [rows, inner] with a (64 x box_rows) box, 128-byte swizzle.
-bool make_row_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows,
-                  uint32_t box_rows) {
-  auto enc = get_encode_fn();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool make_row_maps(RowMaps* maps, const void* ptr, uint64_t inner, uint64_t rows) {
-  for (int i = 0; i < kNumBoxHeights + 1; ++i)
-    if (!make_row_map(&maps->m[i], ptr, inner, rows, static_cast<uint32_t>(kNMax >> i)))
-      return false;
-  return true;
-}
-
-// Weights W[E * k_dim][n_feat] (bf16, features contiguous) viewed in three dimensions,
-// (64 features, E * k_dim rows, n_feat / 64 halves): one (64 x 64 x 2) box is the unit's
-// 128 features x 64 k, laid out as two 8 KB MN-major halves, 128-byte swizzle; with
-// halves = 1 a box is one 8 KB half (the CTA-pair kernel).
-bool make_weight_map(CUtensorMap* m, const void* ptr, uint64_t n_feat, uint64_t rows,
-                     uint32_t halves = 2) {
-  auto enc = get_encode_fn();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[3] = {64, rows, n_feat / 64};
-  cuuint64_t strides[2] = {n_feat * 2, 128};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kBK), halves};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-uint64_t wait_budget_ns() {
-  static uint64_t budget = [] {
-    const char* s = std::getenv("MOE_WAIT_BUDGET_NS");
-    if (s != nullptr && *s) return static_cast<uint64_t>(std::strtoull(s, nullptr, 10));
-    return static_cast<uint64_t>(2000000000ull);  // 2 s
-  }();
-  return budget;
-}
 
 template <int kMode>
 bool ensure_smem_attr() {
@@ -881,20 +707,24 @@ int down_mode() {
 
 moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const void* w1,
                            const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp, int32_t E,
-                           void* out, int32_t* d_status, cudaStream_t stream) {
+                           void* out, void* gate_pre, void* up_pre, int32_t* d_status,
+                           cudaStream_t stream) {
   const int grid = num_sms();
   if (dual) {
     CUtensorMap m_wg, m_wu;
     RowMaps m_x;
-    const uint32_t halves = use_pair_swiglu() ? 1 : 2;
+    // the CTA-pair kernel does not store pre-activations: training uses the one-CTA kernel
+    const bool pair = use_pair_swiglu() && gate_pre == nullptr;
+    const uint32_t halves = pair ? 1 : 2;
     if (!make_weight_map(&m_wg, w0, Hp, static_cast<uint64_t>(E) * H, halves) ||
         !make_weight_map(&m_wu, w1, Hp, static_cast<uint64_t>(E) * H, halves) ||
         !make_row_maps(&m_x, act, H, M) || !ensure_smem_attr<kSwiGLU>())
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
-                    static_cast<int32_t>(H), static_cast<int32_t>(Hp), wait_budget_ns()};
+                    static_cast<int32_t>(H), static_cast<int32_t>(Hp), wait_budget_ns(),
+                    static_cast<__nv_bfloat16*>(gate_pre), static_cast<__nv_bfloat16*>(up_pre)};
     const cudaError_t err =
-        use_pair_swiglu()
+        pair
             ? launch_swiglu_pair(m_wg, m_wu, m_x, a, stream)
             : launch_dependent(grouped_ffn_kernel<kSwiGLU>, dim3(grid), dim3(kThreads),
                                Cfg<kSwiGLU>::kSmemBytes, stream, m_wg, m_wu, m_x, a);
@@ -908,7 +738,8 @@ moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const voi
         !(pair ? ensure_smem_attr<kPair>() : ensure_smem_attr<kSingle>()))
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
-                    static_cast<int32_t>(Hp), static_cast<int32_t>(H), wait_budget_ns()};
+                    static_cast<int32_t>(Hp), static_cast<int32_t>(H), wait_budget_ns(),
+                    nullptr, nullptr};
     const cudaError_t err =
         pair ? launch_dependent(grouped_ffn_kernel<kPair>, dim3(grid), dim3(kThreads),
                                 Cfg<kPair>::kSmemBytes, stream, m_wd, m_wd, m_h, a)

@@ -65,9 +65,33 @@ moe_status launch_combine_backward(const void* grad_out, const void* y, const in
                                    void* grad_y, float* grad_w, cudaStream_t stream);
 
 // One pass of the grouped FFN. dual: h = SwiGLU pass (w0 = gate, w1 = up, act = x_perm,
-// out = h); otherwise the down pass (w0 = down, act = h, out = y).
+// out = h; gate_pre/up_pre non-null also stores the bf16 pre-activations); otherwise the down
+// pass (w0 = down, act = h, out = y; gate_pre/up_pre must be null).
 moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const void* w1,
                            const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp, int32_t E,
-                           void* out, int32_t* d_status, cudaStream_t stream);
+                           void* out, void* gate_pre, void* up_pre, int32_t* d_status,
+                           cudaStream_t stream);
+
+// Backward of the down projection fused with the SwiGLU backward: from grad_y [M,H] and the
+// saved pre-activations [M,H'], d_gate and d_up [M,H'] (bf16).
+moe_status launch_ffn_down_backward(const void* grad_y, const void* w_down, const void* gate_pre,
+                                    const void* up_pre, const int32_t* cu_seqlens, int64_t M,
+                                    int64_t H, int64_t Hp, int32_t E, void* d_gate, void* d_up,
+                                    int32_t* d_status, cudaStream_t stream);
+
+// Backward of the up and gate projections to the input rows:
+// grad_x_perm = d_gate W_gate^T + d_up W_up^T (bf16 [M,H]).
+moe_status launch_ffn_up_gate_backward(const void* d_gate, const void* d_up, const void* w_gate,
+                                       const void* w_up, const int32_t* cu_seqlens, int64_t M,
+                                       int64_t H, int64_t Hp, int32_t E, void* grad_x_perm,
+                                       int32_t* d_status, cudaStream_t stream);
+
+// Weight gradients (fp32, written or added into): grad_w_gate = x^T d_gate, grad_w_up =
+// x^T d_up ([E,H,H']), grad_w_down = h^T grad_y ([E,H',H]), sums over each expert's rows.
+moe_status launch_ffn_weight_grad(const void* x_perm, const void* h, const void* d_gate,
+                                  const void* d_up, const void* grad_y, const int32_t* cu_seqlens,
+                                  int64_t M, int64_t H, int64_t Hp, int32_t E, float* grad_w_gate,
+                                  float* grad_w_up, float* grad_w_down, bool accumulate,
+                                  int32_t* d_status, cudaStream_t stream);
 
 }  // namespace moe

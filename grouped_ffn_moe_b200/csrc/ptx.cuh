@@ -221,6 +221,20 @@ __device__ __forceinline__ uint32_t idesc_bf16_m128_amn_bk(uint32_t n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f16 with bf16 A and B and fp32 D, for any M (64/128 per CTA),
+// N (multiple of 16 up to 256) and either major-ness of each operand (1 = MN-major).
+__device__ __forceinline__ uint32_t idesc_bf16(uint32_t m, uint32_t n, uint32_t a_mn,
+                                               uint32_t b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn << 15) | (b_mn << 16) | ((n >> 3) << 17) |
+         ((m >> 4) << 24);
+}
+
+// Makes this thread's generic-proxy writes to shared memory visible to the async proxy
+// (TMA, tcgen05.mma operand reads) that follows.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Named barrier over `nthreads` threads; threads of a warp may arrive diverged.
 // ----------------------------------------------------------------------------- CTA pairs
 // (a cluster of two CTAs working as one tcgen05 pair: cta_group::2)
@@ -334,6 +348,21 @@ __device__ __forceinline__ uint32_t idesc_bf16_amn_bk(uint32_t m, uint32_t n) {
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier over `nthreads` threads that also ORs a predicate across them: every
+// participant gets the same result (a uniform decision from values read at different times).
+__device__ __forceinline__ bool named_bar_red_or(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 }  // namespace moe

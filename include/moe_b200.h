@@ -173,6 +173,76 @@ moe_status moe_grouped_ffn_down(const void* h_scratch, const void* w_down,
                                 int32_t E, void* y, int32_t* d_status, void* cuda_stream);
 
 /*
+ * moe_grouped_ffn_up_gate_train - moe_grouped_ffn_up_gate for training: the same h, plus the
+ * pre-activations the backward differentiates SwiGLU at, each rounded once to bf16 from the
+ * fp32 accumulator:
+ *   gate_pre[r] = bf16(x_perm[r] . W_gate[e]),   up_pre[r] = bf16(x_perm[r] . W_up[e])
+ *   gate_pre, up_pre  [M, Hp] bf16 out (caller-owned, 16-byte aligned).
+ * Other arguments, requirements and errors as moe_grouped_ffn_up_gate.
+ */
+moe_status moe_grouped_ffn_up_gate_train(const void* x_perm, const void* w_gate,
+                                         const void* w_up, const int32_t* cu_seqlens, int64_t M,
+                                         int64_t H, int64_t Hp, int32_t E, void* h_scratch,
+                                         void* gate_pre, void* up_pre, int32_t* d_status,
+                                         void* cuda_stream);
+
+/*
+ * moe_grouped_ffn_backward - backward of the grouped expert FFN: the chain rule of
+ * Down(SwiGLU(Up x, Gate x)) ("Mixture of Kittens" digest, Step 1) per expert over the rows
+ * cu_seqlens selects, with fp32 weight-gradient buffers laid out like the weights (MoonEP
+ * README, "Gradient buffers"). With g = gate_pre[r], u = up_pre[r], s = sigmoid(g):
+ *   grad_h       = grad_y[r] . W_down[e]^T                      (fp32, not stored)
+ *   d_gate[r]    = bf16(grad_h * u * s * (1 + g * (1 - s)))
+ *   d_up[r]      = bf16(grad_h * g * s)
+ *   grad_x_perm[r] = bf16(d_gate[r] . W_gate[e]^T + d_up[r] . W_up[e]^T)   (one fp32 sum)
+ *   grad_w_gate[e] (+)= sum_r x_perm[r]^T d_gate[r]     [E, H, Hp] fp32
+ *   grad_w_up[e]   (+)= sum_r x_perm[r]^T d_up[r]       [E, H, Hp] fp32
+ *   grad_w_down[e] (+)= sum_r h[r]^T grad_y[r]          [E, Hp, H] fp32
+ * It runs the three calls below on one stream, in this order.
+ *   x_perm [M, H], h [M, Hp], gate_pre, up_pre [M, Hp]: bf16 from the training forward.
+ *   w_gate, w_up [E, H, Hp], w_down [E, Hp, H]: bf16 weights of the forward.
+ *   grad_y [M, H] bf16: gradient of the expert outputs (e.g. from moe_combine_backward).
+ *   d_gate, d_up [M, Hp] bf16 out (kept: the weight gradients read them); grad_x_perm [M, H]
+ *   bf16 out (e.g. into moe_permute_backward).
+ *   accumulate: 0 = the weight gradients are written; 1 = added into the buffers' contents.
+ *   An expert without rows gets a zero gradient (left unchanged when accumulating).
+ * Requirements, d_status and errors as moe_grouped_ffn; every pointer 16-byte aligned.
+ */
+moe_status moe_grouped_ffn_backward(const void* x_perm, const void* h, const void* gate_pre,
+                                    const void* up_pre, const void* w_gate, const void* w_up,
+                                    const void* w_down, const int32_t* cu_seqlens, int64_t M,
+                                    int64_t H, int64_t Hp, int32_t E, const void* grad_y,
+                                    void* d_gate, void* d_up, void* grad_x_perm,
+                                    float* grad_w_gate, float* grad_w_up, float* grad_w_down,
+                                    int32_t accumulate, int32_t* d_status, void* cuda_stream);
+
+/*
+ * The three passes of moe_grouped_ffn_backward, callable on their own (same arguments and
+ * conventions):
+ *   moe_grouped_ffn_down_backward     d_gate, d_up from grad_y, W_down, gate_pre, up_pre
+ *   moe_grouped_ffn_up_gate_backward  grad_x_perm from d_gate, d_up, W_gate, W_up
+ *   moe_grouped_ffn_weight_grad       grad_w_gate, grad_w_up, grad_w_down
+ */
+moe_status moe_grouped_ffn_down_backward(const void* grad_y, const void* w_down,
+                                         const void* gate_pre, const void* up_pre,
+                                         const int32_t* cu_seqlens, int64_t M, int64_t H,
+                                         int64_t Hp, int32_t E, void* d_gate, void* d_up,
+                                         int32_t* d_status, void* cuda_stream);
+
+moe_status moe_grouped_ffn_up_gate_backward(const void* d_gate, const void* d_up,
+                                            const void* w_gate, const void* w_up,
+                                            const int32_t* cu_seqlens, int64_t M, int64_t H,
+                                            int64_t Hp, int32_t E, void* grad_x_perm,
+                                            int32_t* d_status, void* cuda_stream);
+
+moe_status moe_grouped_ffn_weight_grad(const void* x_perm, const void* h, const void* d_gate,
+                                       const void* d_up, const void* grad_y,
+                                       const int32_t* cu_seqlens, int64_t M, int64_t H,
+                                       int64_t Hp, int32_t E, float* grad_w_gate,
+                                       float* grad_w_up, float* grad_w_down, int32_t accumulate,
+                                       int32_t* d_status, void* cuda_stream);
+
+/*
  * moe_unpermute_combine - restore token order, scale by route weight, sum the K results
  * ("Distributed expert parallelism", lifecycle step 8 and "Duplicate route accumulation";
  * MoonEP README, "combine fwd").

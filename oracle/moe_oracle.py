@@ -281,21 +281,37 @@ def swiglu_backward(grad_h: np.ndarray, g_bits: np.ndarray, u_bits: np.ndarray):
             f64_to_bf16_bits(grad_h * (g * s)))
 
 
+def expert_down_backward_rows(grad_y_bits, g_bits, u_bits, w_down_e):
+    """Down projection and SwiGLU backward of one expert's rows: (d_g bits, d_u bits)."""
+    grad_h = bf16_bits_to_f64(grad_y_bits) @ bf16_bits_to_f64(w_down_e).T
+    return swiglu_backward(grad_h, g_bits, u_bits)
+
+
+def expert_up_gate_backward_rows(dg_bits, du_bits, w_gate_e, w_up_e):
+    """Input-row gradient of one expert: bf16(d_g Wg^T + d_u Wu^T), one rounding."""
+    return f64_to_bf16_bits(bf16_bits_to_f64(dg_bits) @ bf16_bits_to_f64(w_gate_e).T +
+                            bf16_bits_to_f64(du_bits) @ bf16_bits_to_f64(w_up_e).T)
+
+
+def expert_weight_grads_rows(x_rows_bits, h_bits, dg_bits, du_bits, grad_y_bits):
+    """Weight gradients of one expert as float64 sums over its rows: (x^T d_g, x^T d_u,
+    h^T grad_y)."""
+    x = bf16_bits_to_f64(x_rows_bits)
+    return (x.T @ bf16_bits_to_f64(dg_bits), x.T @ bf16_bits_to_f64(du_bits),
+            bf16_bits_to_f64(h_bits).T @ bf16_bits_to_f64(grad_y_bits))
+
+
 def expert_ffn_backward_rows(x_rows_bits, g_bits, u_bits, h_bits, grad_y_bits, w_gate_e, w_up_e,
                              w_down_e):
-    """Backward of one expert on a block of rows.
+    """Backward of one expert on a block of rows: the three stages above in order.
 
     Returns (d_g bits, d_u bits, grad_x bits, dWg, dWu, dWd), the weight gradients as
     float64 sums of the block's rows (the caller stores them as fp32).
     """
-    gy = bf16_bits_to_f64(grad_y_bits)
-    grad_h = gy @ bf16_bits_to_f64(w_down_e).T
-    dg_bits, du_bits = swiglu_backward(grad_h, g_bits, u_bits)
-    dg, du = bf16_bits_to_f64(dg_bits), bf16_bits_to_f64(du_bits)
-    grad_x = f64_to_bf16_bits(dg @ bf16_bits_to_f64(w_gate_e).T + du @ bf16_bits_to_f64(w_up_e).T)
-    x = bf16_bits_to_f64(x_rows_bits)
-    h = bf16_bits_to_f64(h_bits)
-    return dg_bits, du_bits, grad_x, x.T @ dg, x.T @ du, h.T @ gy
+    dg_bits, du_bits = expert_down_backward_rows(grad_y_bits, g_bits, u_bits, w_down_e)
+    grad_x = expert_up_gate_backward_rows(dg_bits, du_bits, w_gate_e, w_up_e)
+    return (dg_bits, du_bits, grad_x,
+            *expert_weight_grads_rows(x_rows_bits, h_bits, dg_bits, du_bits, grad_y_bits))
 
 
 def grouped_ffn_preact(x_perm_bits: np.ndarray, cu_seqlens: np.ndarray, get_weights, Hp: int):

@@ -63,3 +63,23 @@ def assert_close_bf16(got_bits: np.ndarray, ref_bits: np.ndarray, what: str = ""
     mx = float(np.abs(diff).max()) / max(rms, 1e-30) if diff.size else 0.0
     return {"rel_fro": float(rel), "max_abs_over_rms": mx, "one_step_flips_over_bar": n_over,
             "exact_fraction": float((diff == 0).mean()) if diff.size else 1.0}
+
+
+# Weight gradients are fp32 sums over an expert's n rows of exact bf16 x bf16 products. A
+# sum of n terms with fp32 additions (rounded or truncated, in any order and grouping) is
+# within (n - 1) * 2^-23 * sum|terms| of the exact sum to first order; the bar takes twice
+# that, plus one final rounding (two when the result is added into a prior fp32 value).
+def assert_close_fp32_sums(got, ref, abs_sum, n_terms: int, what: str = "", added=False):
+    g = np.asarray(got, np.float64)
+    r = np.asarray(ref, np.float64)
+    assert g.shape == r.shape, (what, g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite values"
+    u = 2.0 ** -23
+    bound = 2.0 * n_terms * u * np.asarray(abs_sum, np.float64) + (2 if added else 1) * u * np.abs(r)
+    err = np.abs(g - r)
+    bad = err > bound + 1e-38
+    assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond the fp32 summation bound "
+                           f"(worst excess {float((err - bound).max()):.3e})")
+    nr = np.linalg.norm(r)
+    return {"rel_fro": float(np.linalg.norm(g - r) / max(nr, 1e-30)),
+            "max_err_over_bound": float((err / np.maximum(bound, 1e-38)).max()) if err.size else 0.0}
