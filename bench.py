@@ -43,6 +43,8 @@ def parse_args():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-backward", action="store_true",
+                   help="skip the training-step leg (forward with saved pre-activations + backward)")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="CPU work budget for the oracle baseline sample")
     return p.parse_args()
@@ -109,6 +111,15 @@ def work_model(w, counts=None):
         m["up_gate_bytes"] = 2 * 2 * active * H * Hp + 2 * M * H + 2 * M * Hp
         m["down_flops"] = 2 * M * H * Hp
         m["down_bytes"] = 2 * active * Hp * H + 2 * M * Hp + 2 * M * H
+        # backward (weights read once per pass; fp32 weight gradients written once)
+        m["combine_bwd_bytes"] = 2 * S * H + 4 * M * H + 8 * M
+        m["permute_bwd_bytes"] = 2 * (M + S) * H + 4 * M
+        m["down_bwd_flops"] = 2 * M * H * Hp
+        m["down_bwd_bytes"] = 2 * active * Hp * H + 2 * M * H + 4 * 2 * M * Hp
+        m["up_gate_bwd_flops"] = 4 * M * H * Hp
+        m["up_gate_bwd_bytes"] = 2 * 2 * active * H * Hp + 2 * 2 * M * Hp + 2 * M * H
+        m["wgrad_flops"] = 6 * M * H * Hp
+        m["wgrad_bytes"] = 4 * 3 * E * H * Hp + 2 * M * (2 * H + 3 * Hp)
     return m
 
 
@@ -170,6 +181,114 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "power_w_max": max(pw) if pw else None, "samples": len(inside),
                 "window": window}
+
+
+# ----------------------------------------------------------------------------- training leg
+
+def measure_backward(moe, synth, torch, w, inp, dev, steps, warmup, flush, peaks, peak_src):
+    """Training step of the layer: forward with saved pre-activations, then the backward
+    (combine bwd -> down+SwiGLU bwd -> up/gate bwd -> fp32 weight gradients -> permute bwd),
+    with CUDA events between the kernels; L2 flushed before every step."""
+    buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev, train=True)
+    grads = moe.LayerGrads.allocate(w.S, w.H, w.Hp, w.E, w.K, dev)
+    grad_out = synth.normal_bf16_into(torch.empty(w.S, w.H, dtype=torch.bfloat16, device=dev),
+                                      w.seed, synth.TAG_GRAD)
+    wg, wu, wd = inp["w_gate"], inp["w_up"], inp["w_down"]
+    E, K = w.E, w.K
+
+    def train_step(ev=None):
+        rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
+        rec(0)
+        moe.moe_permute(inp["x"], inp["topk_ids"], E, buf.x_perm, buf.counts, buf.cu_seqlens,
+                        buf.row_id_map, buf.perm_src, buf.maxvio, buf.max_count, buf.workspace,
+                        buf.d_status)
+        rec(1)
+        moe.moe_grouped_ffn_up_gate_train(buf.x_perm, wg, wu, buf.cu_seqlens, buf.h, buf.gate_pre,
+                                          buf.up_pre, buf.d_status)
+        rec(2)
+        moe.moe_grouped_ffn_down(buf.h, wd, buf.cu_seqlens, buf.y, buf.d_status)
+        moe.moe_unpermute_combine(buf.y, buf.row_id_map, inp["route_w"], buf.out)
+        rec(3)
+        moe.moe_combine_backward(grad_out, buf.y, buf.row_id_map, inp["route_w"], grads.grad_y,
+                                 grads.grad_route_w)
+        rec(4)
+        moe.moe_grouped_ffn_down_backward(grads.grad_y, wd, buf.gate_pre, buf.up_pre,
+                                          buf.cu_seqlens, grads.d_gate, grads.d_up, buf.d_status)
+        rec(5)
+        moe.moe_grouped_ffn_up_gate_backward(grads.d_gate, grads.d_up, wg, wu, buf.cu_seqlens,
+                                             grads.grad_x_perm, buf.d_status)
+        rec(6)
+        moe.moe_grouped_ffn_weight_grad(buf.x_perm, buf.h, grads.d_gate, grads.d_up, grads.grad_y,
+                                        buf.cu_seqlens, grads.grad_w_gate, grads.grad_w_up,
+                                        grads.grad_w_down, False, buf.d_status)
+        rec(7)
+        moe.moe_permute_backward(grads.grad_x_perm, buf.row_id_map, grads.grad_x, K)
+        rec(8)
+
+    for _ in range(warmup):
+        flush.zero_()
+        train_step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        train_step(evs[i])
+    torch.cuda.synchronize()
+    status = int(buf.d_status.item())
+    if status != 0:
+        raise RuntimeError(f"device status {status} in the training leg")
+    names = ["permute", "up_gate_train", "down_and_combine", "combine_backward", "down_backward",
+             "up_gate_backward", "weight_grad", "permute_backward"]
+    ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i, n in enumerate(names)}
+    wm = work_model(w, buf.counts.cpu().numpy())
+    st = {
+        "up_gate_train": {"ms": ms["up_gate_train"],
+                          "TFLOP/s": wm["up_gate_flops"] / ms["up_gate_train"] / 1e9},
+        "combine_backward": {"ms": ms["combine_backward"],
+                             "GB/s": wm["combine_bwd_bytes"] / ms["combine_backward"] / 1e6},
+        "down_backward": {"ms": ms["down_backward"],
+                          "TFLOP/s": wm["down_bwd_flops"] / ms["down_backward"] / 1e9},
+        "up_gate_backward": {"ms": ms["up_gate_backward"],
+                             "TFLOP/s": wm["up_gate_bwd_flops"] / ms["up_gate_backward"] / 1e9},
+        "weight_grad": {"ms": ms["weight_grad"],
+                        "TFLOP/s": wm["wgrad_flops"] / ms["weight_grad"] / 1e9,
+                        "GB/s": wm["wgrad_bytes"] / ms["weight_grad"] / 1e6},
+        "permute_backward": {"ms": ms["permute_backward"],
+                             "GB/s": wm["permute_bwd_bytes"] / ms["permute_backward"] / 1e6},
+    }
+    bwd_ms = sum(ms[n] for n in names[3:])
+    # roofline of each backward GEMM pass: the slower of its tensor and HBM times
+    for key, fk, bk in (("down_backward", "down_bwd_flops", "down_bwd_bytes"),
+                        ("up_gate_backward", "up_gate_bwd_flops", "up_gate_bwd_bytes"),
+                        ("weight_grad", "wgrad_flops", "wgrad_bytes")):
+        t_tensor = wm[fk] / (peaks["bf16_tflops"] * 1e12)
+        t_hbm = wm[bk] / (peaks["hbm_gbs"] * 1e9)
+        bound = "tensor" if t_tensor >= t_hbm else "hbm"
+        st[key]["bound"] = bound
+        st[key]["frac_of_roofline"] = max(t_tensor, t_hbm) / (ms[key] / 1e3)
+    dom = max(("down_backward", "up_gate_backward", "weight_grad"), key=lambda k: ms[k])
+    d = st[dom]
+    if d["bound"] == "tensor":
+        roof = {"kernel": dom, "bound": "tensor", "achieved": d["TFLOP/s"],
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        byts = {"down_backward": wm["down_bwd_bytes"], "up_gate_backward": wm["up_gate_bwd_bytes"],
+                "weight_grad": wm["wgrad_bytes"]}[dom]
+        roof = {"kernel": dom, "bound": "hbm", "achieved": byts / ms[dom] / 1e6,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = f"{peak_src} (burst)"
+    return {"tokens_per_s": w.S / ((ms["permute"] + ms["up_gate_train"] + ms["down_and_combine"]
+                                    + bwd_ms) / 1e3),
+            "ms_training_step": sum(ms.values()), "ms_backward": bwd_ms,
+            "forward_train_overhead_ms": ms["up_gate_train"],
+            "stages": st, "roofline": roof,
+            "gpu_launches_per_step": sum(moe.LAUNCHES[n] for n in (
+                "moe_permute", "moe_grouped_ffn_up_gate_train", "moe_grouped_ffn_down",
+                "moe_unpermute_combine", "moe_combine_backward", "moe_grouped_ffn_down_backward",
+                "moe_grouped_ffn_up_gate_backward", "moe_grouped_ffn_weight_grad",
+                "moe_permute_backward")),
+            "weight_grad_dtype": "f32", "steps": steps, "warmup": warmup}
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -311,6 +430,12 @@ def run_ours(args):
         if not torch.equal(hout.to(dev), buf.out):
             raise RuntimeError("e2e output differs from the device-resident run")
 
+    backward = None
+    if not w.identity_ffn and not args.no_backward:
+        peaks0, src0 = load_peaks()
+        backward = measure_backward(moe, synth, torch, w, inp, dev, args.steps, args.warmup, flush,
+                                    peaks0, src0)
+
     if clocks is not None:
         clocks.stop()
 
@@ -335,15 +460,15 @@ def run_ours(args):
             flops, byts, t_s = wm["up_gate_flops"], wm["up_gate_bytes"], mean["up_gate"] / 1e3
             ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
             if flops / byts >= ridge:
-                roof = {"kernel": "grouped_ffn_kernel<true> (up/gate + SwiGLU)", "bound": "tensor",
+                roof = {"kernel": "grouped_ffn_kernel<0> (up/gate + SwiGLU)", "bound": "tensor",
                         "achieved": flops / t_s / 1e12, "peak": peaks["bf16_tflops"],
                         "unit": "TFLOP/s"}
             else:
-                roof = {"kernel": "grouped_ffn_kernel<true> (up/gate + SwiGLU)", "bound": "hbm",
+                roof = {"kernel": "grouped_ffn_kernel<0> (up/gate + SwiGLU)", "bound": "hbm",
                         "achieved": byts / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
         else:
             byts, t_s = wm["permute_bytes"], mean["permute"] / 1e3
-            roof = {"kernel": "moe_permute (4 kernels)", "bound": "hbm", "achieved": byts / t_s / 1e9,
+            roof = {"kernel": "moe_permute (2 kernels)", "bound": "hbm", "achieved": byts / t_s / 1e9,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["peak_source"] = f"{peak_src} (burst)"
@@ -363,6 +488,8 @@ def run_ours(args):
             "device_status": status,
             "clocks": clocks.summary(t0, t1) if clocks else None,
         }
+        if backward is not None:
+            line["training_step"] = backward
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
         print(json.dumps(line), flush=True)

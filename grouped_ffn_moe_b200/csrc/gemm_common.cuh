@@ -130,6 +130,10 @@ bool make_row_maps(RowMaps* maps, const void* ptr, uint64_t inner, uint64_t rows
 // out as `blocks` 8 KB 64-feature slices, 128-byte swizzle.
 bool make_weight_map(CUtensorMap* m, const void* ptr, uint64_t n_feat, uint64_t rows,
                      uint32_t blocks = 2);
+// A row-major fp32 matrix [rows][inner] with a (box_inner x box_rows) box, 128-byte swizzle
+// (box_inner * 4 must be 128): the staging layout of a TMA store or reduce-add.
+bool make_f32_tile_map(CUtensorMap* m, void* ptr, uint64_t inner, uint64_t rows,
+                       uint32_t box_inner, uint32_t box_rows);
 // Bound, in nanoseconds, of every pipeline wait in the GEMM kernels (MOE_WAIT_BUDGET_NS).
 uint64_t wait_budget_ns();
 

@@ -337,8 +337,12 @@ constexpr int kWKB = 64;                    // tokens per stage
 constexpr int kWABytes = 2 * kAHalfBytes;   // 16 KB: 128 X features x 64 tokens (MN-major)
 constexpr int kWBBytes = 4 * kAHalfBytes;   // 32 KB: 256 D features x 64 tokens (MN-major)
 constexpr int kWStageBytes = kWABytes + kWBBytes;
-constexpr int kWStages = 4;
-constexpr int kWOffCu = kWStages * kWStageBytes;
+constexpr int kWStages = 3;
+// epilogue staging: per epilogue warp two 32 x 32 fp32 tiles (4 KB, 128-byte swizzle), each
+// written to the gradient by one TMA store while the other is being filled
+constexpr int kWEpiTileBytes = 32 * 32 * 4;
+constexpr int kWOffEpi = kWStages * kWStageBytes;
+constexpr int kWOffCu = kWOffEpi + (kEpiThreads / 32) * 2 * kWEpiTileBytes;
 constexpr int kWOffBars = (kWOffCu + 4 * (MOE_MAX_EXPERTS + 1) + 7) & ~7;
 constexpr int kWNumBars = 2 * kWStages + 2 * 2 + 1;
 constexpr int kWOffMisc = kWOffBars + 8 * kWNumBars;
@@ -368,8 +372,9 @@ struct WgradArgs {
 };
 
 struct WgradMaps {
-  CUtensorMap x[kWProblems];  // (64, M, fx/64), box (64, 64, 2)
-  CUtensorMap d[kWProblems];  // (64, M, fd/64), box (64, 64, dblocks)
+  CUtensorMap x[kWProblems];    // (64, M, fx/64), box (64, 64, 2)
+  CUtensorMap d[kWProblems];    // (64, M, fd/64), box (64, 64, dblocks)
+  CUtensorMap out[kWProblems];  // fp32 (fd, E * fx), box (32, 32), 128-byte swizzle
 };
 
 struct WUnit {
@@ -424,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int p = 0; p < kWProblems; ++p) {
       tma_prefetch_map(&maps.x[p]);
       tma_prefetch_map(&maps.d[p]);
+      tma_prefetch_map(&maps.out[p]);
     }
   }
   if (warp == 1) {
@@ -552,11 +558,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // Epilogue: warp w owns gradient rows 32*(w%4) .. +31 of the tile (TMEM lanes); group
-    // grp takes the 32-column chunks c with (c / 32) % 2 == grp. A thread writes 32 fp32
-    // of one row (128 contiguous bytes) per chunk.
+    // grp takes the 32-column chunks c with (c / 32) % 2 == grp. A chunk (32 rows x 32 fp32)
+    // goes TMEM -> registers -> a 128-byte-swizzled shared tile (16-byte chunk j of row r at
+    // position j ^ (r % 8), conflict-free) -> one TMA bulk store (or, when accumulating, a
+    // TMA reduce-add: the fp32 addition happens at L2 and the prior values never reach the SM).
     const int q = warp & 3;
     const int grp = (warp - 2) >> 2;
     const uint32_t bar_all = 3;
+    uint8_t* tiles = smem + kWOffEpi + (warp - 2) * 2 * kWEpiTileBytes;
+    int ci = 0;  // chunks this warp has staged; tile (ci & 1) is the next one to fill
     int astage = 0;
     uint32_t aphase = 0;
     for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
@@ -564,15 +574,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WgradProblem& P = args.p[W.p];
       const int T = s_cu[W.e + 1] - s_cu[W.e];
       const int ncols = min(kWN, P.fd - W.nb * kWN);
-      const int64_t row = static_cast<int64_t>(W.e) * P.fx + W.mb * kBM + q * 32 + lane;
-      float* dst_row = P.out + row * P.fd + W.nb * kWN;
+      const int row0 = W.e * P.fx + W.mb * kBM + q * 32;  // first gradient row of this warp
       if (T <= 0) {
         // an expert without tokens: zero gradient (nothing to add when accumulating)
-        if (!args.accumulate)
+        if (!args.accumulate) {
+          float* dst_row = P.out + static_cast<int64_t>(row0 + lane) * P.fd + W.nb * kWN;
           for (int c = grp * kOutChunk; c < ncols; c += kEpiGroups * kOutChunk)
 #pragma unroll
             for (int v = 0; v < 8; ++v)
               *reinterpret_cast<float4*>(dst_row + c + 4 * v) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         continue;
       }
       mbar_wait_bounded(&tfull[astage], aphase, s_abort, args.budget_ns);
@@ -584,21 +595,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         uint32_t r[32];
         tmem_ld_32x32b_x32(tbase + c, r);
+        // the tile about to be filled was stored two chunks ago: its store must have read it
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
         tmem_ld_wait();
+        uint8_t* tile = tiles + (ci & 1) * kWEpiTileBytes;
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          float4 val = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                   __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-          float4* dp = reinterpret_cast<float4*>(dst_row + c + 4 * v);
-          if (args.accumulate) {
-            const float4 old = *dp;
-            val.x += old.x;
-            val.y += old.y;
-            val.z += old.z;
-            val.w += old.w;
-          }
-          *dp = val;
+        for (int v = 0; v < 8; ++v)
+          *reinterpret_cast<uint4*>(tile + lane * 128 + ((v ^ (lane & 7)) * 16)) =
+              make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int x = W.nb * kWN + c;
+          if (args.accumulate)
+            tma_reduce_add_2d(&maps.out[W.p], tile, x, row0);
+          else
+            tma_store_2d(&maps.out[W.p], tile, x, row0);
+          bulk_commit_group();
         }
+        ++ci;
       }
       tc_fence_before();
       __syncwarp();
@@ -608,6 +624,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         aphase ^= 1u;
       }
     }
+    if (lane == 0) bulk_wait_group<0>();  // this warp's stores complete before the CTA exits
+    __syncwarp();
   }
 
   __syncthreads();
@@ -721,7 +739,9 @@ moe_status launch_ffn_weight_grad(const void* x_perm, const void* h, const void*
     WgradProblem& P = a.p[p];
     P.dblocks = static_cast<int32_t>(fds[p] / 64 < 4 ? fds[p] / 64 : 4);
     if (!make_weight_map(&maps.x[p], xs[p], fxs[p], M, 2) ||
-        !make_weight_map(&maps.d[p], ds[p], fds[p], M, static_cast<uint32_t>(P.dblocks)))
+        !make_weight_map(&maps.d[p], ds[p], fds[p], M, static_cast<uint32_t>(P.dblocks)) ||
+        !make_f32_tile_map(&maps.out[p], outs[p], fds[p], static_cast<uint64_t>(E) * fxs[p], 32,
+                           32))
       return MOE_ERR_CUDA;
     P.out = outs[p];
     P.fx = static_cast<int32_t>(fxs[p]);
