@@ -50,21 +50,34 @@ def parse_args():
     return p.parse_args()
 
 
+KERNEL_SOURCES = {
+    # the files a kernel is compiled from: a recorded traffic figure holds only for them
+    "up_gate": ["grouped_ffn.cu", "gemm_common.cuh", "ptx.cuh"],
+    "weight_grad": ["grouped_ffn_bwd.cu", "gemm_common.cuh", "ptx.cuh"],
+}
+
+
+def kernel_source_digest(kind: str) -> str | None:
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kind]:
+        path = os.path.join(ROOT, "grouped_ffn_moe_b200", "csrc", name)
+        if not os.path.exists(path):
+            return None
+        h.update(open(path, "rb").read())
+    return h.hexdigest()
+
+
 def profiled_traffic(kernel_key: str):
     """DRAM bytes per launch of a kernel from the ncu summary in profiles/, if it was taken
-    on the current kernel source (the summary records the source's sha256); else None."""
-    import hashlib
-    import re
-
+    on the current kernel sources (the summary records their sha256); else None.
+    kernel_key is "<kind>/<workload>", kind a key of KERNEL_SOURCES."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "grouped_ffn_moe_b200", "csrc", "grouped_ffn.cu")
-    if not os.path.exists(path) or not os.path.exists(src):
+    if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(kernel_key)
-    if not rec:
-        return None
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    if rec.get("source_sha256") != digest:
+    if not rec or rec.get("source_sha256") != kernel_source_digest(kernel_key.split("/")[0]):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -278,6 +291,7 @@ def measure_backward(moe, synth, torch, w, inp, dev, steps, warmup, flush, peaks
                 "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = f"{peak_src} (burst)"
+    roof["traffic"] = profiled_traffic(f"{dom}/{w.name}")
     return {"tokens_per_s": w.S / ((ms["permute"] + ms["up_gate_train"] + ms["down_and_combine"]
                                     + bwd_ms) / 1e3),
             "ms_training_step": sum(ms.values()), "ms_backward": bwd_ms,

@@ -250,6 +250,10 @@ WORKLOADS: dict[str, Workload] = {
         # per-expert shape of "large" (171 rows per expert) on 32 experts: 2.8 GB of weights,
         # small enough for detailed profiler captures
         Workload("large_slice", 684, 7168, 2048, 32, 8, 2, "capped", 0.2),
+        # the same per-expert shape on 8 experts (K = E: every token visits each once); the
+        # training step's fp32 weight gradients stay at 1.4 GB, small enough for captures of
+        # the backward kernels
+        Workload("large_slice_e8", 171, 7168, 2048, 8, 8, 2, "uniform"),
     ]
     + [_c5(S, mv) for S in (1024, 4096, 16384, 65536) for mv in (0, 1, 20)]
 }
