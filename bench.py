@@ -43,6 +43,9 @@ def parse_args():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--zero-copy", action="store_true",
+                   help="forward step without x_perm: metadata-only permute, SwiGLU pass "
+                        "gathering its token rows from x (TMA gather4)")
     p.add_argument("--no-backward", action="store_true",
                    help="skip the training-step leg (forward with saved pre-activations + backward)")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -328,18 +331,25 @@ def run_ours(args):
     flush = torch.empty(256 << 18, dtype=torch.float32, device=dev)  # 256 MiB > 126 MB L2
     E = w.E
 
+    zero_copy = args.zero_copy and not w.identity_ffn
+
     def step(ev=None):
         if ev is not None:
             ev[0].record()
-        moe.moe_permute(inp["x"], inp["topk_ids"], E, buf.x_perm, buf.counts, buf.cu_seqlens,
-                        buf.row_id_map, buf.perm_src, buf.maxvio, buf.max_count, buf.workspace,
-                        buf.d_status)
+        moe.moe_permute(inp["x"], inp["topk_ids"], E, None if zero_copy else buf.x_perm,
+                        buf.counts, buf.cu_seqlens, buf.row_id_map, buf.perm_src, buf.maxvio,
+                        buf.max_count, buf.workspace, buf.d_status)
         if ev is not None:
             ev[1].record()
         y = buf.x_perm
         if not w.identity_ffn:
-            moe.moe_grouped_ffn_up_gate(buf.x_perm, inp["w_gate"], inp["w_up"], buf.cu_seqlens,
-                                        buf.h, buf.d_status)
+            if zero_copy:
+                moe.moe_grouped_ffn_up_gate_gather(inp["x"], buf.perm_src, w.K, inp["w_gate"],
+                                                   inp["w_up"], buf.cu_seqlens, buf.h,
+                                                   d_status=buf.d_status)
+            else:
+                moe.moe_grouped_ffn_up_gate(buf.x_perm, inp["w_gate"], inp["w_up"],
+                                            buf.cu_seqlens, buf.h, buf.d_status)
             if ev is not None:
                 ev[2].record()
             moe.moe_grouped_ffn_down(buf.h, inp["w_down"], buf.cu_seqlens, buf.y, buf.d_status)
@@ -352,8 +362,10 @@ def run_ours(args):
         if ev is not None:
             ev[4].record()
 
-    launches_per_step = moe.LAUNCHES["moe_permute"] + moe.LAUNCHES["moe_unpermute_combine"] + (
-        0 if w.identity_ffn else moe.LAUNCHES["moe_grouped_ffn"])
+    # the metadata-only permute (zero copy) launches one kernel, not the row copy
+    launches_per_step = (moe.LAUNCHES["moe_permute"] - (1 if zero_copy else 0)
+                         + moe.LAUNCHES["moe_unpermute_combine"]
+                         + (0 if w.identity_ffn else moe.LAUNCHES["moe_grouped_ffn"]))
 
     gpu_id = str(local)
     try:
@@ -422,7 +434,7 @@ def run_ours(args):
             dids.copy_(hids, non_blocking=True)
             dw.copy_(hw, non_blocking=True)
             out = moe.moe_layer_forward(dx, dids, dw, inp.get("w_gate"), inp.get("w_up"),
-                                        inp.get("w_down"), buf)
+                                        inp.get("w_down"), buf, zero_copy=zero_copy)
             hout.copy_(out, non_blocking=True)
 
         for _ in range(args.warmup):
@@ -494,6 +506,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded SplitMix64/Box-Muller inputs, random-init expert weights)",
             "config": {"workload": w.name, "S": w.S, "H": w.H, "Hp": w.Hp, "E": w.E, "K": w.K,
+                       "path": "zero-copy (gather)" if zero_copy else "x_perm copy",
                        "routing": w.routing, "maxvio_measured": maxvio,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed before every step (256 MiB write outside the timed events)"},

@@ -35,7 +35,8 @@ LAUNCHES = {"moe_permute": 2, "moe_grouped_ffn": 2, "moe_grouped_ffn_up_gate": 1
             "moe_combine_backward": 1, "moe_permute_backward": 1,
             "moe_grouped_ffn_up_gate_train": 1, "moe_grouped_ffn_down_backward": 1,
             "moe_grouped_ffn_up_gate_backward": 1, "moe_grouped_ffn_weight_grad": 1,
-            "moe_grouped_ffn_backward": 3}
+            "moe_grouped_ffn_backward": 3, "moe_grouped_ffn_gather": 2,
+            "moe_grouped_ffn_up_gate_gather": 1}
 
 
 class MoeError(RuntimeError):
@@ -88,6 +89,11 @@ def lib() -> ctypes.CDLL:
         L.moe_grouped_ffn_weight_grad.restype = i32
         L.moe_grouped_ffn_weight_grad.argtypes = [p, p, p, p, p, p, i64, i64, i64, i32, p, p, p,
                                                   i32, p, p]
+        L.moe_grouped_ffn_gather.restype = i32
+        L.moe_grouped_ffn_gather.argtypes = [p, p, i64, i32, p, p, p, p, i64, i64, i32, p, p, p, p]
+        L.moe_grouped_ffn_up_gate_gather.restype = i32
+        L.moe_grouped_ffn_up_gate_gather.argtypes = [p, p, i64, i32, p, p, p, i64, i64, i32, p, p,
+                                                     p, p, p]
         L.moe_grouped_ffn_backward.restype = i32
         L.moe_grouped_ffn_backward.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i32, p, p,
                                                p, p, p, p, p, i32, p, p]
@@ -260,6 +266,55 @@ def moe_grouped_ffn_down(h_scratch, w_down, cu_seqlens, y, d_status=None, stream
     st = lib().moe_grouped_ffn_down(_ptr(h_scratch), _ptr(w_down), _ptr(cu_seqlens), M, H, Hp, E,
                                     _ptr(y), _ptr(d_status), _stream(stream, dev))
     _check("moe_grouped_ffn_down", st)
+
+
+def _gather_check(x, perm_src, K, w_gate, w_up, cu_seqlens, h_scratch, d_status):
+    S, H = x.shape
+    M = S * K
+    Hp = h_scratch.shape[1]
+    E = cu_seqlens.numel() - 1
+    dev = x.device
+    _need_shape(x, "x", (S, H), torch.bfloat16, dev)
+    _need(perm_src, "perm_src", torch.int32, dev)
+    if perm_src.numel() != M:
+        raise ValueError(f"perm_src must have S*K = {M} entries")
+    _need_shape(h_scratch, "h_scratch", (M, Hp), torch.bfloat16, dev)
+    _need_shape(w_gate, "w_gate", (E, H, Hp), torch.bfloat16, dev)
+    _need_shape(w_up, "w_up", (E, H, Hp), torch.bfloat16, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(d_status, "d_status", torch.int32, dev)
+    return S, H, Hp, E, M, dev
+
+
+def moe_grouped_ffn_gather(x, perm_src, K, w_gate, w_up, w_down, cu_seqlens, h_scratch, y,
+                           d_status=None, stream=None):
+    """moe_grouped_ffn with the token rows gathered from the token-major x through perm_src
+    (no x_perm): the zero-copy path (see include/moe_b200.h)."""
+    S, H, Hp, E, M, dev = _gather_check(x, perm_src, K, w_gate, w_up, cu_seqlens, h_scratch,
+                                        d_status)
+    _need_shape(w_down, "w_down", (E, Hp, H), torch.bfloat16, dev)
+    _need_shape(y, "y", (M, H), torch.bfloat16, dev)
+    st = lib().moe_grouped_ffn_gather(_ptr(x), _ptr(perm_src), S, K, _ptr(w_gate), _ptr(w_up),
+                                      _ptr(w_down), _ptr(cu_seqlens), H, Hp, E, _ptr(h_scratch),
+                                      _ptr(y), _ptr(d_status), _stream(stream, dev))
+    _check("moe_grouped_ffn_gather", st)
+
+
+def moe_grouped_ffn_up_gate_gather(x, perm_src, K, w_gate, w_up, cu_seqlens, h_scratch,
+                                   gate_pre=None, up_pre=None, d_status=None, stream=None):
+    """First pass of moe_grouped_ffn_gather (optionally storing the pre-activations)."""
+    S, H, Hp, E, M, dev = _gather_check(x, perm_src, K, w_gate, w_up, cu_seqlens, h_scratch,
+                                        d_status)
+    if (gate_pre is None) != (up_pre is None):
+        raise ValueError("gate_pre and up_pre go together")
+    for t, n in ((gate_pre, "gate_pre"), (up_pre, "up_pre")):
+        if t is not None:
+            _need_shape(t, n, (M, Hp), torch.bfloat16, dev)
+    st = lib().moe_grouped_ffn_up_gate_gather(_ptr(x), _ptr(perm_src), S, K, _ptr(w_gate),
+                                              _ptr(w_up), _ptr(cu_seqlens), H, Hp, E,
+                                              _ptr(h_scratch), _ptr(gate_pre), _ptr(up_pre),
+                                              _ptr(d_status), _stream(stream, dev))
+    _check("moe_grouped_ffn_up_gate_gather", st)
 
 
 def moe_grouped_ffn_up_gate_train(x_perm, w_gate, w_up, cu_seqlens, h_scratch, gate_pre, up_pre,
@@ -482,12 +537,23 @@ class LayerBuffers:
             up_pre=torch.empty(M, Hp, **bf) if train else None)
 
 
-def moe_layer_forward(x, topk_ids, route_w, w_gate, w_up, w_down, buf: LayerBuffers, stream=None):
+def moe_layer_forward(x, topk_ids, route_w, w_gate, w_up, w_down, buf: LayerBuffers, stream=None,
+                      zero_copy: bool = False):
     """permute -> grouped FFN -> combine on one stream; returns buf.out.
 
     With w_gate None the experts are the identity (y = x_perm): permute/combine only.
+    zero_copy: the permutation computes the metadata only and the SwiGLU pass gathers its
+    token rows from x (same results, no x_perm; inference only).
     """
     E = buf.counts.numel()
+    if zero_copy and w_gate is not None and buf.gate_pre is None:
+        K = topk_ids.shape[1]
+        moe_permute(x, topk_ids, E, None, buf.counts, buf.cu_seqlens, buf.row_id_map,
+                    buf.perm_src, buf.maxvio, buf.max_count, buf.workspace, buf.d_status, stream)
+        moe_grouped_ffn_gather(x, buf.perm_src, K, w_gate, w_up, w_down, buf.cu_seqlens, buf.h,
+                               buf.y, buf.d_status, stream)
+        moe_unpermute_combine(buf.y, buf.row_id_map, route_w, buf.out, stream)
+        return buf.out
     moe_permute(x, topk_ids, E, buf.x_perm, buf.counts, buf.cu_seqlens, buf.row_id_map,
                 buf.perm_src, buf.maxvio, buf.max_count, buf.workspace, buf.d_status, stream)
     y = buf.x_perm

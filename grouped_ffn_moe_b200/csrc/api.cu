@@ -158,6 +158,52 @@ moe_status moe_grouped_ffn(const void* x_perm, const void* w_gate, const void* w
                               cuda_stream);
 }
 
+moe_status moe_grouped_ffn_up_gate_gather(const void* x, const int32_t* perm_src, int64_t S,
+                                          int32_t K, const void* w_gate, const void* w_up,
+                                          const int32_t* cu_seqlens, int64_t H, int64_t Hp,
+                                          int32_t E, void* h_scratch, void* gate_pre,
+                                          void* up_pre, int32_t* d_status, void* cuda_stream) {
+  if (S < 0 || K < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (S * K > moe::kMaxRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const int64_t M = S * K;
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  if ((gate_pre == nullptr) != (up_pre == nullptr)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!ok_ptr16(x) || perm_src == nullptr || !aligned(perm_src, 4) || !ok_ptr16(w_gate) ||
+      !ok_ptr16(w_up) || !ok_ptr16(h_scratch) || !aligned(gate_pre, 16) ||
+      !aligned(up_pre, 16) || cu_seqlens == nullptr || !aligned(cu_seqlens, 4) ||
+      !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M == 0) return MOE_OK;
+  return moe::launch_ffn_up_gate_gather(x, perm_src, S, K, w_gate, w_up, cu_seqlens, M, H, Hp, E,
+                                        h_scratch, gate_pre, up_pre, d_status,
+                                        static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_grouped_ffn_gather(const void* x, const int32_t* perm_src, int64_t S, int32_t K,
+                                  const void* w_gate, const void* w_up, const void* w_down,
+                                  const int32_t* cu_seqlens, int64_t H, int64_t Hp, int32_t E,
+                                  void* h_scratch, void* y, int32_t* d_status,
+                                  void* cuda_stream) {
+  if (S < 0 || K < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (S * K > moe::kMaxRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const int64_t M = S * K;
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  // validate both passes before launching either
+  if (!ok_ptr16(x) || perm_src == nullptr || !aligned(perm_src, 4) || !ok_ptr16(w_gate) ||
+      !ok_ptr16(w_up) || !ok_ptr16(w_down) || !ok_ptr16(h_scratch) || !ok_ptr16(y) ||
+      cu_seqlens == nullptr || !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M == 0) return MOE_OK;
+  const moe_status s1 =
+      moe_grouped_ffn_up_gate_gather(x, perm_src, S, K, w_gate, w_up, cu_seqlens, H, Hp, E,
+                                     h_scratch, nullptr, nullptr, d_status, cuda_stream);
+  if (s1 != MOE_OK) return s1;
+  return moe_grouped_ffn_down(h_scratch, w_down, cu_seqlens, M, H, Hp, E, y, d_status,
+                              cuda_stream);
+}
+
 moe_status moe_grouped_ffn_up_gate_train(const void* x_perm, const void* w_gate,
                                          const void* w_up, const int32_t* cu_seqlens, int64_t M,
                                          int64_t H, int64_t Hp, int32_t E, void* h_scratch,

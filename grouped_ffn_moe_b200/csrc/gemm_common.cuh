@@ -74,21 +74,22 @@ __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
   return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-// Block prologue, called by all kThreads threads: s_cu = cu_seqlens clamped to [0, M] (so
-// that no row outside [0, M) is ever addressed), s_ustart[e] = first unit of expert e with
-// ceil(rows / nmax) * nfb units per non-empty expert, s_ustart[E] = total units.
-// s_scan holds kThreads / 32 ints.
+// Block prologue, called by all kNT threads of the block: s_cu = cu_seqlens clamped to
+// [0, M] (so that no row outside [0, M) is ever addressed), s_ustart[e] = first unit of
+// expert e with ceil(rows / nmax) * nfb units per non-empty expert, s_ustart[E] = total
+// units. s_scan holds kNT / 32 ints.
+template <int kNT = kThreads>
 __device__ __forceinline__ void unit_starts(const int32_t* cu, int64_t M, int E, int nfb,
                                             int nmax, int32_t* s_cu, int32_t* s_ustart,
                                             int32_t* s_scan) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e <= E; e += kThreads) {
+  for (int e = tid; e <= E; e += kNT) {
     int64_t v = cu[e];
     v = v < 0 ? 0 : (v > M ? M : v);
     s_cu[e] = static_cast<int32_t>(v);
   }
   __syncthreads();
-  const int per = (E + kThreads - 1) / kThreads;  // <= 4 for E <= 1024
+  const int per = (E + kNT - 1) / kNT;  // <= 4 for E <= 1024
   const int beg = min(tid * per, E), end = min(beg + per, E);
   int local = 0;
   for (int e = beg; e < end; ++e) {
@@ -113,7 +114,7 @@ __device__ __forceinline__ void unit_starts(const int32_t* cu, int64_t M, int E,
     s_ustart[e] = run;
     run += units;
   }
-  if (tid == kThreads - 1) s_ustart[E] = off + incl;
+  if (tid == kNT - 1) s_ustart[E] = off + incl;
 }
 
 // ----------------------------------------------------------------------------- host side

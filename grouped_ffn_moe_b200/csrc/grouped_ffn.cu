@@ -45,15 +45,26 @@ namespace {
 
 // Kernel modes.
 //   kSwiGLU: A0 = W_gate, A1 = W_up on the same 128 features; h = silu(acc0) * acc1.
+//   kSwiGLUGather: kSwiGLU whose token tile is gathered straight from the token-major x
+//            (row r of the expert-grouped order is token perm_src[r] / K) by four extra
+//            gather warps' 16-byte cp.async copies into the same swizzled layout: the
+//            permutation's row copy x_perm is never materialised (the zero-copy fusion of the
+//            MoonEP README, "Zero-copy"). Measured alternatives: one TMA tile::gather4 per four
+//            rows (2.9x slower: the per-instruction cost set the pace) and cp.async from the
+//            producer warp alone (2.9x slower: one warp keeps too few copies in flight).
 //   kSingle: A0 = one 128-feature block; two TMEM accumulators double-buffered.
 //   kPair:   A0, A1 = two adjacent 128-feature blocks of one weight tensor sharing the token
 //            tile (half the token-row traffic per feature); y = acc0 | acc1.
-enum Mode : int { kSwiGLU = 0, kSingle = 1, kPair = 2 };
+enum Mode : int { kSwiGLU = 0, kSingle = 1, kPair = 2, kSwiGLUGather = 3 };
 
 template <int kMode>
 struct Cfg {
+  static constexpr bool kSwi = kMode == kSwiGLU || kMode == kSwiGLUGather;
+  // gather: four more warps (10-13) copy the token rows
+  static constexpr int kGatherWarps = kMode == kSwiGLUGather ? 4 : 0;
+  static constexpr int kBlock = kThreads + 32 * kGatherWarps;
   static constexpr int kNumA = kMode == kSingle ? 1 : 2;
-  static constexpr int kNMaxMode = kMode == kSwiGLU ? MOE_SWIGLU_NMAX : kNMax;
+  static constexpr int kNMaxMode = kSwi ? MOE_SWIGLU_NMAX : kNMax;
   // accumulator stages: two when they fit in TMEM (kSingle; kSwiGLU with N <= 128)
   static constexpr int kAccStages = (kMode == kSingle || kNMaxMode <= 128) ? 2 : 1;
   static constexpr int kUpOff = kAccStages == 2 ? kNMaxMode : 256;  // up accumulator column
@@ -67,9 +78,10 @@ struct Cfg {
   static constexpr int kOffBars = (kOffUnits + 4 * (MOE_MAX_EXPERTS + 1) + 7) & ~7;
   static constexpr int kNumBars = 2 * kStages + 2 * 2 + 1;
   static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+  static constexpr int kSmemBytes = kOffMisc + 128 + 1024;  // + alignment slack
 };
 static_assert(Cfg<kSwiGLU>::kSmemBytes <= 232448, "shared memory budget (SwiGLU)");
+static_assert(Cfg<kSwiGLUGather>::kSmemBytes == Cfg<kSwiGLU>::kSmemBytes, "gather layout");
 static_assert(Cfg<kSingle>::kSmemBytes <= 232448, "shared memory budget (single)");
 static_assert(Cfg<kPair>::kSmemBytes <= 232448, "shared memory budget (pair)");
 
@@ -84,10 +96,14 @@ struct FfnArgs {
   uint64_t budget_ns;
   __nv_bfloat16* gate_pre;  // [M, H'] bf16(x.W_gate), pass 1 when training; else null
   __nv_bfloat16* up_pre;    // [M, H'] bf16(x.W_up), with gate_pre
+  const int32_t* perm_src;  // kSwiGLUGather: [M] flat slot of each row; token = slot / route_k
+  int32_t route_k;          // kSwiGLUGather: K
+  const __nv_bfloat16* x;   // kSwiGLUGather: token-major [S, k_dim]
+  int64_t S;                // kSwiGLUGather: rows of x
 };
 
 template <int kMode>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<kMode>::kBlock, 1)
     grouped_ffn_kernel(const __grid_constant__ CUtensorMap tmA0,
                        const __grid_constant__ CUtensorMap tmA1,
                        const __grid_constant__ RowMaps tmB, const FfnArgs args) {
@@ -106,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
-  int32_t* s_scan = reinterpret_cast<int32_t*>(smem + C::kOffMisc + 8);  // [10]
+  int32_t* s_scan = reinterpret_cast<int32_t*>(smem + C::kOffMisc + 8);  // [kBlock / 32]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = args.E;
@@ -116,7 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------------ prologue
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      // gather: the weight loads' arrive.expect_tx plus one cp.async arrival per gather lane
+      mbar_init(&full[s], 1 + 32 * C::kGatherWarps);
       mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -129,8 +146,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&tmA0);
-    if (kMode == kSwiGLU) tma_prefetch_map(&tmA1);
-    for (int i = 0; i < kNumBoxHeights; ++i) tma_prefetch_map(&tmB.m[i]);
+    if (C::kSwi) tma_prefetch_map(&tmA1);
+    if (kMode != kSwiGLUGather)  // gather mode reads no token-row map
+      for (int i = 0; i < kNumBoxHeights; ++i) tma_prefetch_map(&tmB.m[i]);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, kTmemCols);
@@ -140,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // cu_seqlens and the activations come from earlier kernels in the stream
   griddep_wait();
   griddep_launch_dependents();
-  unit_starts(args.cu, args.M, E, nfb, C::kNMaxMode, s_cu, s_ustart, s_scan);
+  unit_starts<C::kBlock>(args.cu, args.M, E, nfb, C::kNMaxMode, s_cu, s_ustart, s_scan);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -148,7 +166,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total_units = s_ustart[E];
 
   // ------------------------------------------------------------------ roles
-  if (warp == 0) {
+  if (kMode == kSwiGLUGather && warp >= 2 + kEpiThreads / 32) {
+    // Gather warps g = 0..3. Per unit each lane loads the tokens of its 16 rows,
+    // r = 16i + 4g + (lane >> 3), into registers (rows past the unit, up to the 16-row
+    // rounding, repeat its last row; their MMA columns are never stored). Per stage, after
+    // the slot is free, lane (8 * row-in-group + piece) copies 16-byte piece `piece` of its
+    // row's 128-byte segment with cp.async into the 128-byte-swizzled K-major token tile
+    // (piece c of row r at r*128 + ((c ^ (r % 8)) * 16)) and arrives when its copies land.
+    const int g = warp - (2 + kEpiThreads / 32);
+    const int piece = lane & 7;
+    const int rsub = lane >> 3;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool stop = false;
+    for (int u = blockIdx.x; u < total_units && !stop; u += gridDim.x) {
+      if (__shfl_sync(0xffffffffu, *s_abort, 0)) break;  // lane 0's view: a uniform exit
+      const Unit U = decode_unit<C::kNMaxMode>(u, s_ustart, s_cu, E);
+      if (U.nrows <= 0) continue;
+      const int n = (U.nrows + 15) & ~15;
+      int tok[C::kNMaxMode / 16];
+#pragma unroll
+      for (int i = 0; i < C::kNMaxMode / 16; ++i) {
+        const int r = min(16 * i + 4 * g + rsub, U.nrows - 1);
+        int64_t t = __ldg(args.perm_src + U.row0 + r) / args.route_k;
+        t = t < 0 ? 0 : (t >= args.S ? args.S - 1 : t);  // any perm_src stays inside x
+        tok[i] = static_cast<int32_t>(t);
+      }
+      for (int kt = 0; kt < KT; ++kt) {
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, s_abort, args.budget_ns);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          stop = true;
+          break;
+        }
+        const uint32_t sb = smem_u32(smem + stage * C::kStageBytes + C::kNumA * kABytes);
+        const __nv_bfloat16* xk = args.x + kt * kBK + piece * 8;
+#pragma unroll
+        for (int i = 0; i < C::kNMaxMode / 16; ++i) {
+          if (16 * i < n) {  // uniform
+            const int r = 16 * i + 4 * g + rsub;
+            cp_async_16(sb + r * kRowBytes + ((piece ^ (r & 7)) << 4),
+                        xk + static_cast<int64_t>(tok[i]) * args.k_dim);
+          }
+        }
+        cp_async_mbar_arrive_noinc(&full[stage]);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // own copies land before the CTA exits
+  } else if (warp == 0) {
     // TMA producer
     if (lane == 0) {
       const uint64_t pol_stream = policy_evict_first();  // weights read by one unit only
@@ -161,7 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit U = decode_unit<C::kNMaxMode>(u, s_ustart, s_cu, E);
         if (U.nrows <= 0) continue;
         const int n = (U.nrows + 15) & ~15;
-        const uint32_t bytes = C::kNumA * kABytes + n * kRowBytes;
+        // gather: the token rows arrive by the gather warps' cp.async, not by TMA
+        const uint32_t bytes = C::kNumA * kABytes + (kMode == kSwiGLUGather ? 0 : n * kRowBytes);
         const uint64_t pol_w = U.ntc > 1 ? pol_keep : pol_stream;
         const int fz = U.fb * (C::kFeatPerUnit / 64);  // 64-feature index of the first feature
         for (int kt = 0; kt < KT; ++kt) {
@@ -170,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int ky = U.e * args.k_dim + kt * kBK;
           mbar_arrive_expect_tx(&full[stage], bytes);
           tma_load_3d_hint(st, &tmA0, &full[stage], 0, ky, fz, pol_w);
-          if (kMode == kSwiGLU) tma_load_3d_hint(st + kABytes, &tmA1, &full[stage], 0, ky, fz, pol_w);
+          if (C::kSwi) tma_load_3d_hint(st + kABytes, &tmA1, &full[stage], 0, ky, fz, pol_w);
           // second block of a pair; past the last feature the box is zero-filled (not stored)
           if (kMode == kPair) tma_load_3d_hint(st + kABytes, &tmA0, &full[stage], 0, ky, fz + 2, pol_w);
           uint8_t* sb = st + C::kNumA * kABytes;
@@ -178,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kNumBoxHeights; ++i) {
             const int h = kNMax >> i;
-            if (n & h) {
+            if (kMode != kSwiGLUGather && (n & h)) {
               tma_load_2d_hint(sb + r * kRowBytes, &tmB.m[i], &full[stage], kt * kBK, U.row0 + r,
                                pol_keep);
               r += h;
@@ -216,13 +286,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait_bounded(&tempty[astage], aphase ^ 1u, s_abort, args.budget_ns)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + astage * kAccCols;  // astage is 0 with one stage
-        const uint32_t d1 = d0 + (kMode == kSwiGLU ? C::kUpOff : kAccCols);
+        const uint32_t d1 = d0 + (C::kSwi ? C::kUpOff : kAccCols);
         bool ok = true;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait_bounded(&full[stage], phase, s_abort, args.budget_ns)) {
             ok = false;
             break;
           }
+          // gather: the token rows were written by cp.async (generic proxy)
+          if (kMode == kSwiGLUGather) fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
           const uint32_t a1 = a0 + kABytes;
@@ -303,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           };
           uint32_t r0[32], r1[32];
           tmem_ld_32x32b_x32(tbase + half * kAccCols + c, r0);
-          if (kMode == kSwiGLU) {
+          if (C::kSwi) {
             tmem_ld_32x32b_x32(tbase + C::kUpOff + c, r1);
             tmem_ld_wait();
 #pragma unroll
@@ -321,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               so[j * kBM + f_local] = __float2bfloat16_rn(__uint_as_float(r0[j]));
           }
           store_chunk(args.out);
-          if (kMode == kSwiGLU && args.gate_pre != nullptr) {
+          if (C::kSwi && args.gate_pre != nullptr) {
             // training: the pre-activations, each rounded once from the fp32 accumulator
 #pragma unroll
             for (int j = 0; j < 32; ++j)
@@ -705,6 +777,30 @@ int down_mode() {
 
 }  // namespace
 
+moe_status launch_ffn_up_gate_gather(const void* x, const int32_t* perm_src, int64_t S, int32_t K,
+                                     const void* w_gate, const void* w_up,
+                                     const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp,
+                                     int32_t E, void* h, void* gate_pre, void* up_pre,
+                                     int32_t* d_status, cudaStream_t stream) {
+  CUtensorMap m_wg, m_wu;
+  RowMaps m_x = {};
+  // token rows come by cp.async from x itself: the row-map table is unused in this mode
+  if (!make_weight_map(&m_wg, w_gate, Hp, static_cast<uint64_t>(E) * H) ||
+      !make_weight_map(&m_wu, w_up, Hp, static_cast<uint64_t>(E) * H) ||
+      !ensure_smem_attr<kSwiGLUGather>())
+    return MOE_ERR_CUDA;
+  const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(h), d_status, M, E,
+                  static_cast<int32_t>(H), static_cast<int32_t>(Hp), wait_budget_ns(),
+                  static_cast<__nv_bfloat16*>(gate_pre), static_cast<__nv_bfloat16*>(up_pre),
+                  perm_src, K, static_cast<const __nv_bfloat16*>(x), S};
+  const cudaError_t err =
+      launch_dependent(grouped_ffn_kernel<kSwiGLUGather>, dim3(num_sms()),
+                       dim3(Cfg<kSwiGLUGather>::kBlock),
+                       Cfg<kSwiGLUGather>::kSmemBytes, stream, m_wg, m_wu, m_x, a);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const void* w1,
                            const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp, int32_t E,
                            void* out, void* gate_pre, void* up_pre, int32_t* d_status,
@@ -722,7 +818,8 @@ moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const voi
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
                     static_cast<int32_t>(H), static_cast<int32_t>(Hp), wait_budget_ns(),
-                    static_cast<__nv_bfloat16*>(gate_pre), static_cast<__nv_bfloat16*>(up_pre)};
+                    static_cast<__nv_bfloat16*>(gate_pre), static_cast<__nv_bfloat16*>(up_pre),
+                    nullptr, 1, nullptr, 0};
     const cudaError_t err =
         pair
             ? launch_swiglu_pair(m_wg, m_wu, m_x, a, stream)
@@ -739,7 +836,7 @@ moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const voi
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
                     static_cast<int32_t>(Hp), static_cast<int32_t>(H), wait_budget_ns(),
-                    nullptr, nullptr};
+                    nullptr, nullptr, nullptr, 1, nullptr, 0};
     const cudaError_t err =
         pair ? launch_dependent(grouped_ffn_kernel<kPair>, dim3(grid), dim3(kThreads),
                                 Cfg<kPair>::kSmemBytes, stream, m_wd, m_wd, m_h, a)

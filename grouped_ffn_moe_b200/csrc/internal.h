@@ -72,6 +72,15 @@ moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const voi
                            void* out, void* gate_pre, void* up_pre, int32_t* d_status,
                            cudaStream_t stream);
 
+// The SwiGLU pass with its token rows gathered from the token-major x [S, H] (row r of the
+// expert-grouped order is token perm_src[r] / K): h, and gate_pre/up_pre when non-null, as
+// launch_ffn_pass(dual) on x_perm would produce them, without x_perm.
+moe_status launch_ffn_up_gate_gather(const void* x, const int32_t* perm_src, int64_t S, int32_t K,
+                                     const void* w_gate, const void* w_up,
+                                     const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp,
+                                     int32_t E, void* h, void* gate_pre, void* up_pre,
+                                     int32_t* d_status, cudaStream_t stream);
+
 // Backward of the down projection fused with the SwiGLU backward: from grad_y [M,H] and the
 // saved pre-activations [M,H'], d_gate and d_up [M,H'] (bf16).
 moe_status launch_ffn_down_backward(const void* grad_y, const void* w_down, const void* gate_pre,

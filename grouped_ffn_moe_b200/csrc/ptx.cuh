@@ -92,6 +92,21 @@ __device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// 16-byte asynchronous global -> shared copy (L2 only, no L1 allocation). The data is written
+// through the generic proxy: a consumer reading it with tcgen05.mma must fence
+// (fence_proxy_async_smem) after observing its completion.
+__device__ __forceinline__ void cp_async_16(uint32_t smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gmem_src)
+               : "memory");
+}
+
+// Arrive on `bar` once all of this thread's prior cp.async copies have landed; the arrival
+// counts toward the barrier's expected count (.noinc).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
 // 2-D tiled bulk tensor store shared -> global (bulk-group completion); x innermost, both
 // coordinates non-negative and inside the tensor.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src,

@@ -173,6 +173,32 @@ moe_status moe_grouped_ffn_down(const void* h_scratch, const void* w_down,
                                 int32_t E, void* y, int32_t* d_status, void* cuda_stream);
 
 /*
+ * moe_grouped_ffn_gather - moe_grouped_ffn without the permuted copy x_perm: the SwiGLU pass
+ * reads each row's token straight from the token-major x (the zero-copy fusion of the MoonEP
+ * README, "Zero-copy": experts read the dispatched rows in place). Row r of the
+ * expert-grouped order is token perm_src[r] / K, so with perm_src and cu_seqlens from
+ * moe_permute (which may then be called with x_perm = NULL) the results h and y equal those
+ * of moe_grouped_ffn on the x_perm that moe_permute would have written, bit for bit.
+ *   x         [S, H] bf16, token-major (16-byte aligned).
+ *   perm_src  device [S*K] int32 from moe_permute; M = S*K rows.
+ * Other arguments, requirements and errors as moe_grouped_ffn.
+ *
+ * moe_grouped_ffn_up_gate_gather is its first pass alone; gate_pre and up_pre (both NULL or
+ * both [M, Hp] bf16) also store the pre-activations as moe_grouped_ffn_up_gate_train does.
+ */
+moe_status moe_grouped_ffn_gather(const void* x, const int32_t* perm_src, int64_t S, int32_t K,
+                                  const void* w_gate, const void* w_up, const void* w_down,
+                                  const int32_t* cu_seqlens, int64_t H, int64_t Hp, int32_t E,
+                                  void* h_scratch, void* y, int32_t* d_status,
+                                  void* cuda_stream);
+
+moe_status moe_grouped_ffn_up_gate_gather(const void* x, const int32_t* perm_src, int64_t S,
+                                          int32_t K, const void* w_gate, const void* w_up,
+                                          const int32_t* cu_seqlens, int64_t H, int64_t Hp,
+                                          int32_t E, void* h_scratch, void* gate_pre,
+                                          void* up_pre, int32_t* d_status, void* cuda_stream);
+
+/*
  * moe_grouped_ffn_up_gate_train - moe_grouped_ffn_up_gate for training: the same h, plus the
  * pre-activations the backward differentiates SwiGLU at, each rounded once to bf16 from the
  * fp32 accumulator:

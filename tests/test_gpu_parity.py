@@ -555,3 +555,76 @@ def test_backward_unit_weight_and_adjoint_exactness(cuda_device):
     torch.cuda.synchronize()
     assert torch.equal(grad_y, buf.x_perm)  # w = 1: the backward re-dispatch is the permutation
     assert torch.equal(grad_x, (x.float() * K).to(torch.bfloat16))
+
+
+# ----------------------------------------------------------------------------- zero copy
+
+def _gather_vs_copy(inp, w, dev):
+    ref = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev)
+    moe.moe_layer_forward(inp["x"], inp["topk_ids"], inp["route_w"], inp["w_gate"], inp["w_up"],
+                          inp["w_down"], ref)
+    zc = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev)
+    zc.x_perm.fill_(float("nan"))  # the zero-copy path must not read x_perm
+    moe.moe_layer_forward(inp["x"], inp["topk_ids"], inp["route_w"], inp["w_gate"], inp["w_up"],
+                          inp["w_down"], zc, zero_copy=True)
+    torch.cuda.synchronize()
+    assert int(ref.d_status.item()) == 0 and int(zc.d_status.item()) == 0
+    assert torch.isnan(zc.x_perm.float()).all()  # metadata-only permute: no row copy
+    for name in ("counts", "cu_seqlens", "row_id_map", "perm_src", "h", "y", "out"):
+        assert torch.equal(getattr(zc, name), getattr(ref, name)), name
+    return ref, zc
+
+
+@pytest.mark.parametrize("wname", ["tiny", "medium", "large", "skew20"])
+def test_zero_copy_gather_equals_copy_path(cuda_device, wname):
+    """The SwiGLU pass gathering its token rows from x through perm_src (TMA tile::gather4)
+    gives h, y and out bit-identical to the path through x_perm, which is itself checked
+    against the oracle above; the tiny layer is also checked against the oracle directly."""
+    w = synth.WORKLOADS[wname]
+    inp = layer_inputs(w, cuda_device)
+    ref, zc = _gather_vs_copy(inp, w, cuda_device)
+    if wname == "tiny":
+        zc.x_perm.copy_(ref.x_perm)  # the oracle check also compares the (unused) x_perm
+        _check_full_layer(inp, w, zc)
+
+
+@pytest.mark.parametrize("H,Hp", [(256, 384), (384, 256)])
+def test_zero_copy_gather_ragged(cuda_device, H, Hp):
+    """Experts of 0 .. 1100 rows (every chunk and 16-row rounding path), K = 2 with
+    duplicate experts inside tokens, against the copy path."""
+    sizes = [0, 1, 15, 16, 17, 255, 256, 257, 600, 1100]
+    E, K = len(sizes), 2
+    ids_np = np.concatenate([np.full(n, e, np.int32) for e, n in enumerate(sizes)])
+    ids_np = np.random.default_rng(12).permutation(ids_np)
+    if len(ids_np) % 2:
+        ids_np = ids_np[:-1]
+    ids_np = ids_np.reshape(-1, K)
+    S = ids_np.shape[0]
+    w = synth.Workload("ragged_k2", S, H, Hp, E, K, 23)
+    inp = {"topk_ids": torch.from_numpy(ids_np).to(cuda_device),
+           "route_w": torch.full((S, K), 0.5, dtype=torch.float32, device=cuda_device)}
+    inp["x"] = synth.normal_bf16_into(torch.empty(S, H, dtype=torch.bfloat16, device=cuda_device),
+                                      23, synth.TAG_X)
+    for name, tag, shape in (("w_gate", synth.TAG_W_GATE, (E, H, Hp)),
+                             ("w_up", synth.TAG_W_UP, (E, H, Hp)),
+                             ("w_down", synth.TAG_W_DOWN, (E, Hp, H))):
+        inp[name] = synth.normal_bf16_into(torch.empty(*shape, dtype=torch.bfloat16,
+                                                       device=cuda_device), 23, tag,
+                                           synth.weight_scale(w, name[2:]))
+    _gather_vs_copy(inp, w, cuda_device)
+
+
+def test_zero_copy_gather_training_preactivations(cuda_device):
+    """The gather pass stores the same pre-activations as the training forward on x_perm."""
+    w = synth.WORKLOADS["medium"]
+    inp = layer_inputs(w, cuda_device)
+    buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, cuda_device, train=True)
+    moe.moe_layer_forward(inp["x"], inp["topk_ids"], inp["route_w"], inp["w_gate"], inp["w_up"],
+                          inp["w_down"], buf)
+    h2 = torch.empty_like(buf.h)
+    g2, u2 = torch.empty_like(buf.gate_pre), torch.empty_like(buf.up_pre)
+    moe.moe_grouped_ffn_up_gate_gather(inp["x"], buf.perm_src, w.K, inp["w_gate"], inp["w_up"],
+                                       buf.cu_seqlens, h2, g2, u2, buf.d_status)
+    torch.cuda.synchronize()
+    assert int(buf.d_status.item()) == 0
+    assert torch.equal(h2, buf.h) and torch.equal(g2, buf.gate_pre) and torch.equal(u2, buf.up_pre)
