@@ -380,6 +380,25 @@ def moe_layer(x_bits: np.ndarray, topk_ids: np.ndarray, route_w: np.ndarray, E: 
                 max_count=mc, x_perm=x_perm, h=h, y=y, out=out)
 
 
+def moe_layer_with_shared(x_bits: np.ndarray, topk_ids: np.ndarray, route_w: np.ndarray, E: int,
+                          get_weights, Hp: int, shared_weights):
+    """MoE(x) = SharedExpert(x) + sum over the top-k of router_weight_k * RoutedExpert_k(x)
+    ("Mixture of Kittens" digest, Step 1, The Math). The shared expert is one SwiGLU FFN
+    (shared_weights = (Wg_s [H,Hs], Wu_s [H,Hs], Wd_s [Hs,H]) bf16 bits) applied to every
+    token; its output y_shared is a stored bf16 tensor like every expert output, and
+    out[t] = bf16(y_shared[t] + sum_k w[t,k] * y[r(t,k)]) with one rounding.
+    Returns moe_layer's dict with y_shared added and out replaced."""
+    S, K = np.asarray(topk_ids).shape
+    base = moe_layer(x_bits, topk_ids, route_w, E, get_weights, Hp)
+    _, ys = expert_ffn_rows(x_bits, *shared_weights)
+    rmap = np.asarray(base["row_id_map"], dtype=np.int64).reshape(S, K)
+    w = np.asarray(route_w, dtype=np.float32).astype(np.float64).reshape(S, K)
+    acc = bf16_bits_to_f64(ys).copy()
+    for k in range(K):
+        acc += w[:, k:k + 1] * bf16_bits_to_f64(base["y"][rmap[:, k]])
+    return dict(base, y_shared=ys, out=f64_to_bf16_bits(acc))
+
+
 def direct_expert_loop(x_bits: np.ndarray, topk_ids: np.ndarray, route_w: np.ndarray, get_weights):
     """The same layer without any permutation: for every token, run each of its K
     experts on the token's own row and add the weighted results ("Distributed expert parallelism", Exercises, item 3).

@@ -542,3 +542,33 @@ def test_preactivations_against_torch():
     tx = torch_bf16_of(x).double()
     np.testing.assert_array_equal(g, bits_of((tx @ torch_bf16_of(wg).double()).to(torch.bfloat16)))
     np.testing.assert_array_equal(u, bits_of((tx @ torch_bf16_of(wu).double()).to(torch.bfloat16)))
+
+
+# ----------------------------------------------------------------------------- shared expert
+
+
+def test_shared_expert_layer_against_direct_loop_and_dense_ffn():
+    """The layer with a shared expert equals a per-token loop that runs the shared FFN and the
+    token's K experts on its own row and sums them in one rounding; with zero route weights
+    it is the dense SwiGLU FFN of the shared weights (torch float64)."""
+    rng = np.random.default_rng(51)
+    S, H, Hp, Hs, E, K = 9, 16, 24, 40, 4, 2
+    x, wg, wu, wd, ids, w = _rand_layer(rng, S, H, Hp, E, K)
+    get = _weights_getter(wg, wu, wd)
+    sh = (O.f64_to_bf16_bits(rng.standard_normal((H, Hs)) / 4),
+          O.f64_to_bf16_bits(rng.standard_normal((H, Hs)) / 4),
+          O.f64_to_bf16_bits(rng.standard_normal((Hs, H)) / 6))
+    res = O.moe_layer_with_shared(x, ids, w, E, get, Hp, sh)
+    f = O.bf16_bits_to_f64
+    for t in range(S):
+        acc = f(O.expert_ffn_rows(x[t:t + 1], *sh)[1])[0].copy()
+        for k in range(K):
+            acc += float(w[t, k]) * f(O.expert_ffn_rows(x[t:t + 1], *get(int(ids[t, k])))[1])[0]
+        np.testing.assert_array_equal(res["out"][t], O.f64_to_bf16_bits(acc))
+    zero = O.moe_layer_with_shared(x, ids, np.zeros_like(w), E, get, Hp, sh)
+    tx = torch.tensor(f(x))
+    g = tx @ torch.tensor(f(sh[0]))
+    u = tx @ torch.tensor(f(sh[1]))
+    hh = torch.tensor(f(O.f64_to_bf16_bits((torch.nn.functional.silu(g) * u).numpy())))
+    dense = (hh @ torch.tensor(f(sh[2]))).numpy()
+    np.testing.assert_array_equal(zero["out"], O.f64_to_bf16_bits(dense))
