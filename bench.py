@@ -16,6 +16,7 @@ Prints one JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -46,6 +47,9 @@ def parse_args():
     p.add_argument("--zero-copy", action="store_true",
                    help="forward step without x_perm: metadata-only permute, SwiGLU pass "
                         "gathering its token rows from x (TMA gather4)")
+    p.add_argument("--shared-experts", type=int, default=0,
+                   help="append N shared experts (each with the routed experts' shape) to the "
+                        "routing and run them in the same launches (no e2e or training leg)")
     p.add_argument("--no-backward", action="store_true",
                    help="skip the training-step leg (forward with saved pre-activations + backward)")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -326,17 +330,26 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = synth.WORKLOADS[args.workload]
-    inp = synth.make_layer_inputs(w, device=str(dev))
-    buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev, with_ffn=not w.identity_ffn)
+    ns = args.shared_experts if not w.identity_ffn else 0
+    inp = synth.make_layer_inputs(w, device=str(dev), n_shared=ns)
+    E, K = w.E + ns, w.K + ns  # shared experts are experts E.. with one slot each per token
+    buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, E, K, dev, with_ffn=not w.identity_ffn)
     flush = torch.empty(256 << 18, dtype=torch.float32, device=dev)  # 256 MiB > 126 MB L2
-    E = w.E
+    if ns:
+        ids_ext = torch.empty(w.S, K, dtype=torch.int32, device=dev)
+        w_ext = torch.empty(w.S, K, dtype=torch.float32, device=dev)
+        routed_mv = torch.empty(1, dtype=torch.float64, device=dev)
+    ids_step = ids_ext if ns else inp["topk_ids"]
+    w_step = w_ext if ns else inp["route_w"]
 
     zero_copy = args.zero_copy and not w.identity_ffn
 
     def step(ev=None):
         if ev is not None:
             ev[0].record()
-        moe.moe_permute(inp["x"], inp["topk_ids"], E, None if zero_copy else buf.x_perm,
+        if ns:
+            moe.moe_append_shared(inp["topk_ids"], inp["route_w"], w.E, ns, ids_ext, w_ext)
+        moe.moe_permute(inp["x"], ids_step, E, None if zero_copy else buf.x_perm,
                         buf.counts, buf.cu_seqlens, buf.row_id_map, buf.perm_src, buf.maxvio,
                         buf.max_count, buf.workspace, buf.d_status)
         if ev is not None:
@@ -344,7 +357,7 @@ def run_ours(args):
         y = buf.x_perm
         if not w.identity_ffn:
             if zero_copy:
-                moe.moe_grouped_ffn_up_gate_gather(inp["x"], buf.perm_src, w.K, inp["w_gate"],
+                moe.moe_grouped_ffn_up_gate_gather(inp["x"], buf.perm_src, K, inp["w_gate"],
                                                    inp["w_up"], buf.cu_seqlens, buf.h,
                                                    d_status=buf.d_status)
             else:
@@ -358,14 +371,18 @@ def run_ours(args):
             ev[2].record()
         if ev is not None:
             ev[3].record()
-        moe.moe_unpermute_combine(y, buf.row_id_map, inp["route_w"], buf.out)
+        moe.moe_unpermute_combine(y, buf.row_id_map, w_step, buf.out)
+        if ns:  # the routed experts' imbalance
+            moe.moe_maxvio(buf.counts[:w.E], w.S, w.K, routed_mv)
         if ev is not None:
             ev[4].record()
 
     # the metadata-only permute (zero copy) launches one kernel, not the row copy
     launches_per_step = (moe.LAUNCHES["moe_permute"] - (1 if zero_copy else 0)
                          + moe.LAUNCHES["moe_unpermute_combine"]
-                         + (0 if w.identity_ffn else moe.LAUNCHES["moe_grouped_ffn"]))
+                         + (0 if w.identity_ffn else moe.LAUNCHES["moe_grouped_ffn"])
+                         + (moe.LAUNCHES["moe_append_shared"] + moe.LAUNCHES["moe_maxvio"]
+                            if ns else 0))
 
     gpu_id = str(local)
     try:
@@ -417,11 +434,11 @@ def run_ours(args):
     mean = {k: sum(v) / len(v) for k, v in per.items()}
     status = int(buf.d_status.item())
     counts = buf.counts.cpu().numpy()
-    maxvio = float(buf.maxvio.item())
+    maxvio = float((routed_mv if ns else buf.maxvio).item())
 
     # e2e: host (pinned) inputs -> device -> layer -> host output, every step
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not ns:
         hx = inp["x"].cpu().pin_memory()
         hids = inp["topk_ids"].cpu().pin_memory()
         hw = inp["route_w"].cpu().pin_memory()
@@ -457,7 +474,7 @@ def run_ours(args):
             raise RuntimeError("e2e output differs from the device-resident run")
 
     backward = None
-    if not w.identity_ffn and not args.no_backward:
+    if not w.identity_ffn and not args.no_backward and not ns:
         peaks0, src0 = load_peaks()
         backward = measure_backward(moe, synth, torch, w, inp, dev, args.steps, args.warmup, flush,
                                     peaks0, src0)
@@ -467,7 +484,7 @@ def run_ours(args):
 
     if rank == 0:
         peaks, peak_src = load_peaks()
-        wm = work_model(w, counts)
+        wm = work_model(dataclasses.replace(w, E=E, K=K), counts)
         stages = {
             "permute": {"ms": mean["permute"],
                         "GB/s": wm["permute_bytes"] / (mean["permute"] / 1e3) / 1e9},
@@ -507,6 +524,7 @@ def run_ours(args):
             "data": "synthetic (seeded SplitMix64/Box-Muller inputs, random-init expert weights)",
             "config": {"workload": w.name, "S": w.S, "H": w.H, "Hp": w.Hp, "E": w.E, "K": w.K,
                        "path": "zero-copy (gather)" if zero_copy else "x_perm copy",
+                       "shared_experts": ns,
                        "routing": w.routing, "maxvio_measured": maxvio,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed before every step (256 MiB write outside the timed events)"},

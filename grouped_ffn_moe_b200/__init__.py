@@ -36,7 +36,7 @@ LAUNCHES = {"moe_permute": 2, "moe_grouped_ffn": 2, "moe_grouped_ffn_up_gate": 1
             "moe_grouped_ffn_up_gate_train": 1, "moe_grouped_ffn_down_backward": 1,
             "moe_grouped_ffn_up_gate_backward": 1, "moe_grouped_ffn_weight_grad": 1,
             "moe_grouped_ffn_backward": 3, "moe_grouped_ffn_gather": 2,
-            "moe_grouped_ffn_up_gate_gather": 1}
+            "moe_grouped_ffn_up_gate_gather": 1, "moe_append_shared": 1}
 
 
 class MoeError(RuntimeError):
@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
         L.moe_grouped_ffn_up_gate_gather.restype = i32
         L.moe_grouped_ffn_up_gate_gather.argtypes = [p, p, i64, i32, p, p, p, i64, i64, i32, p, p,
                                                      p, p, p]
+        L.moe_append_shared.restype = i32
+        L.moe_append_shared.argtypes = [p, p, i64, i32, i32, i32, p, p, p]
         L.moe_grouped_ffn_backward.restype = i32
         L.moe_grouped_ffn_backward.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i32, p, p,
                                                p, p, p, p, p, i32, p, p]
@@ -483,6 +485,20 @@ def moe_permute_backward(grad_x_perm, row_id_map, grad_x, K, stream=None):
     st = lib().moe_permute_backward(_ptr(grad_x_perm), _ptr(row_id_map), S, H, K, _ptr(grad_x),
                                     _stream(stream, dev))
     _check("moe_permute_backward", st)
+
+
+def moe_append_shared(topk_ids, route_w, E, n_shared, ids_out, w_out, stream=None):
+    """Routing with n_shared shared experts appended (experts E .. E+n_shared-1, weight 1 in
+    slots K .. K+n_shared-1; see include/moe_b200.h)."""
+    S, K = topk_ids.shape
+    dev = topk_ids.device
+    _need_shape(topk_ids, "topk_ids", (S, K), torch.int32, dev)
+    _need_shape(route_w, "route_w", (S, K), torch.float32, dev)
+    _need_shape(ids_out, "ids_out", (S, K + n_shared), torch.int32, dev)
+    _need_shape(w_out, "w_out", (S, K + n_shared), torch.float32, dev)
+    st = lib().moe_append_shared(_ptr(topk_ids), _ptr(route_w), S, K, E, n_shared, _ptr(ids_out),
+                                 _ptr(w_out), _stream(stream, dev))
+    _check("moe_append_shared", st)
 
 
 def moe_maxvio(counts, S, K, maxvio, max_count=None, stream=None):

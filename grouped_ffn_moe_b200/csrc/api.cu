@@ -357,6 +357,21 @@ moe_status moe_permute_backward(const void* grad_x_perm, const int32_t* row_id_m
                              static_cast<cudaStream_t>(cuda_stream));
 }
 
+moe_status moe_append_shared(const int32_t* topk_ids, const float* route_w, int64_t S, int32_t K,
+                             int32_t E, int32_t n_shared, int32_t* ids_out, float* w_out,
+                             void* cuda_stream) {
+  if (S < 0 || K < 1 || E < 1 || n_shared < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (static_cast<int64_t>(E) + n_shared > MOE_MAX_EXPERTS ||
+      S * (static_cast<int64_t>(K) + n_shared) > moe::kMaxRows)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (S == 0) return MOE_OK;
+  if (!topk_ids || !route_w || !ids_out || !w_out || !aligned(topk_ids, 4) ||
+      !aligned(route_w, 4) || !aligned(ids_out, 4) || !aligned(w_out, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  return moe::launch_append_shared(topk_ids, route_w, S, K, E, n_shared, ids_out, w_out,
+                                   static_cast<cudaStream_t>(cuda_stream));
+}
+
 moe_status moe_maxvio(const int32_t* counts, int32_t E, int64_t S, int32_t K, double* maxvio,
                       int32_t* max_count, void* cuda_stream) {
   if (E < 1 || S < 1 || K < 1) return MOE_ERR_INVALID_ARGUMENT;

@@ -56,6 +56,12 @@ moe_status launch_permute(const void* x, const int32_t* topk_ids, int64_t S, int
 moe_status launch_maxvio(const int32_t* counts, int32_t E, int64_t S, int32_t K, double* maxvio,
                          int32_t* max_count, cudaStream_t stream);
 
+// Routing [S, K+n_shared]: the token's K routed slots, then experts E .. E+n_shared-1 with
+// weight 1 (shared experts).
+moe_status launch_append_shared(const int32_t* ids, const float* w, int64_t S, int32_t K,
+                                int32_t E, int32_t n_shared, int32_t* ids_out, float* w_out,
+                                cudaStream_t stream);
+
 // route_w == nullptr: unit weights (the permutation's backward).
 moe_status launch_combine(const void* y, const int32_t* row_id_map, const float* route_w,
                           int64_t S, int64_t H, int32_t K, void* out, cudaStream_t stream);

@@ -479,6 +479,43 @@ moe_status launch_maxvio(const int32_t* counts, int32_t E, int64_t S, int32_t K,
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// ----------------------------------------------------------------------------- shared experts
+
+namespace {
+
+// Routing with n_shared always-on experts appended: slot K + j of every token is expert
+// E + j with weight 1 (MoE(x) = SharedExpert(x) + sum_k w_k RoutedExpert_k(x), "Mixture of
+// Kittens" digest, Step 1), so the shared expert's rows join the same grouped launches.
+// One thread per output slot.
+__global__ void append_shared_kernel(const int32_t* __restrict__ ids, const float* __restrict__ w,
+                                     int64_t S, int32_t K, int32_t E, int32_t n_shared,
+                                     int32_t* __restrict__ ids_out, float* __restrict__ w_out) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int32_t K2 = K + n_shared;
+  const int64_t total = S * K2;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / K2;
+    const int32_t k = static_cast<int32_t>(i - t * K2);
+    ids_out[i] = k < K ? ids[t * K + k] : E + (k - K);
+    w_out[i] = k < K ? w[t * K + k] : 1.0f;
+  }
+}
+
+}  // namespace
+
+moe_status launch_append_shared(const int32_t* ids, const float* w, int64_t S, int32_t K,
+                                int32_t E, int32_t n_shared, int32_t* ids_out, float* w_out,
+                                cudaStream_t stream) {
+  const int64_t total = S * (K + n_shared);
+  const int64_t blocks = std::min<int64_t>(ceil_div(total, 256), static_cast<int64_t>(num_sms()) * 8);
+  const cudaError_t err =
+      launch_dependent(append_shared_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                       stream, ids, w, S, K, E, n_shared, ids_out, w_out);
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 // ----------------------------------------------------------------------------- no-alloc entry
 
 // Scratch of moe_permute_no_alloc, in the library's own device memory: every GPU that loads

@@ -173,6 +173,26 @@ moe_status moe_grouped_ffn_down(const void* h_scratch, const void* w_down,
                                 int32_t E, void* y, int32_t* d_status, void* cuda_stream);
 
 /*
+ * moe_append_shared - routing for a layer with shared experts ("Mixture of Kittens" digest,
+ * Step 1: MoE(x) = SharedExpert(x) + sum_k w_k RoutedExpert_k(x)). A shared expert is an
+ * expert every token visits with weight 1; appended to the routing it runs in the same
+ * moe_permute / moe_grouped_ffn / moe_unpermute_combine launches as the routed experts.
+ *   ids_out[t, k] = topk_ids[t, k], w_out[t, k] = route_w[t, k]          for k < K
+ *   ids_out[t, K+j] = E + j,        w_out[t, K+j] = 1.0f                 for j < n_shared
+ *   topk_ids [S, K] int32, route_w [S, K] fp32 in; ids_out [S, K+n_shared] int32,
+ *   w_out [S, K+n_shared] fp32 out (caller-owned, device). The layer then runs with
+ *   E + n_shared experts (weights [E+n_shared, ...], the shared ones last) and
+ *   K + n_shared slots. A shared expert n times as wide as a routed one is n such experts
+ *   holding its column slices (SwiGLU is element-wise over H', so the slices' down
+ *   projections add up to the full one). The routed imbalance is moe_maxvio on the first E
+ *   counts with the routed K; moe_permute's own maxvio covers all E + n_shared experts.
+ * Requires E + n_shared <= MOE_MAX_EXPERTS, S*(K+n_shared) < 2^31.
+ */
+moe_status moe_append_shared(const int32_t* topk_ids, const float* route_w, int64_t S, int32_t K,
+                             int32_t E, int32_t n_shared, int32_t* ids_out, float* w_out,
+                             void* cuda_stream);
+
+/*
  * moe_grouped_ffn_gather - moe_grouped_ffn without the permuted copy x_perm: the SwiGLU pass
  * reads each row's token straight from the token-major x (the zero-copy fusion of the MoonEP
  * README, "Zero-copy": experts read the dispatched rows in place). Row r of the

@@ -277,11 +277,13 @@ def weight_scale(w: Workload, which: str) -> float:
     return 1.0 / math.sqrt(w.H if which in ("gate", "up") else w.Hp)
 
 
-def make_layer_inputs(w: Workload, device: str = "cpu"):
+def make_layer_inputs(w: Workload, device: str = "cpu", n_shared: int = 0):
     """All inputs of one layer call as torch tensors on `device`.
 
     Returns dict with x [S,H] bf16, topk_ids [S,K] int32, route_w [S,K] fp32 and, unless
-    the workload uses identity experts, w_gate/w_up [E,H,H'] and w_down [E,H',H] bf16.
+    the workload uses identity experts, w_gate/w_up [E',H,H'] and w_down [E',H',H] bf16 with
+    E' = E + n_shared: the shared experts' weights follow the routed ones in the same
+    tensors (draws are counter-based, so the routed experts' weights do not change).
     """
     import torch
 
@@ -293,9 +295,10 @@ def make_layer_inputs(w: Workload, device: str = "cpu"):
                               w.seed, TAG_X),
     }
     if not w.identity_ffn:
-        for name, tag, shape in (("w_gate", TAG_W_GATE, (w.E, w.H, w.Hp)),
-                                 ("w_up", TAG_W_UP, (w.E, w.H, w.Hp)),
-                                 ("w_down", TAG_W_DOWN, (w.E, w.Hp, w.H))):
+        E2 = w.E + n_shared
+        for name, tag, shape in (("w_gate", TAG_W_GATE, (E2, w.H, w.Hp)),
+                                 ("w_up", TAG_W_UP, (E2, w.H, w.Hp)),
+                                 ("w_down", TAG_W_DOWN, (E2, w.Hp, w.H))):
             t = torch.empty(*shape, dtype=torch.bfloat16, device=device)
             out[name] = normal_bf16_into(t, w.seed, tag, weight_scale(w, name[2:]))
     return out

@@ -628,3 +628,53 @@ def test_zero_copy_gather_training_preactivations(cuda_device):
     torch.cuda.synchronize()
     assert int(buf.d_status.item()) == 0
     assert torch.equal(h2, buf.h) and torch.equal(g2, buf.gate_pre) and torch.equal(u2, buf.up_pre)
+
+
+# ----------------------------------------------------------------------------- shared experts
+
+@pytest.mark.parametrize("wname,n_shared", [("tiny", 1), ("tiny", 2), ("medium", 1), ("medium", 2)])
+def test_shared_expert_layer(cuda_device, wname, n_shared):
+    """MoE(x) = SharedExpert(x) + sum_k w_k RoutedExpert_k(x) with the shared expert appended
+    to the routing (moe_append_shared) and run in the same launches; a shared expert of width
+    n_shared * H' is n_shared column slices. Routing table exact; routed rows stage-wise
+    within the bar; out end to end against the oracle's single shared FFN, allowing the
+    slices' own roundings; the routed maxvio from moe_maxvio on the routed counts."""
+    w = synth.WORKLOADS[wname]
+    dev = cuda_device
+    inp = synth.make_layer_inputs(w, device=str(dev), n_shared=n_shared)
+    S, K, E = w.S, w.K, w.E
+    K2, E2 = K + n_shared, E + n_shared
+    ids2 = torch.empty(S, K2, dtype=torch.int32, device=dev)
+    w2 = torch.empty(S, K2, dtype=torch.float32, device=dev)
+    moe.moe_append_shared(inp["topk_ids"], inp["route_w"], E, n_shared, ids2, w2)
+    buf = moe.LayerBuffers.allocate(S, w.H, w.Hp, E2, K2, dev)
+    moe.moe_layer_forward(inp["x"], ids2, w2, inp["w_gate"], inp["w_up"], inp["w_down"], buf)
+    mv = torch.empty(1, dtype=torch.float64, device=dev)
+    mc = torch.empty(1, dtype=torch.int32, device=dev)
+    moe.moe_maxvio(buf.counts[:E], S, K, mv, mc)
+    torch.cuda.synchronize()
+    assert int(buf.d_status.item()) == 0
+    ids_np, rw = inp["topk_ids"].cpu().numpy(), inp["route_w"].cpu().numpy()
+    assert np.array_equal(ids2[:, :K].cpu().numpy(), ids_np)
+    assert np.array_equal(ids2[:, K:].cpu().numpy(), np.tile(np.arange(E, E2), (S, 1)))
+    assert np.array_equal(w2[:, :K].cpu().numpy(), rw) and bool((w2[:, K:] == 1).all())
+    counts, _, _, _ = O.permute_metadata(ids_np, E)
+    assert (mv.item(), int(mc.item())) == O.maxvio(counts, S, K)
+    # oracle: routed experts as usual, the shared expert as one FFN over the concatenated
+    # slices
+    wg_b, wu_b, wd_b = bits(inp["w_gate"]), bits(inp["w_up"]), bits(inp["w_down"])
+    get = lambda e: (wg_b[e], wu_b[e], wd_b[e])
+    shared = (np.concatenate([wg_b[E + j] for j in range(n_shared)], axis=1),
+              np.concatenate([wu_b[E + j] for j in range(n_shared)], axis=1),
+              np.concatenate([wd_b[E + j] for j in range(n_shared)], axis=0))
+    ref = O.moe_layer_with_shared(bits(inp["x"]), ids_np, rw, E, get, w.Hp, shared)
+    y = bits(buf.y)
+    M = S * K
+    stats = assert_close_bf16(y[:M], ref["y"], "routed y")
+    print(f"[{wname}+{n_shared}] routed y: {stats}")
+    rmap = ref["row_id_map"].reshape(S, K)
+    slices = [y[M + j * S: M + (j + 1) * S] for j in range(n_shared)]  # shared rows in token order
+    inherited = sum(np.abs(rw[:, k:k + 1]) * bf16_ulp(ref["y"][rmap[:, k]]) for k in range(K))
+    inherited = inherited + sum(bf16_ulp(sl) for sl in slices) + bf16_ulp(ref["y_shared"])
+    stats = assert_close_bf16(bits(buf.out), ref["out"], "out", inherited=inherited)
+    print(f"[{wname}+{n_shared}] out (end to end): {stats}")
