@@ -7,9 +7,10 @@
 //
 //   out[t] = bf16( sum_{k ascending} w[t,k] * float(y[row_id_map[t*K+k]]) )
 //
-// One warp per token. Each lane owns U = 4 16-byte vectors (8 bf16 each) per pass and keeps
-// their fp32 sums in registers; the K source rows of a pass are loaded four slots at a time
-// (16 loads in flight per lane) before the fixed-order FMAs consume them.
+// One warp per (token, row slice of 32*U 16-byte vectors): each lane owns U = 4 vectors (8
+// bf16 each) and keeps their fp32 sums in registers; the K source rows are loaded four slots
+// at a time (16 loads in flight per lane) before the fixed-order FMAs consume them. Slicing
+// the rows keeps every SM busy when there are few tokens.
 #include <algorithm>
 #include <cuda_bf16.h>
 
@@ -58,11 +59,15 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
   griddep_wait();  // y and row_id_map come from earlier kernels in the stream
   griddep_launch_dependents();
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       t < S; t += nwarps) {
+  const int64_t npass = (nvec + 32 * U - 1) / (32 * U);
+  const int64_t items = S * npass;
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       it < items; it += nwarps) {
+    const int64_t t = it / npass;
+    const int64_t v0 = (it - t * npass) * (32 * U);
     const int32_t my_row = (lane < K) ? row_id_map[t * K + lane] : -1;
     const float my_w = (lane < K) ? (route_w != nullptr ? route_w[t * K + lane] : 1.0f) : 0.0f;
-    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
+    {
       float acc[U][8];
 #pragma unroll
       for (int j = 0; j < U; ++j)
@@ -193,7 +198,8 @@ moe_status launch_combine_backward(const void* grad_out, const void* y, const in
 moe_status launch_combine(const void* y, const int32_t* row_id_map, const float* route_w,
                           int64_t S, int64_t H, int32_t K, void* out, cudaStream_t stream) {
   const int64_t nvec = H / 8;
-  const int64_t blocks = std::min<int64_t>(ceil_div(S, 8), static_cast<int64_t>(num_sms()) * 8);
+  const int64_t items = S * ceil_div(nvec, 32 * MOE_COMBINE_U);
+  const int64_t blocks = std::min<int64_t>(ceil_div(items, 8), static_cast<int64_t>(num_sms()) * 8);
   const cudaError_t err = launch_dependent(
       combine_kernel<MOE_COMBINE_U, MOE_COMBINE_SLOTS>, dim3(static_cast<unsigned>(blocks)),
       dim3(256), 0, stream, static_cast<const uint4*>(y), row_id_map, route_w, S, nvec, K,

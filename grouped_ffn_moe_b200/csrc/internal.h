@@ -10,14 +10,21 @@
 
 namespace moe {
 
-// Flat routing slots handled by one warp in the permutation kernels.
-constexpr int kChunk = 512;
+// Flat routing slots handled by one warp in the permutation kernels: 512 for large tables,
+// 64 up to 65536 slots, where 512-slot chunks would leave all but a few SMs idle (a chunk
+// is walked 32 slots at a time by one warp).
+constexpr int kChunkMax = 512;
+constexpr int kChunkSmall = 64;
+constexpr int64_t kSmallTableSlots = 65536;
 constexpr int kWarpsPerTile = 8;
-constexpr int kTile = kChunk * kWarpsPerTile;
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-inline int64_t permute_num_chunks(int64_t F) { return ceil_div(F, kChunk); }
+inline int32_t permute_chunk_slots(int64_t F) {
+  return F <= kSmallTableSlots ? kChunkSmall : kChunkMax;
+}
+
+inline int64_t permute_num_chunks(int64_t F) { return ceil_div(F, permute_chunk_slots(F)); }
 
 // Number of SMs of the current device (cached per device).
 int num_sms();

@@ -8,13 +8,13 @@
 //
 // Two launches, no host synchronisation, no atomics on data. The metadata kernel is one
 // cooperative launch (all CTAs co-resident, grid-wide syncs between its phases):
-//   A  per 512-slot chunk (one warp; the chunk's ids prefetched into registers): per-expert
-//      counts with __match_any_sync
+//   A  per chunk of 512 slots (64 up to 65536 slots; one warp, the chunk's ids prefetched
+//      into registers): per-expert counts with __match_any_sync
 //   B  per expert (one warp): exclusive scan over chunks -> chunk bases, counts
 //   C  exclusive scan of counts -> cu_seqlens (+ max count, maxvio); every warp replays its
 //      chunk with per-expert cursors -> row_id_map, perm_src
-// then permute_rows (one warp per token: the row is read once in 16-byte vectors and written
-// to its K rows) runs as a programmatic dependent launch. The metadata phases also exist as
+// then permute_rows (one warp per token and 1024-element row slice: read once in 16-byte
+// vectors, written to the token's K rows) runs as a programmatic dependent launch. The metadata phases also exist as
 // three ordinary launches ("staged", MOE_PERMUTE_KERNEL=staged); both give identical results.
 #include <cooperative_groups.h>
 
@@ -39,6 +39,7 @@ __device__ __forceinline__ void flag_status(int32_t* d_status, int32_t bit) {
 // chunk b*8 + w. Ids outside [0, E) are not counted and set MOE_ERR_BAD_ROUTING.
 __global__ void __launch_bounds__(256) route_hist_kernel(const int32_t* __restrict__ ids,
                                                          int64_t F, int32_t E, int64_t nchunk,
+                                                         int32_t chunk,
                                                          int32_t* __restrict__ chunk_counts,
                                                          int32_t* d_status) {
   extern __shared__ int32_t s_hist[];  // [8][E]
@@ -49,8 +50,8 @@ __global__ void __launch_bounds__(256) route_hist_kernel(const int32_t* __restri
   int32_t* hist = s_hist + warp * E;
   if (c < nchunk) {
     bool bad = false;
-    for (int step = 0; step < kChunk / 32; ++step) {
-      const int64_t f0 = c * kChunk + step * 32;
+    for (int step = 0; step < chunk / 32; ++step) {
+      const int64_t f0 = c * chunk + step * 32;
       if (f0 >= F) break;  // warp-uniform
       const int64_t f = f0 + lane;
       const int32_t e = (f < F) ? ids[f] : -1;
@@ -70,6 +71,35 @@ __global__ void __launch_bounds__(256) route_hist_kernel(const int32_t* __restri
   }
 }
 
+// In place exclusive scan of one expert's chunk counts by one warp; returns the total. The
+// values of eight 32-chunk steps are loaded before they are scanned (loads in flight).
+__device__ __forceinline__ int32_t scan_chunk_row(int32_t* row, int64_t nchunk, int lane) {
+  constexpr int kB = 8;
+  int32_t carry = 0;
+  for (int64_t base = 0; base < nchunk; base += 32 * kB) {
+    int32_t v[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int64_t i = base + u * 32 + lane;
+      v[u] = (i < nchunk) ? row[i] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      if (base + u * 32 >= nchunk) break;  // warp-uniform
+      const int64_t i = base + u * 32 + lane;
+      int32_t incl = v[u];
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int32_t n = __shfl_up_sync(kFull, incl, d);
+        if (lane >= d) incl += n;
+      }
+      if (i < nchunk) row[i] = carry + incl - v[u];
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+  }
+  return carry;
+}
+
 // In place: chunk_counts[e][c] -> sum_{c' < c} chunk_counts[e][c']; counts[e] = total.
 __global__ void __launch_bounds__(256) route_scan_kernel(int32_t* __restrict__ chunk_counts,
                                                          int64_t nchunk, int32_t E,
@@ -78,19 +108,7 @@ __global__ void __launch_bounds__(256) route_scan_kernel(int32_t* __restrict__ c
   const int e = blockIdx.x * 8 + warp;
   if (e >= E) return;
   int32_t* row = chunk_counts + static_cast<int64_t>(e) * nchunk;
-  int32_t carry = 0;
-  for (int64_t base = 0; base < nchunk; base += 32) {
-    const int64_t i = base + lane;
-    const int32_t v = (i < nchunk) ? row[i] : 0;
-    int32_t incl = v;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int32_t n = __shfl_up_sync(kFull, incl, d);
-      if (lane >= d) incl += n;
-    }
-    if (i < nchunk) row[i] = carry + incl - v;
-    carry += __shfl_sync(kFull, incl, 31);
-  }
+  const int32_t carry = scan_chunk_row(row, nchunk, lane);
   if (lane == 0) counts[e] = carry;
 }
 
@@ -146,7 +164,7 @@ __device__ void block_scan_counts(const int32_t* __restrict__ counts, int32_t E,
 
 __global__ void __launch_bounds__(256) route_rank_kernel(
     const int32_t* __restrict__ ids, int64_t F, int64_t S, int32_t K, int32_t E, int64_t nchunk,
-    const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ counts,
+    int32_t chunk, const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ counts,
     int32_t* __restrict__ cu_seqlens, int32_t* __restrict__ row_id_map,
     int32_t* __restrict__ perm_src, double* maxvio, int32_t* max_count) {
   extern __shared__ int32_t smem[];
@@ -175,8 +193,8 @@ __global__ void __launch_bounds__(256) route_rank_kernel(
   const int64_t c = c0 + warp;
   if (c >= nchunk) return;
   int32_t* cur = s_cursor + warp * E;
-  for (int step = 0; step < kChunk / 32; ++step) {
-    const int64_t f0 = c * kChunk + step * 32;
+  for (int step = 0; step < chunk / 32; ++step) {
+    const int64_t f0 = c * chunk + step * 32;
     if (f0 >= F) break;  // warp-uniform
     const int64_t f = f0 + lane;
     const int32_t e = (f < F) ? ids[f] : -1;
@@ -194,8 +212,9 @@ __global__ void __launch_bounds__(256) route_rank_kernel(
   }
 }
 
-// One warp per token: the token's row is read once (U 16-byte vectors per lane per pass)
-// and written to its K destination rows.
+// One warp per (token, row slice of 32*U 16-byte vectors): the slice is read once and written
+// to the token's K destination rows. Slicing the rows keeps every SM busy when there are few
+// tokens (S = 1024 tokens of 7168 features are 7168 work items, not 1024).
 template <int U>
 __global__ void __launch_bounds__(256) permute_rows_kernel(const uint4* __restrict__ x, int64_t S,
                                                            int64_t nvec, int32_t K,
@@ -205,26 +224,28 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint4* __restri
   griddep_wait();  // row_id_map comes from the metadata kernel
   griddep_launch_dependents();
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       t < S; t += nwarps) {
+  const int64_t npass = (nvec + 32 * U - 1) / (32 * U);
+  const int64_t items = S * npass;
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       it < items; it += nwarps) {
+    const int64_t t = it / npass;
+    const int64_t v0 = (it - t * npass) * (32 * U);
     const int32_t my_row = (lane < K) ? row_id_map[t * K + lane] : -1;
     const uint4* src = x + t * nvec;
-    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
-      uint4 r[U];
+    uint4 r[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int64_t v = v0 + j * 32 + lane;
+      if (v < nvec) r[j] = __ldg(src + v);
+    }
+    for (int k = 0; k < K; ++k) {
+      const int32_t row = (K <= 32) ? __shfl_sync(kFull, my_row, k) : row_id_map[t * K + k];
+      if (row < 0) continue;
+      uint4* dst = x_perm + static_cast<int64_t>(row) * nvec;
 #pragma unroll
       for (int j = 0; j < U; ++j) {
         const int64_t v = v0 + j * 32 + lane;
-        if (v < nvec) r[j] = __ldg(src + v);
-      }
-      for (int k = 0; k < K; ++k) {
-        const int32_t row = (K <= 32) ? __shfl_sync(kFull, my_row, k) : row_id_map[t * K + k];
-        if (row < 0) continue;
-        uint4* dst = x_perm + static_cast<int64_t>(row) * nvec;
-#pragma unroll
-        for (int j = 0; j < U; ++j) {
-          const int64_t v = v0 + j * 32 + lane;
-          if (v < nvec) dst[v] = r[j];
-        }
+        if (v < nvec) dst[v] = r[j];
       }
     }
   }
@@ -253,6 +274,7 @@ struct PermuteArgs {
   const int32_t* ids;
   int64_t S, F, nchunk;
   int32_t K, E;
+  int32_t chunk;  // slots per chunk (permute_chunk_slots)
   int32_t* chunk_counts;
   int32_t* counts;
   int32_t* cu_seqlens;
@@ -264,11 +286,11 @@ struct PermuteArgs {
 };
 
 __device__ __forceinline__ void load_chunk_ids(const PermuteArgs& a, int64_t c, int lane,
-                                               int32_t (&idr)[kChunk / 32]) {
+                                               int32_t (&idr)[kChunkMax / 32]) {
 #pragma unroll
-  for (int j = 0; j < kChunk / 32; ++j) {
-    const int64_t f = c * kChunk + j * 32 + lane;
-    idr[j] = f < a.F ? __ldg(a.ids + f) : -1;
+  for (int j = 0; j < kChunkMax / 32; ++j) {
+    const int64_t f = c * a.chunk + j * 32 + lane;
+    idr[j] = (j < a.chunk / 32 && f < a.F) ? __ldg(a.ids + f) : -1;
   }
 }
 
@@ -293,12 +315,13 @@ __global__ void __launch_bounds__(256) permute_fused_kernel(const PermuteArgs a)
     __syncwarp();
     const int64_t c = cb + warp;
     if (c < a.nchunk) {
-      int32_t idr[kChunk / 32];
+      int32_t idr[kChunkMax / 32];
       load_chunk_ids(a, c, lane, idr);
       bool bad = false;
 #pragma unroll
-      for (int j = 0; j < kChunk / 32; ++j) {
-        const int64_t f = c * kChunk + j * 32 + lane;
+      for (int j = 0; j < kChunkMax / 32; ++j) {
+        if (j >= a.chunk / 32) break;  // uniform
+        const int64_t f = c * a.chunk + j * 32 + lane;
         const int32_t e = idr[j];
         const bool ok = f < a.F && e >= 0 && e < E;
         bad |= (f < a.F) && !ok;
@@ -320,20 +343,7 @@ __global__ void __launch_bounds__(256) permute_fused_kernel(const PermuteArgs a)
 
   // B: per-expert exclusive scan over chunks
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * kWarpsPerTile + warp; e < E; e += wstride) {
-    int32_t* row = a.chunk_counts + e * a.nchunk;
-    int32_t carry = 0;
-    for (int64_t base = 0; base < a.nchunk; base += 32) {
-      const int64_t i = base + lane;
-      const int32_t v = (i < a.nchunk) ? row[i] : 0;
-      int32_t incl = v;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int32_t n = __shfl_up_sync(kFull, incl, d);
-        if (lane >= d) incl += n;
-      }
-      if (i < a.nchunk) row[i] = carry + incl - v;
-      carry += __shfl_sync(kFull, incl, 31);
-    }
+    const int32_t carry = scan_chunk_row(a.chunk_counts + e * a.nchunk, a.nchunk, lane);
     if (lane == 0) a.counts[e] = carry;
   }
   grid.sync();
@@ -357,11 +367,12 @@ __global__ void __launch_bounds__(256) permute_fused_kernel(const PermuteArgs a)
     const int64_t c = cb + warp;
     if (c < a.nchunk) {
       int32_t* cur = s_tab + warp * E;
-      int32_t idr[kChunk / 32];
+      int32_t idr[kChunkMax / 32];
       load_chunk_ids(a, c, lane, idr);
 #pragma unroll
-      for (int j = 0; j < kChunk / 32; ++j) {
-        const int64_t f = c * kChunk + j * 32 + lane;
+      for (int j = 0; j < kChunkMax / 32; ++j) {
+        if (j >= a.chunk / 32) break;  // uniform
+        const int64_t f = c * a.chunk + j * 32 + lane;
         const int32_t e = idr[j];
         const bool ok = f < a.F && e >= 0 && e < E;
         const unsigned peers = __match_any_sync(kFull, ok ? e : -1);
@@ -415,7 +426,8 @@ bool use_staged_permute() {
 cudaError_t launch_rows(const void* x, int64_t S, int64_t H, int32_t K, const int32_t* row_id_map,
                         void* x_perm, cudaStream_t stream) {
   const int64_t nvec = H / 8;
-  const int64_t blocks = std::min<int64_t>(ceil_div(S, 8), static_cast<int64_t>(num_sms()) * 8);
+  const int64_t items = S * ceil_div(nvec, 32 * 4);
+  const int64_t blocks = std::min<int64_t>(ceil_div(items, 8), static_cast<int64_t>(num_sms()) * 8);
   return launch_dependent(permute_rows_kernel<4>, dim3(static_cast<unsigned>(blocks)), dim3(256),
                           0, stream, static_cast<const uint4*>(x), S, nvec, K, row_id_map,
                           static_cast<uint4*>(x_perm));
@@ -430,13 +442,14 @@ moe_status launch_permute(const void* x, const int32_t* topk_ids, int64_t S, int
                           cudaStream_t stream) {
   const int64_t F = S * K;
   const int64_t nchunk = permute_num_chunks(F);
+  const int32_t chunk = permute_chunk_slots(F);
   const int64_t tiles = ceil_div(nchunk, kWarpsPerTile);
   const int per_sm = use_staged_permute() ? 0 : fused_blocks_per_sm();
   if (per_sm > 0) {
     const int64_t want = std::max<int64_t>({tiles, ceil_div(E, kWarpsPerTile), 1});
     const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(per_sm) * num_sms()));
-    PermuteArgs pa{topk_ids, S, F, nchunk, K, E, chunk_counts, counts, cu_seqlens, row_id_map,
-                   perm_src, maxvio, max_count, d_status};
+    PermuteArgs pa{topk_ids, S, F, nchunk, K, E, chunk, chunk_counts, counts, cu_seqlens,
+                   row_id_map, perm_src, maxvio, max_count, d_status};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(256);
@@ -462,11 +475,11 @@ moe_status launch_permute(const void* x, const int32_t* topk_ids, int64_t S, int
   const size_t hist_smem = sizeof(int32_t) * kWarpsPerTile * E;
   const size_t rank_smem = sizeof(int32_t) * (E + 1 + kWarpsPerTile * E);
   route_hist_kernel<<<static_cast<unsigned>(tiles), 256, hist_smem, stream>>>(
-      topk_ids, F, E, nchunk, chunk_counts, d_status);
+      topk_ids, F, E, nchunk, chunk, chunk_counts, d_status);
   route_scan_kernel<<<static_cast<unsigned>(ceil_div(E, 8)), 256, 0, stream>>>(chunk_counts,
                                                                              nchunk, E, counts);
   route_rank_kernel<<<static_cast<unsigned>(tiles), 256, rank_smem, stream>>>(
-      topk_ids, F, S, K, E, nchunk, chunk_counts, counts, cu_seqlens, row_id_map, perm_src,
+      topk_ids, F, S, K, E, nchunk, chunk, chunk_counts, counts, cu_seqlens, row_id_map, perm_src,
       maxvio, max_count);
   if (x_perm != nullptr && launch_rows(x, S, H, K, row_id_map, x_perm, stream) != cudaSuccess)
     return MOE_ERR_CUDA;

@@ -387,15 +387,17 @@ def test_down_kernel_variants_agree(cuda_device, tmp_path):
     assert torch.equal(outs["pair"], outs["single"])
 
 
-def test_permute_variants_agree(cuda_device, tmp_path):
-    """The fused cooperative permutation (default) and the four-launch staged one
+@pytest.mark.parametrize("wname", ["permute_combine_S4096_mv20", "permute_combine_S16384_mv1",
+                                   "medium"])
+def test_permute_variants_agree(cuda_device, tmp_path, wname):
+    """The fused cooperative permutation (default) and the three-launch staged one
     (MOE_PERMUTE_KERNEL=staged) give bit-identical metadata and rows."""
     import subprocess
     import sys
 
     script = (
         "import sys, torch, synth, grouped_ffn_moe_b200 as moe\n"
-        "w = synth.WORKLOADS['permute_combine_S4096_mv20']\n"
+        f"w = synth.WORKLOADS['{wname}']\n"
         "inp = synth.make_layer_inputs(w, device='cuda:0')\n"
         "buf = moe.LayerBuffers.allocate(w.S, w.H, 0, w.E, w.K, torch.device('cuda:0'),"
         " with_ffn=False)\n"
