@@ -133,7 +133,7 @@ def test_permute_edge_cases(cuda_device, name):
     check_permute_exact(r, ids_np, E, xb)
 
 
-@pytest.mark.parametrize("wname", ["tiny", "medium", "large", "skew20",
+@pytest.mark.parametrize("wname", ["tiny", "medium", "large", "skew20", "skew20_last",
                                    "permute_combine_S65536_mv20"])
 def test_permute_workloads(cuda_device, wname):
     w = synth.WORKLOADS[wname]
@@ -297,8 +297,10 @@ def _sampled_rows(cu, hot, rng, per=6):
     return np.array(rows, dtype=np.int64)
 
 
-@pytest.mark.parametrize("wname", ["large", "skew20"])
+@pytest.mark.parametrize("wname", ["large", "skew20", "skew20_last"])
 def test_layer_full_size_sampled(cuda_device, wname):
+    """Full-size layers on sampled rows; skew20_last puts the hot expert (maxvio 20) last, so
+    its units come at the end of the persistent schedule."""
     w = synth.WORKLOADS[wname]
     inp = layer_inputs(w, cuda_device)
     buf = run_layer(inp, w, cuda_device)
