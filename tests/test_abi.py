@@ -88,3 +88,47 @@ def test_host_validation_rejects_without_launch():
     assert L.moe_unpermute_combine(a, a, a, 0, 16, 2, a, null) == 0  # S = 0: no-op
     # maxvio: S*K must be positive
     assert L.moe_maxvio(a, 8, 0, 2, a, null, null) == 1
+
+
+def test_host_validation_of_backward_gather_and_shared_calls():
+    """The entry points of the backward, the zero-copy forward and the shared experts reject
+    bad arguments on the host, before any launch (no GPU needed)."""
+    L = moe.lib()
+    a = fake(0x10000)
+    mis = fake(0x10008)  # 8-byte aligned only
+    null = P(0)
+    # combine / permutation backward: H % 8, grad_w without y, S = 0 no-op
+    assert L.moe_combine_backward(a, a, a, a, 4, 12, 2, a, null, null) == 2
+    assert L.moe_combine_backward(a, null, a, a, 4, 16, 2, a, a, null) == 1
+    assert L.moe_combine_backward(a, a, a, a, 0, 16, 2, a, a, null) == 0
+    assert L.moe_permute_backward(a, a, 4, 16, 0, a, null) == 1
+    assert L.moe_permute_backward(mis, a, 4, 16, 2, a, null) == 1
+    # training forward: both pre-activation outputs required, 16-byte aligned
+    assert L.moe_grouped_ffn_up_gate_train(a, a, a, a, 16, 256, 256, 4, a, null, a, null,
+                                           null) == 1
+    assert L.moe_grouped_ffn_up_gate_train(a, a, a, a, 16, 256, 256, 4, a, a, mis, null,
+                                           null) == 1
+    # FFN backward passes: H' % 128, missing d_up, the accumulate flag, misaligned buffers
+    assert L.moe_grouped_ffn_down_backward(a, a, a, a, a, 16, 256, 200, 4, a, a, null, null) == 2
+    assert L.moe_grouped_ffn_down_backward(a, a, a, a, a, 16, 256, 256, 4, a, null, null,
+                                           null) == 1
+    assert L.moe_grouped_ffn_up_gate_backward(a, a, a, null, a, 16, 256, 256, 4, a, null,
+                                              null) == 1
+    assert L.moe_grouped_ffn_weight_grad(a, a, a, a, a, a, 16, 256, 256, 4, a, a, a, 2, null,
+                                         null) == 1
+    assert L.moe_grouped_ffn_weight_grad(a, a, a, a, a, a, 16, 256, 256, 4, a, mis, a, 0, null,
+                                         null) == 1
+    assert L.moe_grouped_ffn_backward(a, a, a, a, a, a, a, a, 16, 256, 256, 4, a, a, a, null,
+                                      a, a, a, 0, null, null) == 1
+    assert L.moe_grouped_ffn_backward(a, a, a, a, a, a, a, a, 16, 256, 256, 4, a, a, a, a,
+                                      a, a, a, 3, null, null) == 1
+    # zero-copy forward: K < 1, misaligned x, one pre-activation output only, S = 0 no-op
+    assert L.moe_grouped_ffn_gather(a, a, 4, 0, a, a, a, a, 256, 256, 4, a, a, null, null) == 1
+    assert L.moe_grouped_ffn_gather(mis, a, 4, 2, a, a, a, a, 256, 256, 4, a, a, null, null) == 1
+    assert L.moe_grouped_ffn_up_gate_gather(a, a, 4, 2, a, a, a, 256, 256, 4, a, a, null, null,
+                                            null) == 1
+    assert L.moe_grouped_ffn_gather(a, a, 0, 2, a, a, a, a, 256, 256, 4, a, a, null, null) == 0
+    # shared experts: E + n beyond the maximum, n < 1, S = 0 no-op
+    assert L.moe_append_shared(a, a, 4, 2, 1024, 1, a, a, null) == 2
+    assert L.moe_append_shared(a, a, 4, 2, 8, 0, a, a, null) == 1
+    assert L.moe_append_shared(a, a, 0, 2, 8, 1, a, a, null) == 0
