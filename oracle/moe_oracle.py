@@ -357,6 +357,81 @@ def grouped_ffn_backward(x_perm_bits, g_bits, u_bits, h_bits, grad_y_bits, cu_se
     return out
 
 
+# ----------------------------------------------------------------------------- MXFP8
+#
+# "Mixture of Kittens" digest, Step 8 (MXFP8 Support): an MXFP8 mode with weights quantised
+# once ahead of time and activation quantisation fused into dispatch, the GEMMs and SwiGLU;
+# the shared expert stays in bf16. The pages do not spell the format out; these functions
+# follow the public OCP Microscaling (MX) v1.0 definition of MXFP8: blocks of 32 consecutive
+# elements along the reduction dimension share one power-of-two scale X = 2^(floor(log2
+# amax) - 8) (8 = exponent of E4M3's largest normal), stored as E8M0 (exponent in
+# [-127, 127]); each element is V / X rounded to nearest-even in FP8 E4M3 (3 mantissa bits,
+# exponent bias 7, subnormal step 2^-9, largest finite 448, no infinities). Reading: values
+# of V / X above 448 (possible since amax / X lies in [256, 512)) saturate to +-448.
+# Products of two MXFP8 values are exact in float64; dot products here accumulate in float64.
+
+MX_BLOCK = 32
+E4M3_MAX = 448.0
+E4M3_EMAX = 8
+
+
+def e4m3_round(v: np.ndarray) -> np.ndarray:
+    """Round float64 values to FP8 E4M3 (nearest, ties to even), saturating at +-448."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)  # below 2^-6 the spacing is the subnormal step 2^-9
+    step = np.ldexp(1.0, (e - 3).astype(np.int64))
+    q = np.minimum(np.rint(a / step) * step, E4M3_MAX)
+    return np.copysign(q, v)
+
+
+def mx_quantize(v: np.ndarray, axis: int = -1):
+    """MXFP8 quantisation in blocks of 32 along `axis` (its length a multiple of 32).
+
+    Returns (elements, scale exponents): elements are the E4M3 values as float64, with the
+    shape of v; scale exponents are int64 with axis length / 32 blocks along `axis`."""
+    v = np.moveaxis(np.asarray(v, dtype=np.float64), axis, -1)
+    n = v.shape[-1]
+    assert n % MX_BLOCK == 0
+    blocks = v.reshape(v.shape[:-1] + (n // MX_BLOCK, MX_BLOCK))
+    amax = np.abs(blocks).max(axis=-1)
+    sexp = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - E4M3_EMAX,
+                    -127.0)
+    sexp = np.clip(sexp, -127, 127).astype(np.int64)
+    q = e4m3_round(blocks / np.ldexp(1.0, sexp)[..., None])
+    return (np.moveaxis(q.reshape(v.shape), -1, axis),
+            np.moveaxis(sexp, -1, axis))
+
+
+def mx_dequantize(q: np.ndarray, sexp: np.ndarray, axis: int = -1) -> np.ndarray:
+    """Elements times their block's scale (float64, exact)."""
+    q = np.moveaxis(np.asarray(q, dtype=np.float64), axis, -1)
+    s = np.moveaxis(np.asarray(sexp), axis, -1)
+    out = q * np.repeat(np.ldexp(1.0, s), MX_BLOCK, axis=-1)
+    return np.moveaxis(out, -1, axis)
+
+
+def mx_weights(w_bits: np.ndarray):
+    """Pre-quantised expert weights [.., k, n] (bf16 bits): blocks of 32 along k, the
+    reduction dimension (axis -2). Returns (elements, scale exponents)."""
+    return mx_quantize(bf16_bits_to_f64(w_bits), axis=-2)
+
+
+def expert_ffn_rows_mxfp8(x_rows_bits, w_gate_q, w_up_q, w_down_q):
+    """One expert in MXFP8: x quantised along H, h = silu(g) * u quantised along H' (fused in
+    the SwiGLU epilogue), weights pre-quantised along their reduction dimension (mx_weights);
+    products exact, sums in float64; y = bf16(deq(h_q) . deq(Wd_q)). Returns
+    (h elements, h scale exponents, y bits)."""
+    xq, xs = mx_quantize(bf16_bits_to_f64(x_rows_bits), axis=-1)
+    x = mx_dequantize(xq, xs, axis=-1)
+    g = x @ mx_dequantize(*w_gate_q, axis=-2)
+    u = x @ mx_dequantize(*w_up_q, axis=-2)
+    hq, hs = mx_quantize(silu(g) * u, axis=-1)
+    y = mx_dequantize(hq, hs, axis=-1) @ mx_dequantize(*w_down_q, axis=-2)
+    return hq, hs, f64_to_bf16_bits(y)
+
+
 # ----------------------------------------------------------------------------- whole layer
 
 
