@@ -36,7 +36,10 @@ LAUNCHES = {"moe_permute": 2, "moe_grouped_ffn": 2, "moe_grouped_ffn_up_gate": 1
             "moe_grouped_ffn_up_gate_train": 1, "moe_grouped_ffn_down_backward": 1,
             "moe_grouped_ffn_up_gate_backward": 1, "moe_grouped_ffn_weight_grad": 1,
             "moe_grouped_ffn_backward": 3, "moe_grouped_ffn_gather": 2,
-            "moe_grouped_ffn_up_gate_gather": 1, "moe_append_shared": 1}
+            "moe_grouped_ffn_up_gate_gather": 1, "moe_append_shared": 1,
+            "moe_mx_quantize_weights": 1, "moe_mx_permute_quantize": 1,
+            "moe_grouped_ffn_mxfp8": 2, "moe_grouped_ffn_up_gate_mxfp8": 1,
+            "moe_grouped_ffn_down_mxfp8": 1}
 
 
 class MoeError(RuntimeError):
@@ -99,6 +102,20 @@ def lib() -> ctypes.CDLL:
         L.moe_grouped_ffn_backward.restype = i32
         L.moe_grouped_ffn_backward.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i32, p, p,
                                                p, p, p, p, p, i32, p, p]
+        L.moe_mx_weight_scale_bytes.restype = sz
+        L.moe_mx_weight_scale_bytes.argtypes = [i32, i64, i64]
+        L.moe_mx_quantize_weights.restype = i32
+        L.moe_mx_quantize_weights.argtypes = [p, i32, i64, i64, p, p, p]
+        L.moe_mx_permute_quantize.restype = i32
+        L.moe_mx_permute_quantize.argtypes = [p, p, i64, i64, i32, p, p, p]
+        L.moe_grouped_ffn_mxfp8.restype = i32
+        L.moe_grouped_ffn_mxfp8.argtypes = [p, p, p, p, p, p, p, p, p, i64, i64, i64, i32, p, p,
+                                            p, p, p]
+        L.moe_grouped_ffn_up_gate_mxfp8.restype = i32
+        L.moe_grouped_ffn_up_gate_mxfp8.argtypes = [p, p, p, p, p, p, p, i64, i64, i64, i32, p, p,
+                                                    p, p]
+        L.moe_grouped_ffn_down_mxfp8.restype = i32
+        L.moe_grouped_ffn_down_mxfp8.argtypes = [p, p, p, p, p, i64, i64, i64, i32, p, p, p]
         _lib = L
     return _lib
 
@@ -631,3 +648,181 @@ def moe_layer_backward(grad_out, route_w, w_gate, w_up, w_down, buf: LayerBuffer
                              grads.grad_w_down, accumulate, buf.d_status, stream)
     moe_permute_backward(grads.grad_x_perm, buf.row_id_map, grads.grad_x, K, stream)
     return grads
+
+
+# ----------------------------------------------------------------------------- MXFP8
+
+
+def moe_mx_weight_scale_bytes(E: int, R: int, C: int) -> int:
+    return int(lib().moe_mx_weight_scale_bytes(E, R, C))
+
+
+def moe_mx_quantize_weights(w, w_q, w_sf, stream=None):
+    """Quantise weights [E,R,C] bf16 (R the reduction dimension) to MXFP8: w_q [E,R,C] uint8
+    (E4M3 codes), w_sf uint8 with moe_mx_weight_scale_bytes(E,R,C) bytes (E8M0 scales in the
+    chunk order of include/moe_b200.h)."""
+    _need(w, "w", torch.bfloat16, None, 3)
+    dev = w.device
+    _need(w_q, "w_q", torch.uint8, dev)
+    _need(w_sf, "w_sf", torch.uint8, dev)
+    E, R, C = w.shape
+    if tuple(w_q.shape) != (E, R, C):
+        raise ValueError(f"w_q: expected {(E, R, C)}, got {tuple(w_q.shape)}")
+    if w_sf.numel() != moe_mx_weight_scale_bytes(E, R, C):
+        raise ValueError("w_sf: expected moe_mx_weight_scale_bytes(E, R, C) bytes")
+    st = lib().moe_mx_quantize_weights(_ptr(w), E, R, C, _ptr(w_q), _ptr(w_sf),
+                                       _stream(stream, dev))
+    _check("moe_mx_quantize_weights", st)
+
+
+def mx_quantize_weights(w, stream=None):
+    """Allocate and fill (w_q, w_sf) for one projection's bf16 weights [E,R,C]."""
+    E, R, C = w.shape
+    w_q = torch.empty(E, R, C, dtype=torch.uint8, device=w.device)
+    w_sf = torch.empty(max(moe_mx_weight_scale_bytes(E, R, C), 1), dtype=torch.uint8,
+                       device=w.device)
+    moe_mx_quantize_weights(w, w_q, w_sf, stream)
+    return w_q, w_sf
+
+
+def moe_mx_permute_quantize(x, row_id_map, K, x_q, x_sf, stream=None):
+    """Quantise the token rows of x [S,H] bf16 to MXFP8 and write them to their expert-grouped
+    rows: x_q [S*K,H] uint8, x_sf [S*K,H/32] uint8."""
+    _need(x, "x", torch.bfloat16, None, 2)
+    dev = x.device
+    S, H = x.shape
+    _need(row_id_map, "row_id_map", torch.int32, dev)
+    _need(x_q, "x_q", torch.uint8, dev, 2)
+    _need(x_sf, "x_sf", torch.uint8, dev, 2)
+    if row_id_map.numel() != S * K or tuple(x_q.shape) != (S * K, H) or \
+            tuple(x_sf.shape) != (S * K, H // 32):
+        raise ValueError("row_id_map [S*K], x_q [S*K,H] and x_sf [S*K,H/32] expected")
+    st = lib().moe_mx_permute_quantize(_ptr(x), _ptr(row_id_map), S, H, K, _ptr(x_q), _ptr(x_sf),
+                                       _stream(stream, dev))
+    _check("moe_mx_permute_quantize", st)
+
+
+@dataclass
+class MxWeights:
+    """One layer's expert weights in MXFP8 (codes and chunked scales per projection)."""
+
+    w_gate_q: torch.Tensor
+    w_gate_sf: torch.Tensor
+    w_up_q: torch.Tensor
+    w_up_sf: torch.Tensor
+    w_down_q: torch.Tensor
+    w_down_sf: torch.Tensor
+
+    @staticmethod
+    def from_bf16(w_gate, w_up, w_down, stream=None):
+        gq, gs = mx_quantize_weights(w_gate, stream)
+        uq, us = mx_quantize_weights(w_up, stream)
+        dq, ds = mx_quantize_weights(w_down, stream)
+        return MxWeights(gq, gs, uq, us, dq, ds)
+
+
+def _mx_check(x_q, x_sf, mw: MxWeights, cu_seqlens, d_status):
+    M, H = x_q.shape
+    E, H2, Hp = mw.w_gate_q.shape
+    dev = x_q.device
+    _need(x_q, "x_q", torch.uint8, dev, 2)
+    _need(x_sf, "x_sf", torch.uint8, dev, 2)
+    for name in ("w_gate_q", "w_gate_sf", "w_up_q", "w_up_sf", "w_down_q", "w_down_sf"):
+        _need(getattr(mw, name), name, torch.uint8, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(d_status, "d_status", torch.int32, dev)
+    if H2 != H or tuple(mw.w_up_q.shape) != (E, H, Hp) or tuple(mw.w_down_q.shape) != (E, Hp, H):
+        raise ValueError("MXFP8 weights must be w_gate/w_up [E,H,H'] and w_down [E,H',H]")
+    if tuple(x_sf.shape) != (M, H // 32) or cu_seqlens.numel() != E + 1:
+        raise ValueError("x_sf must be [M,H/32] and cu_seqlens have E+1 entries")
+    return M, H, Hp, E, dev
+
+
+def moe_grouped_ffn_up_gate_mxfp8(x_q, x_sf, mw: MxWeights, cu_seqlens, h_q, h_sf, d_status=None,
+                                  stream=None):
+    """MXFP8 SwiGLU pass: h = silu(x Wg) * (x Wu) from MXFP8 operands, stored as MXFP8
+    (h_q [M,H'] uint8, h_sf [M,H'/32] uint8)."""
+    M, H, Hp, E, dev = _mx_check(x_q, x_sf, mw, cu_seqlens, d_status)
+    _need(h_q, "h_q", torch.uint8, dev, 2)
+    _need(h_sf, "h_sf", torch.uint8, dev, 2)
+    if tuple(h_q.shape) != (M, Hp) or tuple(h_sf.shape) != (M, Hp // 32):
+        raise ValueError("h_q must be [M,H'] and h_sf [M,H'/32]")
+    st = lib().moe_grouped_ffn_up_gate_mxfp8(_ptr(x_q), _ptr(x_sf), _ptr(mw.w_gate_q),
+                                             _ptr(mw.w_gate_sf), _ptr(mw.w_up_q),
+                                             _ptr(mw.w_up_sf), _ptr(cu_seqlens), M, H, Hp, E,
+                                             _ptr(h_q), _ptr(h_sf), _ptr(d_status),
+                                             _stream(stream, dev))
+    _check("moe_grouped_ffn_up_gate_mxfp8", st)
+
+
+def moe_grouped_ffn_down_mxfp8(h_q, h_sf, mw: MxWeights, cu_seqlens, y, d_status=None,
+                               stream=None):
+    """MXFP8 down pass: y = bf16(h W_down) from MXFP8 h and W_down."""
+    M, Hp = h_q.shape
+    E, _, H = mw.w_down_q.shape
+    dev = h_q.device
+    _need(h_q, "h_q", torch.uint8, dev, 2)
+    _need(h_sf, "h_sf", torch.uint8, dev, 2)
+    _need(mw.w_down_q, "w_down_q", torch.uint8, dev, 3)
+    _need(mw.w_down_sf, "w_down_sf", torch.uint8, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(d_status, "d_status", torch.int32, dev)
+    _need(y, "y", torch.bfloat16, dev, 2)
+    if tuple(h_sf.shape) != (M, Hp // 32) or tuple(y.shape) != (M, H) or \
+            tuple(mw.w_down_q.shape) != (E, Hp, H) or cu_seqlens.numel() != E + 1:
+        raise ValueError("h_sf [M,H'/32], y [M,H], w_down_q [E,H',H], cu_seqlens [E+1] expected")
+    st = lib().moe_grouped_ffn_down_mxfp8(_ptr(h_q), _ptr(h_sf), _ptr(mw.w_down_q),
+                                          _ptr(mw.w_down_sf), _ptr(cu_seqlens), M, H, Hp, E,
+                                          _ptr(y), _ptr(d_status), _stream(stream, dev))
+    _check("moe_grouped_ffn_down_mxfp8", st)
+
+
+def moe_grouped_ffn_mxfp8(x_q, x_sf, mw: MxWeights, cu_seqlens, h_q, h_sf, y, d_status=None,
+                          stream=None):
+    """Both MXFP8 passes (include/moe_b200.h, moe_grouped_ffn_mxfp8)."""
+    M, H, Hp, E, dev = _mx_check(x_q, x_sf, mw, cu_seqlens, d_status)
+    _need(h_q, "h_q", torch.uint8, dev, 2)
+    _need(h_sf, "h_sf", torch.uint8, dev, 2)
+    _need(y, "y", torch.bfloat16, dev, 2)
+    if tuple(h_q.shape) != (M, Hp) or tuple(h_sf.shape) != (M, Hp // 32) or \
+            tuple(y.shape) != (M, H):
+        raise ValueError("h_q [M,H'], h_sf [M,H'/32] and y [M,H] expected")
+    st = lib().moe_grouped_ffn_mxfp8(_ptr(x_q), _ptr(x_sf), _ptr(mw.w_gate_q), _ptr(mw.w_gate_sf),
+                                     _ptr(mw.w_up_q), _ptr(mw.w_up_sf), _ptr(mw.w_down_q),
+                                     _ptr(mw.w_down_sf), _ptr(cu_seqlens), M, H, Hp, E, _ptr(h_q),
+                                     _ptr(h_sf), _ptr(y), _ptr(d_status), _stream(stream, dev))
+    _check("moe_grouped_ffn_mxfp8", st)
+
+
+@dataclass
+class MxBuffers:
+    """The MXFP8 activations of one layer call: x_q/x_sf [M,H], [M,H/32]; h_q/h_sf [M,H'],
+    [M,H'/32] (uint8)."""
+
+    x_q: torch.Tensor
+    x_sf: torch.Tensor
+    h_q: torch.Tensor
+    h_sf: torch.Tensor
+
+    @staticmethod
+    def allocate(S: int, H: int, Hp: int, K: int, device):
+        M = S * K
+        u8 = dict(dtype=torch.uint8, device=device)
+        return MxBuffers(torch.empty(M, H, **u8), torch.empty(M, H // 32, **u8),
+                         torch.empty(M, Hp, **u8), torch.empty(M, Hp // 32, **u8))
+
+
+def moe_layer_forward_mxfp8(x, topk_ids, route_w, mw: MxWeights, buf: LayerBuffers,
+                            mxbuf: MxBuffers, stream=None):
+    """The layer with MXFP8 experts: routing (moe_permute, no bf16 row copy) -> permute fused
+    with the activations' quantisation -> MXFP8 grouped FFN -> weighted combine; returns
+    buf.out (buf.x_perm and buf.h are not used)."""
+    E = buf.counts.numel()
+    K = topk_ids.shape[1]
+    moe_permute(x, topk_ids, E, None, buf.counts, buf.cu_seqlens, buf.row_id_map, buf.perm_src,
+                buf.maxvio, buf.max_count, buf.workspace, buf.d_status, stream)
+    moe_mx_permute_quantize(x, buf.row_id_map, K, mxbuf.x_q, mxbuf.x_sf, stream)
+    moe_grouped_ffn_mxfp8(mxbuf.x_q, mxbuf.x_sf, mw, buf.cu_seqlens, mxbuf.h_q, mxbuf.h_sf, buf.y,
+                          buf.d_status, stream)
+    moe_unpermute_combine(buf.y, buf.row_id_map, route_w, buf.out, stream)
+    return buf.out

@@ -8,7 +8,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmoe_b200.so")
 SOURCES = ["api.cu", "permute.cu", "combine.cu", "tensor_maps.cu", "grouped_ffn.cu",
-           "grouped_ffn_bwd.cu"]
+           "grouped_ffn_bwd.cu", "grouped_ffn_mx.cu"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC", "-lineinfo",
               "-gencode", "arch=compute_100a,code=sm_100a"]
 

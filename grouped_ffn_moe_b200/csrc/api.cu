@@ -51,7 +51,7 @@ const char* moe_status_string(moe_status s) {
   }
 }
 
-int32_t moe_abi_version(void) { return (1 << 16) | 1; }
+int32_t moe_abi_version(void) { return (1 << 16) | 2; }
 
 size_t moe_permute_workspace_bytes(int64_t S, int32_t K, int32_t E) {
   if (S <= 0 || K <= 0 || E <= 0) return 0;
@@ -379,6 +379,86 @@ moe_status moe_maxvio(const int32_t* counts, int32_t E, int64_t S, int32_t K, do
     return MOE_ERR_INVALID_ARGUMENT;
   return moe::launch_maxvio(counts, E, S, K, maxvio, max_count,
                             static_cast<cudaStream_t>(cuda_stream));
+}
+
+
+// ----------------------------------------------------------------------------- MXFP8
+
+size_t moe_mx_weight_scale_bytes(int32_t E, int64_t R, int64_t C) {
+  if (E <= 0 || R <= 0 || C <= 0 || R % 128 != 0 || C % 128 != 0) return 0;
+  return static_cast<size_t>(E) * static_cast<size_t>(R / 32) * static_cast<size_t>(C);
+}
+
+moe_status moe_mx_quantize_weights(const void* w, int32_t E, int64_t R, int64_t C, void* w_q,
+                                   void* w_sf, void* cuda_stream) {
+  if (E < 1 || R <= 0 || C <= 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (R % 128 != 0 || C % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<int64_t>(E) * R > moe::kMaxRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!ok_ptr16(w) || !ok_ptr16(w_q) || !ok_ptr16(w_sf)) return MOE_ERR_INVALID_ARGUMENT;
+  return moe::launch_mx_quantize_weights(w, E, R, C, w_q, w_sf,
+                                         static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_mx_permute_quantize(const void* x, const int32_t* row_id_map, int64_t S, int64_t H,
+                                   int32_t K, void* x_q, void* x_sf, void* cuda_stream) {
+  if (S < 0 || H <= 0 || K < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (H % 128 != 0 || S * K > moe::kMaxRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (S == 0) return MOE_OK;
+  if (!ok_ptr16(x) || !ok_ptr16(x_q) || !ok_ptr16(x_sf) || row_id_map == nullptr ||
+      !aligned(row_id_map, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  return moe::launch_mx_permute_quantize(x, S, H, K, row_id_map, x_q, x_sf,
+                                         static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_grouped_ffn_up_gate_mxfp8(const void* x_q, const void* x_sf, const void* w_gate_q,
+                                         const void* w_gate_sf, const void* w_up_q,
+                                         const void* w_up_sf, const int32_t* cu_seqlens, int64_t M,
+                                         int64_t H, int64_t Hp, int32_t E, void* h_q, void* h_sf,
+                                         int32_t* d_status, void* cuda_stream) {
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  if (!ok_ptr16(x_q) || !ok_ptr16(x_sf) || !ok_ptr16(w_gate_q) || !ok_ptr16(w_gate_sf) ||
+      !ok_ptr16(w_up_q) || !ok_ptr16(w_up_sf) || !ok_ptr16(h_q) || !ok_ptr16(h_sf) ||
+      cu_seqlens == nullptr || !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M == 0) return MOE_OK;
+  return moe::launch_mx_ffn_pass(true, x_q, x_sf, w_gate_q, w_gate_sf, w_up_q, w_up_sf,
+                                 cu_seqlens, M, H, Hp, E, h_q, h_sf, d_status,
+                                 static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_grouped_ffn_down_mxfp8(const void* h_q, const void* h_sf, const void* w_down_q,
+                                      const void* w_down_sf, const int32_t* cu_seqlens, int64_t M,
+                                      int64_t H, int64_t Hp, int32_t E, void* y, int32_t* d_status,
+                                      void* cuda_stream) {
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  if (!ok_ptr16(h_q) || !ok_ptr16(h_sf) || !ok_ptr16(w_down_q) || !ok_ptr16(w_down_sf) ||
+      !ok_ptr16(y) || cu_seqlens == nullptr || !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (M == 0) return MOE_OK;
+  return moe::launch_mx_ffn_pass(false, h_q, h_sf, w_down_q, w_down_sf, nullptr, nullptr,
+                                 cu_seqlens, M, H, Hp, E, y, nullptr, d_status,
+                                 static_cast<cudaStream_t>(cuda_stream));
+}
+
+moe_status moe_grouped_ffn_mxfp8(const void* x_q, const void* x_sf, const void* w_gate_q,
+                                 const void* w_gate_sf, const void* w_up_q, const void* w_up_sf,
+                                 const void* w_down_q, const void* w_down_sf,
+                                 const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp,
+                                 int32_t E, void* h_q, void* h_sf, void* y, int32_t* d_status,
+                                 void* cuda_stream) {
+  const moe_status st = check_ffn_shapes(M, H, Hp, E);
+  if (st != MOE_OK) return st;
+  if (!ok_ptr16(w_down_q) || !ok_ptr16(w_down_sf) || !ok_ptr16(y))
+    return MOE_ERR_INVALID_ARGUMENT;
+  const moe_status s1 = moe_grouped_ffn_up_gate_mxfp8(x_q, x_sf, w_gate_q, w_gate_sf, w_up_q,
+                                                      w_up_sf, cu_seqlens, M, H, Hp, E, h_q, h_sf,
+                                                      d_status, cuda_stream);
+  if (s1 != MOE_OK) return s1;
+  return moe_grouped_ffn_down_mxfp8(h_q, h_sf, w_down_q, w_down_sf, cu_seqlens, M, H, Hp, E, y,
+                                    d_status, cuda_stream);
 }
 
 }  // extern "C"

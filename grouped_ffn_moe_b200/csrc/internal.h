@@ -116,4 +116,23 @@ moe_status launch_ffn_weight_grad(const void* x_perm, const void* h, const void*
                                   float* grad_w_up, float* grad_w_down, bool accumulate,
                                   int32_t* d_status, cudaStream_t stream);
 
+// MXFP8 (E4M3 elements, E8M0 scales per 32 elements along the reduction dimension; layouts in
+// grouped_ffn_mx.cu). Weights [E][R][C] bf16 -> q [E][R][C] and chunked scales
+// [E][C/128][R/128][512]; R and C multiples of 128.
+moe_status launch_mx_quantize_weights(const void* w, int32_t E, int64_t R, int64_t C, void* q,
+                                      void* sf, cudaStream_t stream);
+
+// x [S][H] bf16 -> x_q [S*K][H] E4M3 and x_sf [S*K][H/32] at the rows of row_id_map.
+moe_status launch_mx_permute_quantize(const void* x, int64_t S, int64_t H, int32_t K,
+                                      const int32_t* row_id_map, void* xq, void* xsf,
+                                      cudaStream_t stream);
+
+// One MXFP8 pass. dual: h_q/h_sf = SwiGLU pass (w0 = gate, w1 = up, act = x_q/x_sf);
+// otherwise y (bf16) = down pass (w0 = down, act = h_q/h_sf, out_sf unused).
+moe_status launch_mx_ffn_pass(bool dual, const void* act_q, const void* act_sf, const void* w0_q,
+                              const void* w0_sf, const void* w1_q, const void* w1_sf,
+                              const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp,
+                              int32_t E, void* out, void* out_sf, int32_t* d_status,
+                              cudaStream_t stream);
+
 }  // namespace moe

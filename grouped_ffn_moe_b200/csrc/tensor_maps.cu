@@ -69,6 +69,19 @@ bool make_f32_tile_map(CUtensorMap* m, void* ptr, uint64_t inner, uint64_t rows,
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_u8_tile_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows,
+                      uint32_t box_inner, uint32_t box_rows) {
+  auto enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 uint64_t wait_budget_ns() {
   static uint64_t budget = [] {
     const char* s = std::getenv("MOE_WAIT_BUDGET_NS");

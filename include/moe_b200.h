@@ -337,6 +337,74 @@ moe_status moe_permute_backward(const void* grad_x_perm, const int32_t* row_id_m
 moe_status moe_maxvio(const int32_t* counts, int32_t E, int64_t S, int32_t K, double* maxvio,
                       int32_t* max_count, void* cuda_stream);
 
+/*
+ * MXFP8 expert FFN ("Mixture of Kittens" digest, Step 8: the expert GEMMs run in MXFP8). The
+ * format is that of the OCP Microscaling Formats v1.0: blocks of 32 consecutive elements along
+ * the reduction dimension share one E8M0 scale 2^s, s = floor(log2(amax of the block)) - 8
+ * (at least -127; s = -127 for an all-zero block), stored as the byte s + 127; each element is
+ * v / 2^s rounded to FP8 E4M3, nearest-even, magnitudes above 448 saturating to 448.
+ *
+ * moe_mx_quantize_weights - quantise one projection's weights once, ahead of the layer:
+ *   w     [E, R, C] bf16, device, C contiguous, R the reduction dimension (R = H, C = H' for
+ *         W_gate and W_up; R = H', C = H for W_down).
+ *   w_q   [E, R, C] uint8 out: E4M3 codes, same layout as w.
+ *   w_sf  uint8 out, moe_mx_weight_scale_bytes(E, R, C) = E*R*C/32 bytes: the scale of rows
+ *         32b..32b+31 of column c of expert e is the byte
+ *           ((e*(C/128) + c/128)*(R/128) + b/4)*512 + (c%128 % 32)*16 + (c%128 / 32)*4 + b%4,
+ *         i.e. one 512-byte chunk per 128 columns x 128 rows, in the order the block-scaled
+ *         tensor-core MMA takes its scales.
+ *   Requires R % 128 == 0, C % 128 == 0; w, w_q, w_sf 16-byte aligned; caller-owned buffers.
+ */
+size_t moe_mx_weight_scale_bytes(int32_t E, int64_t R, int64_t C);
+
+moe_status moe_mx_quantize_weights(const void* w, int32_t E, int64_t R, int64_t C, void* w_q,
+                                   void* w_sf, void* cuda_stream);
+
+/*
+ * moe_mx_permute_quantize - moe_permute's row copy fused with the activations' quantisation:
+ * each token row of x is quantised once (blocks of 32 along H) and its codes and scales are
+ * written to the K rows row_id_map[t*K+k] of the expert-grouped order (rows of -1 skipped):
+ *   x      [S, H] bf16 in.   row_id_map [S*K] int32 from moe_permute (which may be called with
+ *   x_perm = NULL to produce the routing only).
+ *   x_q    [S*K, H] uint8 out (E4M3);  x_sf [S*K, H/32] uint8 out (E8M0, row-major).
+ *   Requires H % 128 == 0; x, x_q, x_sf 16-byte aligned. Launched as a dependent of the
+ *   preceding kernel on the stream (programmatic dependent launch).
+ */
+moe_status moe_mx_permute_quantize(const void* x, const int32_t* row_id_map, int64_t S, int64_t H,
+                                   int32_t K, void* x_q, void* x_sf, void* cuda_stream);
+
+/*
+ * moe_grouped_ffn_mxfp8 - moe_grouped_ffn in MXFP8 on block-scaled tcgen05 MMAs (fp32
+ * accumulation):
+ *   h[r] = silu(x[r] . Wg[e]) * (x[r] . Wu[e])   with x, Wg, Wu the dequantised MXFP8 values,
+ *          stored quantised to MXFP8 along H' (h_q [M, Hp] uint8, h_sf [M, Hp/32] uint8) --
+ *          the quantisation runs in the SwiGLU epilogue on the fp32 values;
+ *   y[r] = bf16(h[r] . Wd[e])                   (dequantised h_q and W_down).
+ *   x_q, x_sf  [M, H], [M, H/32] from moe_mx_permute_quantize.
+ *   *_q, *_sf  weights from moe_mx_quantize_weights (W_gate, W_up: R = H, C = Hp; W_down:
+ *              R = Hp, C = H).
+ *   cu_seqlens, M, H, Hp, E, d_status and the requirements as moe_grouped_ffn; y [M, H] bf16.
+ *
+ * moe_grouped_ffn_up_gate_mxfp8 and moe_grouped_ffn_down_mxfp8 are its two passes alone.
+ */
+moe_status moe_grouped_ffn_mxfp8(const void* x_q, const void* x_sf, const void* w_gate_q,
+                                 const void* w_gate_sf, const void* w_up_q, const void* w_up_sf,
+                                 const void* w_down_q, const void* w_down_sf,
+                                 const int32_t* cu_seqlens, int64_t M, int64_t H, int64_t Hp,
+                                 int32_t E, void* h_q, void* h_sf, void* y, int32_t* d_status,
+                                 void* cuda_stream);
+
+moe_status moe_grouped_ffn_up_gate_mxfp8(const void* x_q, const void* x_sf, const void* w_gate_q,
+                                         const void* w_gate_sf, const void* w_up_q,
+                                         const void* w_up_sf, const int32_t* cu_seqlens, int64_t M,
+                                         int64_t H, int64_t Hp, int32_t E, void* h_q, void* h_sf,
+                                         int32_t* d_status, void* cuda_stream);
+
+moe_status moe_grouped_ffn_down_mxfp8(const void* h_q, const void* h_sf, const void* w_down_q,
+                                      const void* w_down_sf, const int32_t* cu_seqlens, int64_t M,
+                                      int64_t H, int64_t Hp, int32_t E, void* y, int32_t* d_status,
+                                      void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

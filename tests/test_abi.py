@@ -132,3 +132,44 @@ def test_host_validation_of_backward_gather_and_shared_calls():
     assert L.moe_append_shared(a, a, 4, 2, 1024, 1, a, a, null) == 2
     assert L.moe_append_shared(a, a, 4, 2, 8, 0, a, a, null) == 1
     assert L.moe_append_shared(a, a, 0, 2, 8, 1, a, a, null) == 0
+
+
+def test_host_validation_of_mxfp8_calls():
+    L = moe.lib()
+    a = fake(0x10000)
+    null = P(0)
+    # scale bytes: E*R*C/32 for multiples of 128, else 0
+    assert moe.moe_mx_weight_scale_bytes(2, 256, 384) == 2 * 8 * 384
+    assert moe.moe_mx_weight_scale_bytes(2, 200, 384) == 0
+    # weight quantisation: R or C not a multiple of 128; null or misaligned buffers
+    assert L.moe_mx_quantize_weights(a, 2, 192, 256, a, a, null) == 2
+    assert L.moe_mx_quantize_weights(a, 2, 256, 160, a, a, null) == 2
+    assert L.moe_mx_quantize_weights(a, 0, 256, 256, a, a, null) == 1
+    assert L.moe_mx_quantize_weights(a, 2, 256, 256, null, a, null) == 1
+    assert L.moe_mx_quantize_weights(a, 2, 256, 256, a, fake(0x10004), null) == 1
+    # permute-quantise: H % 128, missing row map, misaligned outputs; S == 0 is a no-op
+    assert L.moe_mx_permute_quantize(a, a, 16, 96, 2, a, a, null) == 2
+    assert L.moe_mx_permute_quantize(a, null, 16, 256, 2, a, a, null) == 1
+    assert L.moe_mx_permute_quantize(a, a, 16, 256, 2, a, fake(0x10008), null) == 1
+    assert L.moe_mx_permute_quantize(null, null, 0, 256, 2, null, null, null) == 0
+    # FFN passes: shapes as moe_grouped_ffn; every operand required; M == 0 is a no-op
+    args_ug = [a, a, a, a, a, a, a, 64, 256, 256, 4, a, a, null, null]
+    bad = list(args_ug)
+    bad[8] = 200  # H % 128
+    assert L.moe_grouped_ffn_up_gate_mxfp8(*bad) == 2
+    bad = list(args_ug)
+    bad[1] = null  # x_sf
+    assert L.moe_grouped_ffn_up_gate_mxfp8(*bad) == 1
+    bad = list(args_ug)
+    bad[12] = fake(0x10002)  # h_sf misaligned
+    assert L.moe_grouped_ffn_up_gate_mxfp8(*bad) == 1
+    zero = list(args_ug)
+    zero[7] = 0
+    assert L.moe_grouped_ffn_up_gate_mxfp8(*zero) == 0
+    assert L.moe_grouped_ffn_down_mxfp8(a, null, a, a, a, 64, 256, 256, 4, a, null, null) == 1
+    assert L.moe_grouped_ffn_down_mxfp8(a, a, a, a, a, 64, 256, 384 + 64, 4, a, null, null) == 2
+    assert L.moe_grouped_ffn_down_mxfp8(a, a, a, a, a, 0, 256, 256, 4, a, null, null) == 0
+    assert L.moe_grouped_ffn_mxfp8(a, a, a, a, a, a, a, null, a, 64, 256, 256, 4, a, a, a, null,
+                                   null) == 1
+    assert L.moe_grouped_ffn_mxfp8(a, a, a, a, a, a, a, a, a, 64, 256, 256, 0, a, a, a, null,
+                                   null) == 1
