@@ -53,6 +53,9 @@ def parse_args():
                         "routing and run them in the same launches (no e2e or training leg)")
     p.add_argument("--no-backward", action="store_true",
                    help="skip the training-step leg (forward with saved pre-activations + backward)")
+    p.add_argument("--mxfp8", action="store_true",
+                   help="experts in MXFP8 (E4M3 + E8M0 block scales): weights quantised once "
+                        "before timing, activations quantised inside the step")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="CPU work budget for the oracle baseline sample")
     return p.parse_args()
@@ -62,6 +65,7 @@ KERNEL_SOURCES = {
     # the files a kernel is compiled from: a recorded traffic figure holds only for them
     "up_gate": ["grouped_ffn.cu", "gemm_common.cuh", "ptx.cuh"],
     "weight_grad": ["grouped_ffn_bwd.cu", "gemm_common.cuh", "ptx.cuh"],
+    "up_gate_mx": ["grouped_ffn_mx.cu", "gemm_common.cuh", "ptx.cuh"],
 }
 
 
@@ -141,6 +145,11 @@ def work_model(w, counts=None):
         m["up_gate_bwd_bytes"] = 2 * 2 * active * H * Hp + 2 * 2 * M * Hp + 2 * M * H
         m["wgrad_flops"] = 6 * M * H * Hp
         m["wgrad_bytes"] = 4 * 3 * E * H * Hp + 2 * M * (2 * H + 3 * Hp)
+        # MXFP8: one byte per element plus one scale byte per 32 (weights, x_q, h_q)
+        q = 33 / 32
+        m["permute_mx_bytes"] = 2 * S * H + q * M * H + 12 * M + 8 * E
+        m["up_gate_mx_bytes"] = q * (2 * active * H * Hp + M * H + M * Hp)
+        m["down_mx_bytes"] = q * (active * Hp * H + M * Hp) + 2 * M * H
     return m
 
 
@@ -362,20 +371,37 @@ def run_ours(args):
     ids_step = ids_ext if ns else inp["topk_ids"]
     w_step = w_ext if ns else inp["route_w"]
 
-    zero_copy = args.zero_copy and not w.identity_ffn
+    mx = args.mxfp8 and not w.identity_ffn and not ns
+    zero_copy = args.zero_copy and not w.identity_ffn and not mx
+    if mx:
+        # weights quantised once, ahead of the layer (not part of a step)
+        mw = moe.MxWeights.from_bf16(inp["w_gate"], inp["w_up"], inp["w_down"])
+        mxbufs = [moe.MxBuffers.allocate(w.S, w.H, w.Hp, K, dev)]
+        mxbuf = mxbufs[0]
+        torch.cuda.synchronize()
 
     def step(ev=None):
         if ev is not None:
             ev[0].record()
         if ns:
             moe.moe_append_shared(inp["topk_ids"], inp["route_w"], w.E, ns, ids_ext, w_ext)
-        moe.moe_permute(inp["x"], ids_step, E, None if zero_copy else buf.x_perm,
+        moe.moe_permute(inp["x"], ids_step, E, None if (zero_copy or mx) else buf.x_perm,
                         buf.counts, buf.cu_seqlens, buf.row_id_map, buf.perm_src, buf.maxvio,
                         buf.max_count, buf.workspace, buf.d_status)
+        if mx:
+            moe.moe_mx_permute_quantize(inp["x"], buf.row_id_map, K, mxbuf.x_q, mxbuf.x_sf)
         if ev is not None:
             ev[1].record()
         y = buf.x_perm
-        if not w.identity_ffn:
+        if mx:
+            moe.moe_grouped_ffn_up_gate_mxfp8(mxbuf.x_q, mxbuf.x_sf, mw, buf.cu_seqlens,
+                                              mxbuf.h_q, mxbuf.h_sf, buf.d_status)
+            if ev is not None:
+                ev[2].record()
+            moe.moe_grouped_ffn_down_mxfp8(mxbuf.h_q, mxbuf.h_sf, mw, buf.cu_seqlens, buf.y,
+                                           buf.d_status)
+            y = buf.y
+        elif not w.identity_ffn:
             if zero_copy:
                 moe.moe_grouped_ffn_up_gate_gather(inp["x"], buf.perm_src, K, inp["w_gate"],
                                                    inp["w_up"], buf.cu_seqlens, buf.h,
@@ -398,8 +424,9 @@ def run_ours(args):
             ev[4].record()
 
     # the metadata-only permute (zero copy) launches one kernel, not the row copy
-    launches_per_step = (moe.LAUNCHES["moe_permute"] - (1 if zero_copy else 0)
+    launches_per_step = (moe.LAUNCHES["moe_permute"] - (1 if (zero_copy or mx) else 0)
                          + moe.LAUNCHES["moe_unpermute_combine"]
+                         + (moe.LAUNCHES["moe_mx_permute_quantize"] if mx else 0)
                          + (0 if w.identity_ffn else moe.LAUNCHES["moe_grouped_ffn"])
                          + (moe.LAUNCHES["moe_append_shared"] + moe.LAUNCHES["moe_maxvio"]
                             if ns else 0))
@@ -473,6 +500,16 @@ def run_ours(args):
         dw = [torch.empty_like(inp["route_w"]) for _ in range(2)]
         bufs = [buf, moe.LayerBuffers.allocate(w.S, w.H, w.Hp, E, K, dev,
                                                with_ffn=not w.identity_ffn)]
+        if mx:
+            mxbufs.append(moe.MxBuffers.allocate(w.S, w.H, w.Hp, K, dev))
+
+        def layer(k, stream):
+            if mx:
+                return moe.moe_layer_forward_mxfp8(dx[k], dids[k], dw[k], mw, bufs[k], mxbufs[k],
+                                                   stream=stream)
+            return moe.moe_layer_forward(dx[k], dids[k], dw[k], inp.get("w_gate"),
+                                         inp.get("w_up"), inp.get("w_down"), bufs[k],
+                                         stream=stream, zero_copy=zero_copy)
         s_up, s_run, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), \
             torch.cuda.Stream(dev)
         h2d_bytes = hx.numel() * 2 + hids.numel() * 4 + hw.numel() * 4
@@ -495,9 +532,7 @@ def run_ours(args):
                     s_run.wait_event(up)
                     if read[k] is not None:
                         s_run.wait_event(read[k])
-                    out = moe.moe_layer_forward(dx[k], dids[k], dw[k], inp.get("w_gate"),
-                                                inp.get("w_up"), inp.get("w_down"), bufs[k],
-                                                stream=s_run, zero_copy=zero_copy)
+                    out = layer(k, s_run)
                     ran[k] = torch.cuda.Event()
                     ran[k].record(s_run)
                 with torch.cuda.stream(s_down):
@@ -512,9 +547,7 @@ def run_ours(args):
                     dx[0].copy_(hx, non_blocking=True)
                     dids[0].copy_(hids, non_blocking=True)
                     dw[0].copy_(hw, non_blocking=True)
-                    out = moe.moe_layer_forward(dx[0], dids[0], dw[0], inp.get("w_gate"),
-                                                inp.get("w_up"), inp.get("w_down"), bufs[0],
-                                                stream=s_run, zero_copy=zero_copy)
+                    out = layer(0, s_run)
                     hout[0].copy_(out, non_blocking=True)
 
         def timed(fn):
@@ -548,7 +581,7 @@ def run_ours(args):
                               "ms_per_step": serial_ms}}
 
     backward = None
-    if not w.identity_ffn and not args.no_backward and not ns:
+    if not w.identity_ffn and not args.no_backward and not ns and not mx:
         peaks0, src0 = load_peaks()
         backward = measure_backward(moe, synth, torch, w, inp, dev, args.steps, args.warmup, flush,
                                     peaks0, src0)
@@ -561,7 +594,8 @@ def run_ours(args):
         wm = work_model(dataclasses.replace(w, E=E, K=K), counts)
         stages = {
             "permute": {"ms": mean["permute"],
-                        "GB/s": wm["permute_bytes"] / (mean["permute"] / 1e3) / 1e9},
+                        "GB/s": wm["permute_mx_bytes" if mx else "permute_bytes"]
+                        / (mean["permute"] / 1e3) / 1e9},
             "combine": {"ms": mean["combine"],
                         "GB/s": wm["combine_bytes"] / (mean["combine"] / 1e3) / 1e9},
         }
@@ -574,30 +608,39 @@ def run_ours(args):
                 "ms": mean["ffn"],
                 "TFLOP/s": (wm["up_gate_flops"] + wm["down_flops"]) / (mean["ffn"] / 1e3) / 1e12}
             # dominant kernel: the SwiGLU (up/gate) pass
-            flops, byts, t_s = wm["up_gate_flops"], wm["up_gate_bytes"], mean["up_gate"] / 1e3
-            ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+            flops, t_s = wm["up_gate_flops"], mean["up_gate"] / 1e3
+            byts = wm["up_gate_mx_bytes" if mx else "up_gate_bytes"]
+            kname = ("grouped_ffn_mx_kernel<true> (MXFP8 up/gate + SwiGLU + h quantisation)" if mx
+                     else "grouped_ffn_kernel<0> (up/gate + SwiGLU)")
+            # MXFP8: the measured bf16 peak times the nominal fp8:bf16 ratio (4.5 / 2.25)
+            tpeak = peaks["bf16_tflops"] * (2.0 if mx else 1.0)
+            ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)
             if flops / byts >= ridge:
-                roof = {"kernel": "grouped_ffn_kernel<0> (up/gate + SwiGLU)", "bound": "tensor",
-                        "achieved": flops / t_s / 1e12, "peak": peaks["bf16_tflops"],
-                        "unit": "TFLOP/s"}
+                roof = {"kernel": kname, "bound": "tensor", "achieved": flops / t_s / 1e12,
+                        "peak": tpeak, "unit": "TFLOP/s"}
             else:
-                roof = {"kernel": "grouped_ffn_kernel<0> (up/gate + SwiGLU)", "bound": "hbm",
-                        "achieved": byts / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+                roof = {"kernel": kname, "bound": "hbm", "achieved": byts / t_s / 1e9,
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s"}
         else:
             byts, t_s = wm["permute_bytes"], mean["permute"] / 1e3
             roof = {"kernel": "moe_permute (2 kernels)", "bound": "hbm", "achieved": byts / t_s / 1e9,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["peak_source"] = f"{peak_src} (burst)"
-        roof["traffic"] = (profiled_traffic(f"up_gate/{w.name}") if not w.identity_ffn
-                           else None)
+        if mx and roof["bound"] == "tensor":
+            roof["peak_source"] = f"{peak_src} bf16 (burst) x 2, the nominal fp8:bf16 ratio"
+        roof["traffic"] = (profiled_traffic(f"{'up_gate_mx' if mx else 'up_gate'}/{w.name}")
+                           if not w.identity_ffn else None)
         line = {
             "metric": METRIC, "value": job_throughput(w.S, world, ms_step), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "mxfp8 (e4m3, e8m0 scales per 32; fp32 accumulate; bf16 y/out)" if mx
+            else "bf16",
             "data": "synthetic (seeded SplitMix64/Box-Muller inputs, random-init expert weights)",
             "config": {"workload": w.name, "S": w.S, "H": w.H, "Hp": w.Hp, "E": w.E, "K": w.K,
-                       "path": "zero-copy (gather)" if zero_copy else "x_perm copy",
+                       "path": ("mxfp8 (permute fused with quantisation)" if mx else
+                                "zero-copy (gather)" if zero_copy else "x_perm copy"),
                        "shared_experts": ns,
                        "routing": w.routing, "maxvio_measured": maxvio,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -611,7 +654,8 @@ def run_ours(args):
         if backward is not None:
             line["training_step"] = backward
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
+            line["cpu_baseline"] = (cpu_baseline_mx(w, inp, args.cpu_seconds) if mx
+                                    else cpu_baseline(w, inp, args.cpu_seconds))
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -670,6 +714,43 @@ def cpu_baseline(w, inp, budget_s):
     return {"value": done / el, "unit": UNIT, "cores": _cores(), "kind": "oracle",
             "sample": f"first {S_sample} tokens of workload {w.name} (full weights), "
                       f"repeated for {el:.1f} s; numpy fp64"}
+
+
+def cpu_baseline_mx(w, inp, budget_s, n_tokens=2):
+    """The oracle's MXFP8 expert path (permutation, per-row quantisation, expert_ffn_rows_mxfp8,
+    combine) on the first n_tokens tokens; the weights of the experts they visit are quantised
+    once beforehand, as the GPU run quantises them before timing."""
+    import numpy as np
+
+    from oracle import moe_oracle as O
+
+    host = _host_inputs_from_device(w, inp)
+    S, K = n_tokens, w.K
+    ids = host["topk_ids"][:S]
+    rw = host["route_w"][:S]
+    x = host["x"][:S]
+    qw = {}
+    for e in sorted(set(int(v) for v in np.asarray(ids).ravel())):
+        wg, wu, wd = host["get"](e)
+        qw[e] = (O.mx_weights(wg), O.mx_weights(wu), O.mx_weights(wd))
+    done, t_start = 0, time.perf_counter()
+    while True:
+        counts, cu, rmap, psrc = O.permute_metadata(ids, w.E)
+        x_perm = O.permute_rows(x, psrc, K)
+        y = np.zeros((S * K, w.H), np.uint16)
+        for e in range(w.E):
+            r0, r1 = int(cu[e]), int(cu[e + 1])
+            if r1 > r0:
+                y[r0:r1] = O.expert_ffn_rows_mxfp8(x_perm[r0:r1], *qw[e])[2]
+        O.unpermute_combine(y, rmap, rw, S, K)
+        done += S
+        el = time.perf_counter() - t_start
+        if el >= budget_s:
+            break
+    return {"value": done / el, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "sample": f"first {S} tokens of workload {w.name}, MXFP8 oracle path (weights of "
+                      f"their {len(qw)} experts quantised beforehand), repeated for {el:.1f} s; "
+                      f"numpy fp64"}
 
 
 def run_reference(args):

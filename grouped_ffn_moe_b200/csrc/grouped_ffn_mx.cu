@@ -23,7 +23,8 @@
 //               reads the scale of operand row f for its k block kb (the byte is selected by
 //               bits 30-31 of the scale address and the sf_id fields of the descriptor).
 //   activations q [M][D] E4M3, sf [M][D/32] E8M0 (D = H for x, H' for h). A scale warp
-//               rearranges each stage's 4 bytes per token row into the same chunk order.
+//               copies each stage's 4 bytes per token row into the same chunk order (4-byte
+//               cp.async, completion counted on the stage's barrier).
 //
 // Tiles as in grouped_ffn.cu ("swap AB": M = 128 features, N = the unit's tokens), with units of
 // at most 224 tokens so that the accumulators and the scales of every pipeline stage share the
@@ -141,6 +142,12 @@ __device__ __forceinline__ void umma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// 4-byte asynchronous global -> shared copy (generic proxy, like cp_async_16).
+__device__ __forceinline__ void cp_async_4(uint32_t smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_dst), "l"(gmem_src)
+               : "memory");
+}
+
 // Contiguous global -> shared bulk copy (16-byte aligned addresses, size a multiple of 16),
 // completion counted on `bar` in bytes.
 __device__ __forceinline__ void bulk_load_hint(void* smem_dst, const void* src, uint32_t bytes,
@@ -208,7 +215,8 @@ __global__ void __launch_bounds__(MxCfg<kSwi>::kBlock, 1)
   // ------------------------------------------------------------------ prologue
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 2);  // the TMA lane's arrive.expect_tx + the scale warp's arrival
+      // the TMA lane's arrive.expect_tx + one cp.async arrival per scale-warp lane
+      mbar_init(&full[s], 1 + 32);
       mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -239,10 +247,12 @@ __global__ void __launch_bounds__(MxCfg<kSwi>::kBlock, 1)
 
   // ------------------------------------------------------------------ roles
   if (warp == kMxScaleWarp) {
-    // Activation scales: per stage, token i = lane + 32 j (j < 8) of the unit contributes its
-    // 4 scale bytes (k blocks 4 kt .. 4 kt + 3) to chunk i / 128 at line i % 32, word
-    // (i / 32) % 4. Rows past the unit (up to 256) get scale 1 (their MMA columns are not
-    // stored). The next stage's loads are issued before waiting for the slot.
+    // Activation scales: per stage, token i = lane + 32 j (j < 8, i < the unit's rows) copies
+    // its 4 scale bytes (k blocks 4 kt .. 4 kt + 3) with a 4-byte cp.async to chunk i / 128,
+    // line i % 32, word (i / 32) % 4; each lane then arrives on the stage's full barrier when
+    // its copies land, so the copies overlap like the TMA loads (as deep as the stage ring).
+    // Rows past the unit (up to the 16-row rounding) keep whatever the slot held: their MMA
+    // columns are never stored.
     int stage = 0;
     uint32_t phase = 0;
     bool stop = false;
@@ -251,44 +261,29 @@ __global__ void __launch_bounds__(MxCfg<kSwi>::kBlock, 1)
       const Unit U = decode_unit<kMxN>(u, s_ustart, s_cu, E);
       if (U.nrows <= 0) continue;
       const uint8_t* base = args.act_sf + static_cast<int64_t>(U.row0) * sf_row;
-      uint32_t nxt[8];
-      auto load = [&](int kt, uint32_t (&v)[8]) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i = lane + 32 * j;
-          v[j] = i < U.nrows ? __ldg(reinterpret_cast<const uint32_t*>(
-                                   base + static_cast<int64_t>(i) * sf_row + kt * 4))
-                             : 0x7F7F7F7Fu;
-        }
-      };
-      load(0, nxt);
       for (int kt = 0; kt < KT; ++kt) {
-        uint32_t cur[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
-        if (kt + 1 < KT) load(kt + 1, nxt);
         int ok = 1;
         if (lane == 0) ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, s_abort, args.budget_ns);
         if (!__shfl_sync(0xffffffffu, ok, 0)) {
           stop = true;
           break;
         }
-        uint8_t* sfb = smem + stage * C::kStageBytes + C::kOffSfb;
+        const uint32_t sfb = smem_u32(smem + stage * C::kStageBytes + C::kOffSfb);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int i = lane + 32 * j;
-          *reinterpret_cast<uint32_t*>(sfb + (i >> 7) * kMxChunk + (i & 31) * 16 +
-                                       ((i >> 5) & 3) * 4) = cur[j];
+          if (i < U.nrows)
+            cp_async_4(sfb + (i >> 7) * kMxChunk + (i & 31) * 16 + ((i >> 5) & 3) * 4,
+                       base + static_cast<int64_t>(i) * sf_row + kt * 4);
         }
-        fence_proxy_async_smem();  // generic-proxy writes, read next by tcgen05.cp
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[stage]);
+        cp_async_mbar_arrive_noinc(&full[stage]);
         if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // own copies land before the CTA exits
   } else if (warp == 0) {
     // TMA producer
     if (lane == 0) {
@@ -366,6 +361,7 @@ __global__ void __launch_bounds__(MxCfg<kSwi>::kBlock, 1)
             ok = false;
             break;
           }
+          fence_proxy_async_smem();  // the activation scales arrived by cp.async (generic proxy)
           tc_fence_after();
           const uint32_t st = smem_u32(smem + stage * C::kStageBytes);
           const uint32_t sf = tmem_base + kMxSfCol + stage * kMxSfStageCols;
