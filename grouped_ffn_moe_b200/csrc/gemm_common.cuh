@@ -135,11 +135,6 @@ bool make_weight_map(CUtensorMap* m, const void* ptr, uint64_t n_feat, uint64_t 
 // (box_inner * 4 must be 128): the staging layout of a TMA store or reduce-add.
 bool make_f32_tile_map(CUtensorMap* m, void* ptr, uint64_t inner, uint64_t rows,
                        uint32_t box_inner, uint32_t box_rows);
-// A row-major byte matrix [rows][inner] (E4M3 elements) with a (box_inner x box_rows) box,
-// 128-byte swizzle (box_inner must be 128): K-major token tiles and MN-major weight tiles of
-// the MXFP8 passes.
-bool make_u8_tile_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows,
-                      uint32_t box_inner, uint32_t box_rows);
 // Bound, in nanoseconds, of every pipeline wait in the GEMM kernels (MOE_WAIT_BUDGET_NS).
 uint64_t wait_budget_ns();
 

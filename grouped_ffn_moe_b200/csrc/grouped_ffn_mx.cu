@@ -42,6 +42,13 @@
 #include "gemm_common.cuh"
 
 namespace moe {
+
+// Host-side builder (tensor_maps.cu): a row-major byte matrix [rows][inner] (E4M3 elements)
+// with a (box_inner x box_rows) box, 128-byte swizzle (box_inner must be 128): the K-major token
+// tiles and MN-major weight tiles of the MXFP8 passes.
+bool make_u8_tile_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows,
+                      uint32_t box_inner, uint32_t box_rows);
+
 namespace {
 
 constexpr int kMxBK = 128;                  // k elements (= bytes) per stage

@@ -8,6 +8,13 @@
  *   moe_unpermute_combine  out[t] = sum_k w[t,k] * y[row of (t,k)]
  *   moe_maxvio             max_e(T_e / T_bar) - 1
  *
+ * Further calls, each documented where it is declared: the permutation without a workspace
+ * argument (moe_permute_no_alloc); the layer's backward (moe_combine_backward,
+ * moe_grouped_ffn_*_backward, moe_grouped_ffn_weight_grad, moe_permute_backward); the SwiGLU
+ * pass reading token rows in place (moe_grouped_ffn_gather); shared experts
+ * (moe_append_shared); and experts in MXFP8 (moe_mx_quantize_weights,
+ * moe_mx_permute_quantize, moe_grouped_ffn_*mxfp8; "Mixture of Kittens" digest, Step 8).
+ *
  * Sources (page title, section):
  *   "Distributed expert parallelism" (open-llm-engineering): "The dispatch-compute-combine
  *     lifecycle" (copy each token k times, sort copies by expert, grouped expert FFNs,

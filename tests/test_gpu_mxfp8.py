@@ -230,3 +230,33 @@ def test_mx_layer_end_to_end(cuda_device):
     out_r = O.unpermute_combine(y_r, rmap, np.asarray(rw, np.float32), S, K)
     st = assert_close_bf16(bits(out), out_r, "layer out")
     print(f"layer out {st}")
+
+
+def test_mx_device_wait_timeout_reports_status(cuda_device):
+    """Failure detection without a fault: with a 1 ns wait budget the MXFP8 passes' pipeline
+    waits run out; they record MOE_ERR_DEVICE_TIMEOUT, drain their own copies (TMA, the scale
+    warp's cp.async) and MMAs, free TMEM and return, and the CUDA context stays usable."""
+    import os
+    import subprocess
+    import sys
+
+    script = (
+        "import torch, synth, grouped_ffn_moe_b200 as moe\n"
+        "w = synth.WORKLOADS['tiny']\n"
+        "dev = torch.device('cuda:0')\n"
+        "inp = synth.make_layer_inputs(w, device='cuda:0')\n"
+        "mw = moe.MxWeights.from_bf16(inp['w_gate'], inp['w_up'], inp['w_down'])\n"
+        "buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev)\n"
+        "mxb = moe.MxBuffers.allocate(w.S, w.H, w.Hp, w.K, dev)\n"
+        "moe.moe_layer_forward_mxfp8(inp['x'], inp['topk_ids'], inp['route_w'], mw, buf, mxb)\n"
+        "torch.cuda.synchronize()\n"
+        "st = int(buf.d_status.item())\n"
+        "assert st & moe.MOE_ERR_DEVICE_TIMEOUT, st\n"
+        "assert torch.arange(1000, device='cuda:0').sum().item() == 499500\n"
+        "print('timeout status', st)\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, PYTHONPATH=root, MOE_WAIT_BUDGET_NS="1")
+    r = subprocess.run([sys.executable, "-c", script], env=env, cwd=root, timeout=600,
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "timeout status" in r.stdout
