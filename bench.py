@@ -58,7 +58,11 @@ def parse_args():
                         "before timing, activations quantised inside the step")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="CPU work budget for the oracle baseline sample")
-    return p.parse_args()
+    args = p.parse_args()
+    if args.mxfp8 and (args.shared_experts or args.zero_copy):
+        p.error("--mxfp8 runs its own permute-quantise path: it does not combine with "
+                "--shared-experts or --zero-copy")
+    return args
 
 
 KERNEL_SOURCES = {
