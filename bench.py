@@ -720,40 +720,53 @@ def cpu_baseline(w, inp, budget_s):
                       f"repeated for {el:.1f} s; numpy fp64"}
 
 
-def cpu_baseline_mx(w, inp, budget_s, n_tokens=2):
-    """The oracle's MXFP8 expert path (permutation, per-row quantisation, expert_ffn_rows_mxfp8,
-    combine) on the first n_tokens tokens; the weights of the experts they visit are quantised
-    once beforehand, as the GPU run quantises them before timing."""
+def _mx_oracle_setup(w, host, n_tokens):
+    """The first n_tokens tokens of the workload and the MXFP8 weights of the experts they
+    visit, quantised by the oracle (ahead of timing, as the GPU run quantises its weights)."""
     import numpy as np
 
     from oracle import moe_oracle as O
 
-    host = _host_inputs_from_device(w, inp)
-    S, K = n_tokens, w.K
-    ids = host["topk_ids"][:S]
-    rw = host["route_w"][:S]
-    x = host["x"][:S]
+    ids = host["topk_ids"][:n_tokens]
     qw = {}
     for e in sorted(set(int(v) for v in np.asarray(ids).ravel())):
         wg, wu, wd = host["get"](e)
         qw[e] = (O.mx_weights(wg), O.mx_weights(wu), O.mx_weights(wd))
+    return ids, qw
+
+
+def _oracle_sample_mx(w, host, ids, qw):
+    """The oracle's MXFP8 layer on the tokens of `ids`: permutation, expert_ffn_rows_mxfp8
+    per expert (x and h quantised inside), combine."""
+    import numpy as np
+
+    from oracle import moe_oracle as O
+
+    S, K = ids.shape
+    counts, cu, rmap, psrc = O.permute_metadata(ids, w.E)
+    x_perm = O.permute_rows(host["x"][:S], psrc, K)
+    y = np.zeros((S * K, w.H), np.uint16)
+    for e in range(w.E):
+        r0, r1 = int(cu[e]), int(cu[e + 1])
+        if r1 > r0:
+            y[r0:r1] = O.expert_ffn_rows_mxfp8(x_perm[r0:r1], *qw[e])[2]
+    return O.unpermute_combine(y, rmap, host["route_w"][:S], S, K)
+
+
+def cpu_baseline_mx(w, inp, budget_s, n_tokens=2):
+    """The oracle's MXFP8 layer on the first n_tokens tokens, repeated for budget_s."""
+    host = _host_inputs_from_device(w, inp)
+    ids, qw = _mx_oracle_setup(w, host, n_tokens)
     done, t_start = 0, time.perf_counter()
     while True:
-        counts, cu, rmap, psrc = O.permute_metadata(ids, w.E)
-        x_perm = O.permute_rows(x, psrc, K)
-        y = np.zeros((S * K, w.H), np.uint16)
-        for e in range(w.E):
-            r0, r1 = int(cu[e]), int(cu[e + 1])
-            if r1 > r0:
-                y[r0:r1] = O.expert_ffn_rows_mxfp8(x_perm[r0:r1], *qw[e])[2]
-        O.unpermute_combine(y, rmap, rw, S, K)
-        done += S
+        _oracle_sample_mx(w, host, ids, qw)
+        done += n_tokens
         el = time.perf_counter() - t_start
         if el >= budget_s:
             break
     return {"value": done / el, "unit": UNIT, "cores": _cores(), "kind": "oracle",
-            "sample": f"first {S} tokens of workload {w.name}, MXFP8 oracle path (weights of "
-                      f"their {len(qw)} experts quantised beforehand), repeated for {el:.1f} s; "
+            "sample": f"first {n_tokens} tokens of workload {w.name}, MXFP8 oracle path (weights "
+                      f"of their {len(qw)} experts quantised beforehand), repeated for {el:.1f} s; "
                       f"numpy fp64"}
 
 
@@ -767,24 +780,33 @@ def run_reference(args):
     w = synth.WORKLOADS[args.workload]
     inp = synth.make_layer_inputs(w, device="cpu")
     host = _host_inputs_from_device(w, inp)
-    S_sample = min(w.S, _sample_tokens(w))
+    mx = args.mxfp8 and not w.identity_ffn
+    if mx:
+        S_sample = 2
+        ids, qw = _mx_oracle_setup(w, host, S_sample)
+        run = lambda: _oracle_sample_mx(w, host, ids, qw)  # noqa: E731
+    else:
+        S_sample = min(w.S, _sample_tokens(w))
+        run = lambda: _oracle_sample(w, S_sample, host)  # noqa: E731
     for _ in range(args.warmup):
-        _oracle_sample(w, S_sample, host)
+        run()
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        _oracle_sample(w, S_sample, host)
+        run()
         times.append(time.perf_counter() - t0)
     sec = sum(times) / len(times)
     value = S_sample / sec
     sample = (f"first {S_sample} of {w.S} tokens of workload {w.name} per step (full weights); "
-              f"numpy fp64 oracle")
+              f"numpy fp64 oracle" + (", MXFP8 path (the visited experts' weights quantised "
+                                      "before timing)" if mx else ""))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": w.name, "S": w.S, "H": w.H, "Hp": w.Hp,
-                                        "E": w.E, "K": w.K, "routing": w.routing},
+                                        "E": w.E, "K": w.K, "routing": w.routing,
+                                        "path": "mxfp8" if mx else "bf16"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
