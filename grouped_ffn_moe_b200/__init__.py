@@ -8,7 +8,11 @@ Functions carry the C ABI's names:
     moe_permute, moe_grouped_ffn (= moe_grouped_ffn_up_gate + moe_grouped_ffn_down),
     moe_unpermute_combine, moe_maxvio, moe_permute_workspace_bytes, moe_status_string
 plus `LayerBuffers` / `moe_layer_forward`, which allocate the layer's buffers once and
-chain the three calls (permute -> grouped FFN -> combine) on one stream.
+chain the three calls (permute -> grouped FFN -> combine) on one stream; the backward
+(`moe_layer_backward` and its per-stage calls), the in-place token gather
+(`moe_grouped_ffn_gather`), shared experts (`moe_append_shared`) and MXFP8 experts
+(`moe_mx_quantize_weights`, `moe_mx_permute_quantize`, `moe_grouped_ffn_mxfp8`, with
+`MxWeights` / `MxBuffers` / `moe_layer_forward_mxfp8`).
 """
 from __future__ import annotations
 

@@ -37,6 +37,7 @@
 #include <cuda_fp8.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 
 #include "gemm_common.cuh"
@@ -593,17 +594,19 @@ __global__ void __launch_bounds__(256) mx_permute_quantize_kernel(
   }
 }
 
+// The kernel's dynamic shared-memory opt-in, once per device.
 template <bool kSwi>
 bool ensure_mx_smem_attr() {
-  static int done = 0;  // 1 ok, -1 failed
-  if (done == 0) {
-    done = cudaFuncSetAttribute(grouped_ffn_mx_kernel<kSwi>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                MxCfg<kSwi>::kSmemBytes) == cudaSuccess
-               ? 1
-               : -1;
-  }
-  return done == 1;
+  static std::atomic<int> done_dev_mask{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const int bit = 1 << (dev & 31);
+  if (done_dev_mask.load() & bit) return true;
+  if (cudaFuncSetAttribute(grouped_ffn_mx_kernel<kSwi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           MxCfg<kSwi>::kSmemBytes) != cudaSuccess)
+    return false;
+  done_dev_mask.fetch_or(bit);
+  return true;
 }
 
 bool make_mx_row_maps(MxRowMaps* maps, const void* ptr, uint64_t inner, uint64_t rows) {
