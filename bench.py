@@ -7,7 +7,7 @@ fused), moe_grouped_ffn_up_gate, moe_grouped_ffn_down, moe_unpermute_combine. Th
 is flushed before every timed step, outside the timed events (a 256 MiB write, then a
 256 MiB read of another buffer so that the write's dirty lines leave L2 there).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload medium]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload large]
     python bench.py --impl reference ...     (the CPU oracle on the host cores)
 
 Multi-GPU: replicas only (one process per GPU under torchrun, each running the whole
@@ -32,7 +32,7 @@ if ROOT not in sys.path:
 
 METRIC = "MoE layer tokens/sec on 1 B200; grouped-FFN TFLOP/s; permute+combine HBM GB/s"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "medium"
+DEFAULT_WORKLOAD = "large"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -47,7 +47,7 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--zero-copy", action="store_true",
                    help="forward step without x_perm: metadata-only permute, SwiGLU pass "
-                        "gathering its token rows from x (TMA gather4)")
+                        "gathering its token rows from x (cp.async gather warps)")
     p.add_argument("--shared-experts", type=int, default=0,
                    help="append N shared experts (each with the routed experts' shape) to the "
                         "routing and run them in the same launches (no e2e or training leg)")
@@ -58,6 +58,9 @@ def parse_args():
                         "before timing, activations quantised inside the step")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="CPU work budget for the oracle baseline sample")
+    p.add_argument("--no-sweep", action="store_true",
+                   help="skip the maxvio sweep (skew1/skew10/skew20) that follows the large "
+                        "workload")
     args = p.parse_args()
     if args.mxfp8 and (args.shared_experts or args.zero_copy):
         p.error("--mxfp8 runs its own permute-quantise path: it does not combine with "
@@ -590,6 +593,46 @@ def run_ours(args):
         backward = measure_backward(moe, synth, torch, w, inp, dev, args.steps, args.warmup, flush,
                                     peaks0, src0)
 
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_base = (cpu_baseline_mx(w, inp, args.cpu_seconds) if mx
+                    else cpu_baseline(w, inp, args.cpu_seconds))
+
+    # flat in maxvio: the same step on the full-size geometry's skewed routings (maxvio 1, 10
+    # and 20), each workload's inputs made afresh (the previous ones freed first)
+    sweep = None
+    if (w.name == "large" and not (mx or ns or zero_copy) and not args.no_sweep):
+        sweep = {"large": {"ms_per_step": ms_step, "maxvio_measured": maxvio,
+                           "tokens_per_s": job_throughput(w.S, world, ms_step)}}
+        for sname in ("skew1", "skew10", "skew20"):
+            sw = synth.WORKLOADS[sname]
+            inp = None
+            torch.cuda.empty_cache()
+            inp = synth.make_layer_inputs(sw, device=str(dev))
+            ids_step, w_step = inp["topk_ids"], inp["route_w"]
+            for _ in range(args.warmup):
+                flush()
+                step()
+            swevs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                     for _ in range(args.steps)]
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            for i in range(args.steps):
+                flush(i)
+                swevs[i][0].record()
+                step()
+                swevs[i][1].record()
+            torch.cuda.synchronize()
+            if int(buf.d_status.item()) != 0:
+                raise RuntimeError(f"device status {int(buf.d_status.item())} in {sname}")
+            sms = reduce_step_time(sum(e[0].elapsed_time(e[1]) for e in swevs) / args.steps,
+                                   world, dev)
+            sweep[sname] = {"ms_per_step": sms, "maxvio_measured": float(buf.maxvio.item()),
+                            "tokens_per_s": job_throughput(sw.S, world, sms)}
+        t_all = [v["ms_per_step"] for v in sweep.values()]
+        sweep["spread"] = (max(t_all) - min(t_all)) / min(t_all)
+
     if clocks is not None:
         clocks.stop()
 
@@ -657,9 +700,10 @@ def run_ours(args):
         }
         if backward is not None:
             line["training_step"] = backward
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = (cpu_baseline_mx(w, inp, args.cpu_seconds) if mx
-                                    else cpu_baseline(w, inp, args.cpu_seconds))
+        if sweep is not None:
+            line["maxvio_sweep"] = sweep
+        if cpu_base is not None:
+            line["cpu_baseline"] = cpu_base
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -685,6 +729,9 @@ def _oracle_sample(w, S_sample, host):
 
 
 def _host_inputs_from_device(w, inp):
+    """Host copies (numpy bits) of one layer's inputs for the oracle. Expert weights are
+    fetched from the device one expert at a time, when the oracle first asks for them, so
+    that a sample of a few tokens copies only the experts it visits."""
     import numpy as np
     import torch
 
@@ -692,17 +739,47 @@ def _host_inputs_from_device(w, inp):
         return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
     host = {"x": bits(inp["x"]), "topk_ids": inp["topk_ids"].cpu().numpy(),
-            "route_w": inp["route_w"].cpu().numpy()}
+            "route_w": inp["route_w"].cpu().numpy(), "get": None}
     if not w.identity_ffn:
-        wg, wu, wd = bits(inp["w_gate"]), bits(inp["w_up"]), bits(inp["w_down"])
-        host["get"] = lambda e: (wg[e], wu[e], wd[e])
-    else:
-        host["get"] = None
+        cache = {}
+
+        def get(e):
+            if e not in cache:
+                cache[e] = (bits(inp["w_gate"][e]), bits(inp["w_up"][e]), bits(inp["w_down"][e]))
+            return cache[e]
+        host["get"] = get
+    return host
+
+
+def _host_inputs_generated(w):
+    """The same inputs made on the host by the generator (counter-based draws, identical to
+    the device's); an expert's weights are generated when the oracle first asks for them."""
+    import synth
+
+    ids, rw = synth.routing_for(w)
+    host = {"x": synth.normal_bf16_bits(w.seed, synth.TAG_X, w.S * w.H).reshape(w.S, w.H),
+            "topk_ids": ids, "route_w": rw, "get": None}
+    if not w.identity_ffn:
+        cache = {}
+
+        def get(e):
+            if e not in cache:
+                n = w.H * w.Hp
+                cache[e] = tuple(
+                    synth.normal_bf16_bits(w.seed, tag, n, synth.weight_scale(w, which),
+                                           offset=e * n).reshape(shape)
+                    for tag, which, shape in ((synth.TAG_W_GATE, "gate", (w.H, w.Hp)),
+                                              (synth.TAG_W_UP, "up", (w.H, w.Hp)),
+                                              (synth.TAG_W_DOWN, "down", (w.Hp, w.H))))
+            return cache[e]
+        host["get"] = get
     return host
 
 
 def _sample_tokens(w):
-    return {"tiny": 256, "medium": 128}.get(w.name, 16 if not w.identity_ffn else 1024)
+    """Tokens per oracle sample: a few seconds of host work at most per pass (the full-size
+    geometry's two tokens visit 16 experts, 1.4 GB of weights)."""
+    return {"tiny": 256, "medium": 128}.get(w.name, 2 if not w.identity_ffn else 1024)
 
 
 def cpu_baseline(w, inp, budget_s):
@@ -778,8 +855,7 @@ def run_reference(args):
     import synth
 
     w = synth.WORKLOADS[args.workload]
-    inp = synth.make_layer_inputs(w, device="cpu")
-    host = _host_inputs_from_device(w, inp)
+    host = _host_inputs_generated(w)
     mx = args.mxfp8 and not w.identity_ffn
     if mx:
         S_sample = 2

@@ -162,10 +162,27 @@ def moe_permute_workspace_bytes(S: int, K: int, E: int) -> int:
     return int(lib().moe_permute_workspace_bytes(S, K, E))
 
 
-def moe_permute(x, topk_ids, E, x_perm, counts, cu_seqlens, row_id_map, perm_src=None, maxvio=None,
-                max_count=None, workspace=None, d_status=None, stream=None):
-    """Route top-k copies into expert-contiguous order (see include/moe_b200.h)."""
+def _permute_check(x, topk_ids, E, x_perm, counts, cu_seqlens, row_id_map, perm_src, maxvio,
+                   max_count, d_status):
+    """Dtypes, devices and sizes of moe_permute's buffers (the C ABI cannot see sizes, so a
+    short buffer is refused here, before any launch). Returns (S, K, H)."""
+    if topk_ids is None or counts is None or cu_seqlens is None or row_id_map is None:
+        raise ValueError("topk_ids, counts, cu_seqlens and row_id_map are required")
+    if topk_ids.dim() != 2 or (x is not None and x.dim() != 2):
+        raise ValueError("topk_ids must be [S,K] and x [S,H]")
     S, K = topk_ids.shape
+    H = x.shape[1] if x is not None else 0
+    if x is not None and x.shape[0] != S:
+        raise ValueError(f"x: expected {S} rows, got {x.shape[0]}")
+    if x_perm is not None and (x is None or tuple(x_perm.shape) != (S * K, H)):
+        raise ValueError(f"x_perm: expected {(S * K, H)} (and x), got {tuple(x_perm.shape)}")
+    if counts.numel() != E or cu_seqlens.numel() != E + 1 or row_id_map.numel() != S * K:
+        raise ValueError("counts/cu_seqlens/row_id_map sizes do not match (S, K, E)")
+    if perm_src is not None and perm_src.numel() != S * K:
+        raise ValueError("perm_src: expected S*K entries")
+    for t, n in ((maxvio, "maxvio"), (max_count, "max_count"), (d_status, "d_status")):
+        if t is not None and t.numel() < 1:
+            raise ValueError(f"{n}: needs one element")
     dev = topk_ids.device
     _need(topk_ids, "topk_ids", torch.int32, dev, 2)
     _need(x, "x", torch.bfloat16, dev, 2)
@@ -174,13 +191,15 @@ def moe_permute(x, topk_ids, E, x_perm, counts, cu_seqlens, row_id_map, perm_src
                  (perm_src, "perm_src"), (max_count, "max_count"), (d_status, "d_status")):
         _need(t, n, torch.int32, dev)
     _need(maxvio, "maxvio", torch.float64, dev)
-    H = x.shape[1] if x is not None else 0
-    if x_perm is not None and tuple(x_perm.shape) != (S * K, H):
-        raise ValueError(f"x_perm: expected {(S * K, H)}, got {tuple(x_perm.shape)}")
-    if counts.numel() != E or cu_seqlens.numel() != E + 1 or row_id_map.numel() != S * K:
-        raise ValueError("counts/cu_seqlens/row_id_map sizes do not match (S, K, E)")
-    if perm_src is not None and perm_src.numel() != S * K:
-        raise ValueError("perm_src: expected S*K entries")
+    return S, K, H
+
+
+def moe_permute(x, topk_ids, E, x_perm, counts, cu_seqlens, row_id_map, perm_src=None, maxvio=None,
+                max_count=None, workspace=None, d_status=None, stream=None):
+    """Route top-k copies into expert-contiguous order (see include/moe_b200.h)."""
+    S, K, H = _permute_check(x, topk_ids, E, x_perm, counts, cu_seqlens, row_id_map, perm_src,
+                             maxvio, max_count, d_status)
+    dev = topk_ids.device
     need = moe_permute_workspace_bytes(S, K, E)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -200,16 +219,9 @@ def moe_permute_no_alloc(x, topk_ids, E, x_perm, counts, cu_seqlens, row_id_map,
     """moe_permute without a workspace argument, for callers that may not allocate device
     memory: the scratch is a fixed 4 MiB array inside the library (see include/moe_b200.h
     for the size limit and the sharing rules). Allocates nothing."""
-    S, K = topk_ids.shape
+    S, K, H = _permute_check(x, topk_ids, E, x_perm, counts, cu_seqlens, row_id_map, perm_src,
+                             maxvio, max_count, d_status)
     dev = topk_ids.device
-    _need(topk_ids, "topk_ids", torch.int32, dev, 2)
-    _need(x, "x", torch.bfloat16, dev, 2)
-    _need(x_perm, "x_perm", torch.bfloat16, dev, 2)
-    for t, n in ((counts, "counts"), (cu_seqlens, "cu_seqlens"), (row_id_map, "row_id_map"),
-                 (perm_src, "perm_src"), (max_count, "max_count"), (d_status, "d_status")):
-        _need(t, n, torch.int32, dev)
-    _need(maxvio, "maxvio", torch.float64, dev)
-    H = x.shape[1] if x is not None else 0
     st = lib().moe_permute_no_alloc(_ptr(x), _ptr(topk_ids), S, H, K, E, _ptr(x_perm),
                                     _ptr(counts), _ptr(cu_seqlens), _ptr(row_id_map),
                                     _ptr(perm_src), _ptr(maxvio), _ptr(max_count),
@@ -554,24 +566,30 @@ class LayerBuffers:
 
     @staticmethod
     def allocate(S: int, H: int, Hp: int, E: int, K: int, device, with_ffn: bool = True,
-                 train: bool = False):
+                 train: bool = False, alloc=None):
+        """alloc(shape, dtype) -> tensor on `device` (default torch.empty), e.g. an allocator
+        that surrounds each buffer with guard bytes."""
         M = S * K
-        i32 = dict(dtype=torch.int32, device=device)
-        bf = dict(dtype=torch.bfloat16, device=device)
+        new = _allocator(alloc, device)
+        i32, bf = torch.int32, torch.bfloat16
         train = train and with_ffn
+        d_status = new((1,), i32)
+        d_status.zero_()
         return LayerBuffers(
-            x_perm=torch.empty(M, H, **bf), counts=torch.empty(E, **i32),
-            cu_seqlens=torch.empty(E + 1, **i32), row_id_map=torch.empty(M, **i32),
-            perm_src=torch.empty(M, **i32),
-            maxvio=torch.empty(1, dtype=torch.float64, device=device),
-            max_count=torch.empty(1, **i32),
-            workspace=torch.empty(max(moe_permute_workspace_bytes(S, K, E), 16), dtype=torch.uint8,
-                                  device=device),
-            h=torch.empty(M, Hp, **bf) if with_ffn else None,
-            y=torch.empty(M, H, **bf) if with_ffn else None,
-            out=torch.empty(S, H, **bf), d_status=torch.zeros(1, **i32),
-            gate_pre=torch.empty(M, Hp, **bf) if train else None,
-            up_pre=torch.empty(M, Hp, **bf) if train else None)
+            x_perm=new((M, H), bf), counts=new((E,), i32), cu_seqlens=new((E + 1,), i32),
+            row_id_map=new((M,), i32), perm_src=new((M,), i32), maxvio=new((1,), torch.float64),
+            max_count=new((1,), i32),
+            workspace=new((max(moe_permute_workspace_bytes(S, K, E), 16),), torch.uint8),
+            h=new((M, Hp), bf) if with_ffn else None, y=new((M, H), bf) if with_ffn else None,
+            out=new((S, H), bf), d_status=d_status,
+            gate_pre=new((M, Hp), bf) if train else None,
+            up_pre=new((M, Hp), bf) if train else None)
+
+
+def _allocator(alloc, device):
+    if alloc is not None:
+        return alloc
+    return lambda shape, dtype: torch.empty(shape, dtype=dtype, device=device)
 
 
 def moe_layer_forward(x, topk_ids, route_w, w_gate, w_up, w_down, buf: LayerBuffers, stream=None,
@@ -624,16 +642,15 @@ class LayerGrads:
     grad_w_down: torch.Tensor   # [E,H',H] fp32
 
     @staticmethod
-    def allocate(S: int, H: int, Hp: int, E: int, K: int, device):
+    def allocate(S: int, H: int, Hp: int, E: int, K: int, device, alloc=None):
         M = S * K
-        bf = dict(dtype=torch.bfloat16, device=device)
-        f32 = dict(dtype=torch.float32, device=device)
+        new = _allocator(alloc, device)
+        bf, f32 = torch.bfloat16, torch.float32
         return LayerGrads(
-            grad_y=torch.empty(M, H, **bf), d_gate=torch.empty(M, Hp, **bf),
-            d_up=torch.empty(M, Hp, **bf), grad_x_perm=torch.empty(M, H, **bf),
-            grad_x=torch.empty(S, H, **bf), grad_route_w=torch.empty(S, K, **f32),
-            grad_w_gate=torch.empty(E, H, Hp, **f32), grad_w_up=torch.empty(E, H, Hp, **f32),
-            grad_w_down=torch.empty(E, Hp, H, **f32))
+            grad_y=new((M, H), bf), d_gate=new((M, Hp), bf), d_up=new((M, Hp), bf),
+            grad_x_perm=new((M, H), bf), grad_x=new((S, H), bf), grad_route_w=new((S, K), f32),
+            grad_w_gate=new((E, H, Hp), f32), grad_w_up=new((E, H, Hp), f32),
+            grad_w_down=new((E, Hp, H), f32))
 
 
 def moe_layer_backward(grad_out, route_w, w_gate, w_up, w_down, buf: LayerBuffers,
@@ -809,11 +826,12 @@ class MxBuffers:
     h_sf: torch.Tensor
 
     @staticmethod
-    def allocate(S: int, H: int, Hp: int, K: int, device):
+    def allocate(S: int, H: int, Hp: int, K: int, device, alloc=None):
         M = S * K
-        u8 = dict(dtype=torch.uint8, device=device)
-        return MxBuffers(torch.empty(M, H, **u8), torch.empty(M, H // 32, **u8),
-                         torch.empty(M, Hp, **u8), torch.empty(M, Hp // 32, **u8))
+        new = _allocator(alloc, device)
+        u8 = torch.uint8
+        return MxBuffers(new((M, H), u8), new((M, H // 32), u8), new((M, Hp), u8),
+                         new((M, Hp // 32), u8))
 
 
 def moe_layer_forward_mxfp8(x, topk_ids, route_w, mw: MxWeights, buf: LayerBuffers,

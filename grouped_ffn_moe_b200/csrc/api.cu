@@ -1,5 +1,6 @@
 // C ABI entry points (include/moe_b200.h): argument validation, workspace sizing, launch.
 // Nothing here allocates device memory or synchronises the host.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -22,6 +23,70 @@ int num_sms() {
     n = 148;
   if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
   return n;
+}
+
+namespace {
+
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename F>
+F driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<F>(p);
+}
+
+}  // namespace
+
+uint64_t current_context_id() {
+  static const PfnCtxGetCurrent get_current = driver_fn<PfnCtxGetCurrent>("cuCtxGetCurrent");
+  static const PfnCtxGetId get_id = driver_fn<PfnCtxGetId>("cuCtxGetId");
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return static_cast<uint64_t>(id) + 1;  // 0 stays "no context"
+}
+
+bool ContextCache::find(uint64_t ctx, void** value) {
+  if (ctx == 0) return false;
+  std::lock_guard<std::mutex> lock(mu_);
+  for (int i = 0; i < n_; ++i)
+    if (ids_[i] == ctx) {
+      *value = values_[i];
+      return true;
+    }
+  return false;
+}
+
+void ContextCache::put(uint64_t ctx, void* value) {
+  if (ctx == 0) return;
+  std::lock_guard<std::mutex> lock(mu_);
+  for (int i = 0; i < n_; ++i)
+    if (ids_[i] == ctx) {
+      values_[i] = value;
+      return;
+    }
+  if (n_ < kSlots) {
+    ids_[n_] = ctx;
+    values_[n_] = value;
+    ++n_;
+  }
+}
+
+bool set_smem_optin(const void* kernel, int bytes, ContextCache& done) {
+  void* v = nullptr;
+  if (done.find(current_context_id(), &v)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  done.put(current_context_id(), reinterpret_cast<void*>(uintptr_t{1}));  // context exists now
+  return true;
 }
 
 namespace {

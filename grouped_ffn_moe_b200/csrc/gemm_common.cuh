@@ -36,7 +36,7 @@ constexpr uint64_t kDrainBudgetNs = 200000000ull;
 // unit's N rows (a multiple of 16) load as the binary decomposition of N, i.e. at most five
 // boxes and no row beyond the 16-row rounding.
 struct RowMaps {
-  CUtensorMap m[kNumBoxHeights + 1];  // + an 8-row box for the CTA-pair kernel's half tiles
+  CUtensorMap m[kNumBoxHeights];
 };
 
 // A unit of a token-chunked pass: expert e, feature block fb, rows [row0, row0 + nrows).
@@ -124,7 +124,7 @@ __device__ __forceinline__ void unit_starts(const int32_t* cu, int64_t M, int E,
 // a K-major operand tile whose rows are tokens (or weight rows).
 bool make_row_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows,
                   uint32_t box_rows);
-// The six token-row maps (256 ... 8 rows) of one activation matrix.
+// The five token-row maps (256 ... 16 rows) of one activation matrix.
 bool make_row_maps(RowMaps* maps, const void* ptr, uint64_t inner, uint64_t rows);
 // A row-major bf16 matrix [rows][n_feat] viewed as (64 features, rows, n_feat / 64) with a
 // (64 x 64 x blocks) box: an MN-major operand tile of 64 * blocks features x 64 rows, laid

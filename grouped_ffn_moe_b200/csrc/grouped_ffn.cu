@@ -30,10 +30,6 @@
 // bf16(x.W_gate) and bf16(x.W_up) that the backward differentiates SwiGLU at.
 // Every wait is bounded (globaltimer); on expiry the CTA records MOE_ERR_DEVICE_TIMEOUT,
 // drains its own copies and MMAs with bounded waits, frees TMEM and exits.
-#include <atomic>
-#include <cstdlib>
-#include <string>
-
 #include "gemm_common.cuh"
 
 namespace moe {
@@ -52,10 +48,9 @@ namespace {
 //            MoonEP README, "Zero-copy"). Measured alternatives: one TMA tile::gather4 per four
 //            rows (2.9x slower: the per-instruction cost set the pace) and cp.async from the
 //            producer warp alone (2.9x slower: one warp keeps too few copies in flight).
-//   kSingle: A0 = one 128-feature block; two TMEM accumulators double-buffered.
 //   kPair:   A0, A1 = two adjacent 128-feature blocks of one weight tensor sharing the token
 //            tile (half the token-row traffic per feature); y = acc0 | acc1.
-enum Mode : int { kSwiGLU = 0, kSingle = 1, kPair = 2, kSwiGLUGather = 3 };
+enum Mode : int { kSwiGLU = 0, kPair = 2, kSwiGLUGather = 3 };
 
 template <int kMode>
 struct Cfg {
@@ -63,10 +58,10 @@ struct Cfg {
   // gather: four more warps (10-13) copy the token rows
   static constexpr int kGatherWarps = kMode == kSwiGLUGather ? 4 : 0;
   static constexpr int kBlock = kThreads + 32 * kGatherWarps;
-  static constexpr int kNumA = kMode == kSingle ? 1 : 2;
+  static constexpr int kNumA = 2;
   static constexpr int kNMaxMode = kSwi ? MOE_SWIGLU_NMAX : kNMax;
-  // accumulator stages: two when they fit in TMEM (kSingle; kSwiGLU with N <= 128)
-  static constexpr int kAccStages = (kMode == kSingle || kNMaxMode <= 128) ? 2 : 1;
+  // accumulator stages: two when they fit in TMEM (N <= 128 tokens per unit)
+  static constexpr int kAccStages = kNMaxMode <= 128 ? 2 : 1;
   static constexpr int kUpOff = kAccStages == 2 ? kNMaxMode : 256;  // up accumulator column
   static constexpr int kFeatPerUnit = kMode == kPair ? 2 * kBM : kBM;
   static constexpr int kStageBytes = kNumA * kABytes + kNMaxMode * kBK * 2;
@@ -82,7 +77,6 @@ struct Cfg {
 };
 static_assert(Cfg<kSwiGLU>::kSmemBytes <= 232448, "shared memory budget (SwiGLU)");
 static_assert(Cfg<kSwiGLUGather>::kSmemBytes == Cfg<kSwiGLU>::kSmemBytes, "gather layout");
-static_assert(Cfg<kSingle>::kSmemBytes <= 232448, "shared memory budget (single)");
 static_assert(Cfg<kPair>::kSmemBytes <= 232448, "shared memory budget (pair)");
 
 struct FfnArgs {
@@ -108,7 +102,6 @@ __global__ void __launch_bounds__(Cfg<kMode>::kBlock, 1)
                        const __grid_constant__ CUtensorMap tmA1,
                        const __grid_constant__ RowMaps tmB, const FfnArgs args) {
   using C = Cfg<kMode>;
-  constexpr bool kDual = C::kNumA == 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint8_t* s_out = smem + C::kOffOut;
@@ -304,8 +297,7 @@ __global__ void __launch_bounds__(Cfg<kMode>::kBlock, 1)
             const uint64_t bdesc = smem_desc_sw128(b0 + kk * 32, 16, 1024);
             const uint32_t acc = (kt | kk) != 0 ? 1u : 0u;
             umma_f16(d0, smem_desc_sw128(a0 + kk * 2048, kAHalfBytes, 1024), bdesc, idesc, acc);
-            if (kDual)
-              umma_f16(d1, smem_desc_sw128(a1 + kk * 2048, kAHalfBytes, 1024), bdesc, idesc, acc);
+            umma_f16(d1, smem_desc_sw128(a1 + kk * 2048, kAHalfBytes, 1024), bdesc, idesc, acc);
           }
           issued_any = true;
           umma_commit(&empty[stage]);  // frees the smem stage when these MMAs complete
@@ -426,353 +418,13 @@ __global__ void __launch_bounds__(Cfg<kMode>::kBlock, 1)
   }
 }
 
-// ----------------------------------------------------------------------------- CTA-pair SwiGLU
-
-// SwiGLU pass on CTA pairs (clusters of two CTAs on neighbouring SMs, tcgen05 cta_group::2).
-// A pair owns 128 output features of a unit; CTA r (0 or 1) owns features 64r..64r+63. Its
-// 128 A rows are those 64 features of W_gate followed by the same 64 features of W_up, so one
-// M=256 MMA (issued by CTA 0) leaves gate in TMEM lanes 0-63 and up in lanes 64-127 of each
-// CTA: the SiLU(gate)*up epilogue stays inside the CTA. The token tile is split: CTA r loads
-// tokens rN/2 .. rN/2+N/2-1 and the MMA reads both halves. An accumulator takes N <= 256 TMEM
-// columns, so two of them double-buffer the epilogue against the next unit's MMAs, and a
-// pipeline stage is 16 KB of weights + at most 16 KB of tokens, six stages deep.
-#ifndef MOE_PAIR_KBLOCKS
-#define MOE_PAIR_KBLOCKS 2
-#endif
-constexpr int kPairKBlocks = MOE_PAIR_KBLOCKS;     // 64-element k blocks per stage
-constexpr int kPairStages = 6 / kPairKBlocks;
-constexpr int kPairABlockBytes = 2 * kAHalfBytes;  // [gate 64 f | up 64 f] x 64 k
-constexpr int kPairBBlockBytes = 128 * kRowBytes;  // up to 128 token rows (half of N) x 64 k
-constexpr int kPairAStageBytes = kPairKBlocks * kPairABlockBytes;
-constexpr int kPairBStageBytes = kPairKBlocks * kPairBBlockBytes;
-constexpr int kPairStageBytes = kPairAStageBytes + kPairBStageBytes;
-constexpr int kPairXBytes = kOutChunk * 64 * 4;    // up values of a chunk, fp32 [32 tok][64 f]
-constexpr int kPairOBytes = kOutChunk * 64 * 2;    // h of a chunk, bf16 [32 tok][64 f]
-constexpr int kPairOffX = kPairStages * kPairStageBytes;
-constexpr int kPairOffO = kPairOffX + kEpiGroups * kPairXBytes;
-constexpr int kPairOffCu = kPairOffO + kEpiGroups * kPairOBytes;
-constexpr int kPairOffUnits = kPairOffCu + 4 * (MOE_MAX_EXPERTS + 1);
-constexpr int kPairOffBars = (kPairOffUnits + 4 * (MOE_MAX_EXPERTS + 1) + 7) & ~7;
-constexpr int kPairNumBars = 2 * kPairStages + 2 * 2 + 1;
-constexpr int kPairOffMisc = kPairOffBars + 8 * kPairNumBars;
-constexpr int kPairSmemBytes = kPairOffMisc + 64 + 1024;
-static_assert(kPairSmemBytes <= 232448, "shared memory budget (CTA pair)");
-constexpr uint64_t kPairExitDelayNs = 10000000ull;  // after a time-out: let stray copies land
-
-__global__ void __launch_bounds__(kThreads, 1)
-    swiglu_pair_kernel(const __grid_constant__ CUtensorMap tmG,
-                       const __grid_constant__ CUtensorMap tmU,
-                       const __grid_constant__ RowMaps tmB, const FfnArgs args) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align_1024(smem_raw);
-  float* s_x = reinterpret_cast<float*>(smem + kPairOffX);
-  __nv_bfloat16* s_o = reinterpret_cast<__nv_bfloat16*>(smem + kPairOffO);
-  int32_t* s_cu = reinterpret_cast<int32_t*>(smem + kPairOffCu);
-  int32_t* s_ustart = reinterpret_cast<int32_t*>(smem + kPairOffUnits);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPairOffBars);
-  uint64_t* full = bars;                    // used in CTA 0 only
-  uint64_t* empty = bars + kPairStages;     // both CTAs
-  uint64_t* tfull = bars + 2 * kPairStages; // both CTAs
-  uint64_t* tempty = tfull + 2;             // used in CTA 0 only (arrivals from both)
-  uint64_t* drain = tempty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kPairOffMisc);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kPairOffMisc + 4);
-  int32_t* s_scan = reinterpret_cast<int32_t*>(smem + kPairOffMisc + 8);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int cid = static_cast<int>(cluster_id_x());
-  const int ncl = static_cast<int>(num_clusters_x());
-  const int E = args.E;
-  const int nfb = args.n_feat / kBM;
-  const int KT = args.k_dim / kBK;
-
-  if (tid == 0) {
-    for (int s = 0; s < kPairStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&tfull[s], 1);
-      mbar_init(&tempty[s], 2 * kEpiThreads / 32);  // every epilogue warp of both CTAs
-    }
-    mbar_init(drain, 1);
-    *s_abort = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_map(&tmG);
-    tma_prefetch_map(&tmU);
-    for (int i = 0; i < kNumBoxHeights + 1; ++i) tma_prefetch_map(&tmB.m[i]);
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(s_tmem, kTmemCols);
-    tmem_relinquish_pair();
-  }
-  cluster_sync();  // both CTAs' barriers exist before either signals the other
-  griddep_wait();
-  griddep_launch_dependents();
-  unit_starts(args.cu, args.M, E, nfb, 256, s_cu, s_ustart, s_scan);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *s_tmem;
-  const int total_units = s_ustart[E];
-
-  if (warp == 0) {
-    // producers (both CTAs): this CTA's weight half and token half of every stage, counted on
-    // CTA 0's full barrier
-    if (lane == 0) {
-      const uint64_t pol_stream = policy_evict_first();
-      const uint64_t pol_keep = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int u = cid; u < total_units && !*s_abort; u += ncl) {
-        const Unit U = decode_unit(u, s_ustart, s_cu, E);
-        if (U.nrows <= 0) continue;
-        const int n = (U.nrows + 15) & ~15;
-        const int nh = n >> 1;  // token rows per CTA, a multiple of 8
-        const uint64_t pol_w = U.ntc > 1 ? pol_keep : pol_stream;
-        const int fz = U.fb * 2 + static_cast<int>(rank);
-        const int my_row0 = U.row0 + static_cast<int>(rank) * nh;
-        const uint32_t bytes_pair =
-            2u * static_cast<uint32_t>(kPairKBlocks * (kPairABlockBytes + nh * kRowBytes));
-        for (int kt = 0; kt < KT; kt += kPairKBlocks) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, s_abort, args.budget_ns)) break;
-          uint8_t* st = smem + stage * kPairStageBytes;
-          const uint32_t fbar = map_to_cta(smem_u32(&full[stage]), 0);
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], bytes_pair);
-#pragma unroll
-          for (int kb = 0; kb < kPairKBlocks; ++kb) {
-            const int ky = U.e * args.k_dim + (kt + kb) * kBK;
-            uint8_t* sa = st + kb * kPairABlockBytes;
-            tma_load_3d_pair(sa, &tmG, fbar, 0, ky, fz, pol_w);
-            tma_load_3d_pair(sa + kAHalfBytes, &tmU, fbar, 0, ky, fz, pol_w);
-            uint8_t* sb = st + kPairAStageBytes + kb * kPairBBlockBytes;
-            int r = 0;
-#pragma unroll
-            for (int i = 1; i < kNumBoxHeights + 1; ++i) {  // 128, 64, 32, 16, 8 rows
-              const int h = 256 >> i;
-              if (nh & h) {
-                tma_load_2d_pair(sb + r * kRowBytes, &tmB.m[i], fbar, (kt + kb) * kBK,
-                                 my_row0 + r, pol_keep);
-                r += h;
-              }
-            }
-          }
-          if (++stage == kPairStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // MMA issuer: CTA 0 only
-    if (lane == 0 && rank == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int astage = 0;
-      uint32_t aphase = 0;
-      bool issued_any = false;
-      for (int u = cid; u < total_units && !*s_abort; u += ncl) {
-        const Unit U = decode_unit(u, s_ustart, s_cu, E);
-        if (U.nrows <= 0) continue;
-        const uint32_t n = static_cast<uint32_t>((U.nrows + 15) & ~15);
-        const uint32_t idesc = idesc_bf16_amn_bk(256, n);
-        if (!mbar_wait_bounded(&tempty[astage], aphase ^ 1u, s_abort, args.budget_ns)) break;
-        tc_fence_after();
-        const uint32_t d = tmem_base + astage * kAccCols;
-        bool ok = true;
-        for (int kt = 0; kt < KT; kt += kPairKBlocks) {
-          if (!mbar_wait_bounded(&full[stage], phase, s_abort, args.budget_ns)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * kPairStageBytes);
-          const uint32_t b0 = a0 + kPairAStageBytes;
-#pragma unroll
-          for (int kb = 0; kb < kPairKBlocks; ++kb)
-#pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)
-              umma_f16_pair(d,
-                            smem_desc_sw128(a0 + kb * kPairABlockBytes + kk * 2048, kAHalfBytes,
-                                            1024),
-                            smem_desc_sw128(b0 + kb * kPairBBlockBytes + kk * 32, 16, 1024),
-                            idesc, (kt | kb | kk) != 0 ? 1u : 0u);
-          issued_any = true;
-          umma_commit_pair(&empty[stage]);  // frees the stage in both CTAs
-          if (++stage == kPairStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-        umma_commit_pair(&tfull[astage]);  // accumulator ready in both CTAs
-        if (++astage == 2) {
-          astage = 0;
-          aphase ^= 1u;
-        }
-      }
-      if (*s_abort && issued_any) {
-        umma_commit_pair(drain);
-        volatile int dummy = 0;
-        mbar_wait_bounded(drain, 0, &dummy, kDrainBudgetNs);
-      }
-    }
-  } else if (warp >= 2) {
-    // epilogue: warps 2..9, two groups of four alternating 32-token chunks; in each group the
-    // warps on TMEM lanes 64-127 (up) hand their values to the warps on lanes 0-63 (gate)
-    const int q = warp & 3;
-    const int grp = (warp - 2) >> 2;
-    const int gt = (tid - 64) & 127;
-    const uint32_t bar_grp = 1 + grp, bar_all = 3;
-    float* xs = s_x + grp * (kPairXBytes / 4);
-    __nv_bfloat16* os = s_o + grp * (kPairOBytes / 2);
-    const uint32_t tempty_leader0 = map_to_cta(smem_u32(&tempty[0]), 0);
-    int astage = 0;
-    uint32_t aphase = 0;
-    for (int u = cid; u < total_units; u += ncl) {
-      const Unit U = decode_unit(u, s_ustart, s_cu, E);
-      if (U.nrows <= 0) continue;
-      mbar_wait_bounded(&tfull[astage], aphase, s_abort, args.budget_ns);
-      // every epilogue warp takes the same decision
-      if (named_bar_red_or(bar_all, kEpiThreads, *s_abort != 0)) break;
-      tc_fence_after();
-      const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + astage * kAccCols;
-      const int f0 = U.fb * kBM + static_cast<int>(rank) * 64;
-      for (int c = grp * kOutChunk; c < U.nrows; c += kEpiGroups * kOutChunk) {
-        __syncwarp();
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tbase + c, r);
-        tmem_ld_wait();
-        if (q >= 2) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) xs[j * 64 + (q - 2) * 32 + lane] = __uint_as_float(r[j]);
-        }
-        named_bar_sync(bar_grp, 128);
-        if (q < 2) {
-          const int f = q * 32 + lane;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float g = __uint_as_float(r[j]);
-            const float hval = __fdividef(g, 1.0f + __expf(-g)) * xs[j * 64 + f];
-            os[j * 64 + f] = __float2bfloat16_rn(hval);
-          }
-        }
-        named_bar_sync(bar_grp, 128);
-#pragma unroll
-        for (int p = 0; p < (kOutChunk * 64 * 2 / 16) / 128; ++p) {
-          const int vid = gt + 128 * p;
-          const int j = vid >> 3, c8 = vid & 7;
-          if (c + j < U.nrows) {
-            const uint4 val = *reinterpret_cast<const uint4*>(os + j * 64 + c8 * 8);
-            __nv_bfloat16* dst =
-                args.out + static_cast<int64_t>(U.row0 + c + j) * args.n_feat + f0 + c8 * 8;
-            *reinterpret_cast<uint4*>(dst) = val;
-          }
-        }
-        named_bar_sync(bar_grp, 128);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty_leader0 + astage * 8);
-      if (++astage == 2) {
-        astage = 0;
-        aphase ^= 1u;
-      }
-    }
-  }
-
-  __syncthreads();
-  if (*s_abort) {
-    if (tid == 0 && args.d_status != nullptr) atomicOr(args.d_status, MOE_ERR_DEVICE_TIMEOUT);
-    const uint64_t t0 = global_timer_ns();  // bounded: copies signalled to the other CTA
-    while (global_timer_ns() - t0 < kPairExitDelayNs) {
-    }
-  }
-  cluster_sync();  // CTA 0's MMAs read this CTA's shared memory and write its TMEM
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc_pair(tmem_base, kTmemCols);
-  }
-}
-
 // ----------------------------------------------------------------------------- host side
 
 template <int kMode>
 bool ensure_smem_attr() {
-  static std::atomic<int> done_dev_mask{0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  const int bit = 1 << (dev & 31);
-  if (done_dev_mask.load() & bit) return true;
-  if (cudaFuncSetAttribute(grouped_ffn_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Cfg<kMode>::kSmemBytes) != cudaSuccess)
-    return false;
-  done_dev_mask.fetch_or(bit);
-  return true;
-}
-
-// SwiGLU kernel: "single" (one CTA per unit, default) or "pair" (CTA pairs), from
-// MOE_SWIGLU_KERNEL; both give identical results. On B200 the pair kernel is measured slower
-// at these token counts (N <= 192 per unit leaves too little MMA work per stage to hide the
-// pair's cross-SM signalling), so it is opt-in.
-bool use_pair_swiglu() {
-  static const bool pair = [] {
-    const char* s = std::getenv("MOE_SWIGLU_KERNEL");
-    return s != nullptr && std::string(s) == "pair";
-  }();
-  return pair;
-}
-
-cudaError_t launch_swiglu_pair(const CUtensorMap& g, const CUtensorMap& u, const RowMaps& b,
-                               const FfnArgs& args, cudaStream_t stream) {
-  static std::atomic<int> done_dev_mask{0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidValue;
-  const int bit = 1 << (dev & 31);
-  if (!(done_dev_mask.load() & bit)) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        swiglu_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes);
-    if (e != cudaSuccess) return e;
-    done_dev_mask.fetch_or(bit);
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kPairSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, swiglu_pair_kernel, g, u, b, args);
-  if (err != cudaSuccess) {
-    (void)cudaGetLastError();
-    cfg.numAttrs = 1;  // without the dependent-launch attribute
-    err = cudaLaunchKernelEx(&cfg, swiglu_pair_kernel, g, u, b, args);
-  }
-  return err;
-}
-
-// Down-projection kernel: "pair" (two 128-feature blocks per unit, default) or "single",
-// from MOE_DOWN_KERNEL; both give identical results.
-int down_mode() {
-  static int mode = [] {
-    const char* s = std::getenv("MOE_DOWN_KERNEL");
-    return (s != nullptr && std::string(s) == "single") ? static_cast<int>(kSingle)
-                                                        : static_cast<int>(kPair);
-  }();
-  return mode;
+  static ContextCache done;
+  return set_smem_optin(reinterpret_cast<const void*>(grouped_ffn_kernel<kMode>),
+                        Cfg<kMode>::kSmemBytes, done);
 }
 
 }  // namespace
@@ -809,11 +461,8 @@ moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const voi
   if (dual) {
     CUtensorMap m_wg, m_wu;
     RowMaps m_x;
-    // the CTA-pair kernel does not store pre-activations: training uses the one-CTA kernel
-    const bool pair = use_pair_swiglu() && gate_pre == nullptr;
-    const uint32_t halves = pair ? 1 : 2;
-    if (!make_weight_map(&m_wg, w0, Hp, static_cast<uint64_t>(E) * H, halves) ||
-        !make_weight_map(&m_wu, w1, Hp, static_cast<uint64_t>(E) * H, halves) ||
+    if (!make_weight_map(&m_wg, w0, Hp, static_cast<uint64_t>(E) * H) ||
+        !make_weight_map(&m_wu, w1, Hp, static_cast<uint64_t>(E) * H) ||
         !make_row_maps(&m_x, act, H, M) || !ensure_smem_attr<kSwiGLU>())
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
@@ -821,27 +470,21 @@ moe_status launch_ffn_pass(bool dual, const void* act, const void* w0, const voi
                     static_cast<__nv_bfloat16*>(gate_pre), static_cast<__nv_bfloat16*>(up_pre),
                     nullptr, 1, nullptr, 0};
     const cudaError_t err =
-        pair
-            ? launch_swiglu_pair(m_wg, m_wu, m_x, a, stream)
-            : launch_dependent(grouped_ffn_kernel<kSwiGLU>, dim3(grid), dim3(kThreads),
-                               Cfg<kSwiGLU>::kSmemBytes, stream, m_wg, m_wu, m_x, a);
+        launch_dependent(grouped_ffn_kernel<kSwiGLU>, dim3(grid), dim3(kThreads),
+                         Cfg<kSwiGLU>::kSmemBytes, stream, m_wg, m_wu, m_x, a);
     if (err != cudaSuccess) return MOE_ERR_CUDA;
   } else {
     CUtensorMap m_wd;
     RowMaps m_h;
-    const bool pair = down_mode() == kPair;
     if (!make_weight_map(&m_wd, w0, H, static_cast<uint64_t>(E) * Hp) ||
-        !make_row_maps(&m_h, act, Hp, M) ||
-        !(pair ? ensure_smem_attr<kPair>() : ensure_smem_attr<kSingle>()))
+        !make_row_maps(&m_h, act, Hp, M) || !ensure_smem_attr<kPair>())
       return MOE_ERR_CUDA;
     const FfnArgs a{cu_seqlens, static_cast<__nv_bfloat16*>(out), d_status, M, E,
                     static_cast<int32_t>(Hp), static_cast<int32_t>(H), wait_budget_ns(),
                     nullptr, nullptr, nullptr, 1, nullptr, 0};
-    const cudaError_t err =
-        pair ? launch_dependent(grouped_ffn_kernel<kPair>, dim3(grid), dim3(kThreads),
-                                Cfg<kPair>::kSmemBytes, stream, m_wd, m_wd, m_h, a)
-             : launch_dependent(grouped_ffn_kernel<kSingle>, dim3(grid), dim3(kThreads),
-                                Cfg<kSingle>::kSmemBytes, stream, m_wd, m_wd, m_h, a);
+    const cudaError_t err = launch_dependent(grouped_ffn_kernel<kPair>, dim3(grid),
+                                             dim3(kThreads), Cfg<kPair>::kSmemBytes, stream,
+                                             m_wd, m_wd, m_h, a);
     if (err != cudaSuccess) return MOE_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

@@ -31,9 +31,6 @@
 // accumulator stages of 256 TMEM columns let the epilogue of one unit overlap the next unit's
 // MMAs. Every wait is bounded (globaltimer) and a time-out leaves MOE_ERR_DEVICE_TIMEOUT in
 // d_status after the CTA has drained its own copies and MMAs.
-#include <atomic>
-#include <cstdlib>
-#include <string>
 
 #include "gemm_common.cuh"
 
@@ -679,312 +676,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// ----------------------------------------------------------------------------- CTA pairs
-
-// Weight gradients on CTA pairs (clusters of two CTAs on neighbouring SMs, tcgen05
-// cta_group::2): a unit is a 256 x 256 gradient tile; CTA r holds gradient rows
-// 128r .. 128r+127 (its X-feature slice, the A operand) and loads half of the unit's D
-// columns (the B operand); CTA 0 issues one M = 256 MMA that reads both CTAs' tiles, and each
-// CTA's TMEM receives its 128 rows x all 256 columns, so two accumulator stages still fit.
-// Per SM a stage is 32 KB for the same MMA work as the one-CTA kernel's 48 KB: a third less
-// operand feed from L2, and six stages in flight.
-//
-// Stage protocol: each CTA's TMA lands on its own `full` barrier; its warp 1 waits for it,
-// zeroes the rows past the expert's end in its own tile when this is the expert's last
-// block, fences generic->async and arrives on CTA 0's `ready` barrier (two arrivals); CTA 0's
-// MMA thread waits on `ready`, issues the MMAs and commits to `empty` in both CTAs. Epilogue
-// warps of both CTAs arrive on CTA 0's `tempty`.
-constexpr int kWPSliceBytes = kAHalfBytes;            // 64 features x 64 tokens
-constexpr int kWPStageBytes = 4 * kWPSliceBytes;      // A: 2 slices, B: 2 slices
-constexpr int kWPStages = 6;
-constexpr int kWPOffEpi = kWPStages * kWPStageBytes;
-constexpr int kWPOffBars = kWPOffEpi + (kEpiThreads / 32) * kWEpiTileBytes;
-constexpr int kWPNumBars = 3 * kWPStages + 2 * 2 + 1;
-constexpr int kWPOffMisc = kWPOffBars + 8 * kWPNumBars;
-constexpr int kWPSmemBytes = kWPOffMisc + 64 + 1024;
-static_assert(kWPSmemBytes <= 232448, "shared memory budget (weight gradients, CTA pairs)");
-constexpr uint64_t kWPExitDelayNs = 10000000ull;  // after a time-out: let stray copies land
-
-__global__ void __launch_bounds__(kThreads, 1)
-    wgrad_pair_kernel(const __grid_constant__ WgradMaps maps,
-                      const __grid_constant__ WgradArgs args) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align_1024(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWPOffBars);
-  uint64_t* full = bars;                      // this CTA's TMA for the stage landed
-  uint64_t* ready = bars + kWPStages;         // CTA 0: both CTAs' tiles ready (2 arrivals)
-  uint64_t* empty = bars + 2 * kWPStages;     // both CTAs: MMAs done with the stage
-  uint64_t* tfull = bars + 3 * kWPStages;     // both CTAs
-  uint64_t* tempty = tfull + 2;               // CTA 0: epilogue warps of both CTAs
-  uint64_t* drain = tempty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kWPOffMisc);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kWPOffMisc + 4);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int cid = static_cast<int>(cluster_id_x());
-  const int ncl = static_cast<int>(num_clusters_x());
-  const int total_units = args.pstart[kWProblems];
-
-  if (tid == 0) {
-    for (int s = 0; s < kWPStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&ready[s], 2);
-      mbar_init(&empty[s], 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&tfull[s], 1);
-      mbar_init(&tempty[s], 2 * kEpiThreads / 32);
-    }
-    mbar_init(drain, 1);
-    *s_abort = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    for (int p = 0; p < kWProblems; ++p) {
-      tma_prefetch_map(&maps.x[p]);
-      tma_prefetch_map(&maps.d[p]);
-      tma_prefetch_map(&maps.out[p]);
-    }
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(s_tmem, kTmemCols);
-    tmem_relinquish_pair();
-  }
-  cluster_sync();  // both CTAs' barriers exist before either signals the other
-  griddep_wait();
-  griddep_launch_dependents();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *s_tmem;
-
-  if (warp == 0) {
-    // TMA producer of this CTA's half: its 128 X features and its N/2 D features
-    if (lane == 0) {
-      const uint64_t pol_keep = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued_mask = 0, issued_phase = 0;
-      for (int u = cid; u < total_units && !*s_abort; u += ncl) {
-        const WUnit W = decode_wunit(u, args);
-        int r0, T;
-        expert_span_global(args, W.e, r0, T);
-        const int nkb = (T + kWKB - 1) / kWKB;
-        const int n = min(kWN, args.p[W.p].fd - W.nb * kWN);
-        const int xz = W.mb * 4 + static_cast<int>(rank) * 2;
-        const int dz = (W.nb * kWN + static_cast<int>(rank) * (n >> 1)) / 64;
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, s_abort, args.budget_ns)) break;
-          uint8_t* st = smem + stage * kWPStageBytes;
-          mbar_arrive_expect_tx(&full[stage], kWPStageBytes);
-          tma_load_3d_hint(st, &maps.x[W.p], &full[stage], 0, r0 + kb * kWKB, xz, pol_keep);
-          tma_load_3d_hint(st + 2 * kWPSliceBytes, &maps.d[W.p], &full[stage], 0,
-                           r0 + kb * kWKB, dz, pol_keep);
-          issued_mask |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == kWPStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      if (*s_abort) {
-        volatile int dummy = 0;
-        for (int s = 0; s < kWPStages; ++s)
-          if (issued_mask & (1u << s))
-            mbar_wait_bounded(&full[s], (issued_phase >> s) & 1u, &dummy, kDrainBudgetNs);
-      }
-    }
-  } else if (warp == 1) {
-    // Whole warp in both CTAs: forward this CTA's landed tile to CTA 0's `ready` (after
-    // zeroing the rows past the expert's end); in CTA 0, lane 0 then issues the pair MMAs.
-    const uint32_t ready0 = map_to_cta(smem_u32(&ready[0]), 0);
-    int stage = 0;
-    uint32_t phase = 0;
-    int astage = 0;
-    uint32_t aphase = 0;
-    bool issued_any = false;
-    for (int u = cid; u < total_units; u += ncl) {
-      if (__shfl_sync(0xffffffffu, *s_abort, 0)) break;  // lane 0's view: a uniform exit
-      const WUnit W = decode_wunit(u, args);
-      int r0, T;
-      expert_span_global(args, W.e, r0, T);
-      if (T <= 0) continue;
-      const int nkb = (T + kWKB - 1) / kWKB;
-      const uint32_t n = static_cast<uint32_t>(min(kWN, args.p[W.p].fd - W.nb * kWN));
-      const uint32_t idesc = idesc_bf16(256, n, 1, 1);
-      int ok = 1;
-      if (rank == 0 && lane == 0)
-        ok = mbar_wait_bounded(&tempty[astage], aphase ^ 1u, s_abort, args.budget_ns);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      const uint32_t d = tmem_base + astage * kAccCols;
-      for (int kb = 0; kb < nkb; ++kb) {
-        if (lane == 0) ok = mbar_wait_bounded(&full[stage], phase, s_abort, args.budget_ns);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        uint8_t* st = smem + stage * kWPStageBytes;
-        const int valid = min(kWKB, T - kb * kWKB);
-        const int kcut = (valid + 15) & ~15;
-        if (valid < kcut) {
-          // rows valid .. kcut-1 of this CTA's four slices belong to the next expert (or lie
-          // past the end of the matrix): zero them (whole 128-byte rows)
-          const int rows = kcut - valid;
-          for (int i = lane; i < 4 * rows * 8; i += 32) {
-            const int slice = i / (rows * 8);
-            const int rem = i - slice * rows * 8;
-            const int row = valid + rem / 8, v16 = rem & 7;
-            *reinterpret_cast<uint4*>(st + slice * kWPSliceBytes + row * 128 + v16 * 16) =
-                make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(ready0 + stage * 8);
-        if (rank == 0) {
-          if (lane == 0) ok = mbar_wait_bounded(&ready[stage], phase, s_abort, args.budget_ns);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) break;
-          if (lane == 0) {
-            tc_fence_after();
-            const uint32_t a0 = smem_u32(st);
-            const uint32_t b0 = a0 + 2 * kWPSliceBytes;
-            for (int kk = 0; kk < kcut / 16; ++kk)
-              umma_f16_pair(d, smem_desc_sw128(a0 + kk * 2048, kWPSliceBytes, 1024),
-                            smem_desc_sw128(b0 + kk * 2048, kWPSliceBytes, 1024), idesc,
-                            (kb | kk) != 0 ? 1u : 0u);
-            umma_commit_pair(&empty[stage]);  // frees the stage in both CTAs
-          }
-          issued_any = true;
-        }
-        __syncwarp();
-        if (++stage == kWPStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-      if (!ok) break;
-      if (rank == 0 && lane == 0) umma_commit_pair(&tfull[astage]);
-      __syncwarp();
-      if (++astage == 2) {
-        astage = 0;
-        aphase ^= 1u;
-      }
-    }
-    if (rank == 0 && lane == 0 && *s_abort && issued_any) {
-      umma_commit_pair(drain);
-      volatile int dummy = 0;
-      mbar_wait_bounded(drain, 0, &dummy, kDrainBudgetNs);
-    }
-    __syncwarp();
-  } else {
-    // Epilogue (both CTAs): this CTA's 128 gradient rows of the tile, TMEM -> registers ->
-    // swizzled shared tile -> TMA store (reduce-add when accumulating), as the one-CTA kernel.
-    const int q = warp & 3;
-    const int grp = (warp - 2) >> 2;
-    const uint32_t bar_all = 3;
-    const uint32_t tempty0 = map_to_cta(smem_u32(&tempty[0]), 0);
-    uint8_t* tile = smem + kWPOffEpi + (warp - 2) * kWEpiTileBytes;
-    int astage = 0;
-    uint32_t aphase = 0;
-    for (int u = cid; u < total_units; u += ncl) {
-      const WUnit W = decode_wunit(u, args);
-      const WgradProblem& P = args.p[W.p];
-      int r0_unused, T;
-      expert_span_global(args, W.e, r0_unused, T);
-      const int ncols = min(kWN, P.fd - W.nb * kWN);
-      const int lrow = W.mb * 256 + static_cast<int>(rank) * kBM + q * 32;  // row in expert
-      const bool rows_ok = lrow < P.fx;  // past fx (odd number of 128-row blocks): no rows
-      const int row0 = W.e * P.fx + lrow;
-      if (T <= 0) {
-        if (!args.accumulate && rows_ok) {
-          float* dst_row = P.out + static_cast<int64_t>(row0 + lane) * P.fd + W.nb * kWN;
-          for (int c = grp * kOutChunk; c < ncols; c += kEpiGroups * kOutChunk)
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              *reinterpret_cast<float4*>(dst_row + c + 4 * v) = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        continue;
-      }
-      mbar_wait_bounded(&tfull[astage], aphase, s_abort, args.budget_ns);
-      if (named_bar_red_or(bar_all, kEpiThreads, *s_abort != 0)) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + astage * kAccCols;
-      for (int c = grp * kOutChunk; c < ncols; c += kEpiGroups * kOutChunk) {
-        __syncwarp();
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tbase + c, r);
-        if (lane == 0) bulk_wait_group_read<0>();  // the tile's previous store has read it
-        __syncwarp();
-        tmem_ld_wait();
-#pragma unroll
-        for (int v = 0; v < 8; ++v)
-          *reinterpret_cast<uint4*>(tile + lane * 128 + ((v ^ (lane & 7)) * 16)) =
-              make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && rows_ok) {
-          const int x = W.nb * kWN + c;
-          if (args.accumulate)
-            tma_reduce_add_2d(&maps.out[W.p], tile, x, row0);
-          else
-            tma_store_2d(&maps.out[W.p], tile, x, row0);
-          bulk_commit_group();
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty0 + astage * 8);
-      if (++astage == 2) {
-        astage = 0;
-        aphase ^= 1u;
-      }
-    }
-    if (lane == 0) bulk_wait_group<0>();
-    __syncwarp();
-  }
-
-  __syncthreads();
-  if (*s_abort) {
-    if (tid == 0 && args.d_status != nullptr) atomicOr(args.d_status, MOE_ERR_DEVICE_TIMEOUT);
-    const uint64_t t0 = global_timer_ns();  // bounded: copies signalled to the other CTA
-    while (global_timer_ns() - t0 < kWPExitDelayNs) {
-    }
-  }
-  cluster_sync();  // CTA 0's MMAs read this CTA's shared memory and write its TMEM
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc_pair(tmem_base, kTmemCols);
-  }
-}
-
 // ----------------------------------------------------------------------------- host side
 
 template <typename Kernel>
-bool ensure_smem(Kernel kernel, int bytes, std::atomic<int>& done_dev_mask) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  const int bit = 1 << (dev & 31);
-  if (done_dev_mask.load() & bit) return true;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-      cudaSuccess)
-    return false;
-  done_dev_mask.fetch_or(bit);
-  return true;
+bool ensure_smem(Kernel kernel, int bytes, ContextCache& done) {
+  return set_smem_optin(reinterpret_cast<const void*>(kernel), bytes, done);
 }
 
-std::atomic<int> g_smem_down{0}, g_smem_upgate{0}, g_smem_wgrad{0}, g_smem_wgrad_pair{0};
-
-// Weight-gradient kernel: "single" (one CTA per 128 x 256 tile, default) or "pair" (CTA pairs
-// on 256 x 256 tiles), from MOE_WGRAD_KERNEL; both give identical results.
-bool use_pair_wgrad() {
-  static const bool pair = [] {
-    const char* s = std::getenv("MOE_WGRAD_KERNEL");
-    return s != nullptr && std::string(s) == "pair";
-  }();
-  return pair;
-}
+ContextCache g_smem_down, g_smem_upgate, g_smem_wgrad;
 
 }  // namespace
 
@@ -1053,7 +752,6 @@ moe_status launch_ffn_weight_grad(const void* x_perm, const void* h, const void*
                                   float* grad_w_up, float* grad_w_down, bool accumulate,
                                   int32_t* d_status, cudaStream_t stream) {
   WgradMaps maps;
-  const bool pair = use_pair_wgrad();
   // problem 0: x^T d_gate, 1: x^T d_up ([H, H']), 2: h^T grad_y ([H', H])
   const void* xs[kWProblems] = {x_perm, x_perm, h};
   const void* ds[kWProblems] = {d_gate, d_up, grad_y};
@@ -1070,8 +768,7 @@ moe_status launch_ffn_weight_grad(const void* x_perm, const void* h, const void*
   int64_t units = 0;
   for (int p = 0; p < kWProblems; ++p) {
     WgradProblem& P = a.p[p];
-    // pair: each CTA loads half of a unit's (up to) 256 D columns, two 64-feature slices
-    P.dblocks = pair ? 2 : static_cast<int32_t>(fds[p] / 64 < 4 ? fds[p] / 64 : 4);
+    P.dblocks = static_cast<int32_t>(fds[p] / 64 < 4 ? fds[p] / 64 : 4);
     if (!make_weight_map(&maps.x[p], xs[p], fxs[p], M, 2) ||
         !make_weight_map(&maps.d[p], ds[p], fds[p], M, static_cast<uint32_t>(P.dblocks)) ||
         !make_f32_tile_map(&maps.out[p], outs[p], fds[p], static_cast<uint64_t>(E) * fxs[p], 32,
@@ -1080,38 +777,13 @@ moe_status launch_ffn_weight_grad(const void* x_perm, const void* h, const void*
     P.out = outs[p];
     P.fx = static_cast<int32_t>(fxs[p]);
     P.fd = static_cast<int32_t>(fds[p]);
-    P.mbs = static_cast<int32_t>(pair ? ceil_div(fxs[p], 2 * kBM) : fxs[p] / kBM);
+    P.mbs = static_cast<int32_t>(fxs[p] / kBM);
     P.nbs = static_cast<int32_t>(ceil_div(fds[p], kWN));
     a.pstart[p] = static_cast<int32_t>(units);
     units += static_cast<int64_t>(E) * P.mbs * P.nbs;
   }
   if (units > INT32_MAX) return MOE_ERR_UNSUPPORTED_SHAPE;
   a.pstart[kWProblems] = static_cast<int32_t>(units);
-  if (pair) {
-    if (!ensure_smem(wgrad_pair_kernel, kWPSmemBytes, g_smem_wgrad_pair)) return MOE_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kWPSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    cudaError_t err = cudaLaunchKernelEx(&cfg, wgrad_pair_kernel, maps, a);
-    if (err != cudaSuccess) {
-      (void)cudaGetLastError();
-      cfg.numAttrs = 1;  // without the dependent-launch attribute
-      err = cudaLaunchKernelEx(&cfg, wgrad_pair_kernel, maps, a);
-    }
-    if (err != cudaSuccess) return MOE_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-  }
   if (!ensure_smem(wgrad_kernel, kWSmemBytes, g_smem_wgrad)) return MOE_ERR_CUDA;
   const cudaError_t err = launch_dependent(wgrad_kernel, dim3(num_sms()), dim3(kThreads),
                                            kWSmemBytes, stream, maps, a);

@@ -597,16 +597,9 @@ __global__ void __launch_bounds__(256) mx_permute_quantize_kernel(
 // The kernel's dynamic shared-memory opt-in, once per device.
 template <bool kSwi>
 bool ensure_mx_smem_attr() {
-  static std::atomic<int> done_dev_mask{0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  const int bit = 1 << (dev & 31);
-  if (done_dev_mask.load() & bit) return true;
-  if (cudaFuncSetAttribute(grouped_ffn_mx_kernel<kSwi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           MxCfg<kSwi>::kSmemBytes) != cudaSuccess)
-    return false;
-  done_dev_mask.fetch_or(bit);
-  return true;
+  static ContextCache done;
+  return set_smem_optin(reinterpret_cast<const void*>(grouped_ffn_mx_kernel<kSwi>),
+                        MxCfg<kSwi>::kSmemBytes, done);
 }
 
 bool make_mx_row_maps(MxRowMaps* maps, const void* ptr, uint64_t inner, uint64_t rows) {

@@ -2,6 +2,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 #include <utility>
 
 #include <cuda_runtime.h>
@@ -28,6 +29,32 @@ inline int64_t permute_num_chunks(int64_t F) { return ceil_div(F, permute_chunk_
 
 // Number of SMs of the current device (cached per device).
 int num_sms();
+
+// Process-unique id of the CUDA context current on the calling thread, 0 when there is none
+// yet (the runtime creates the primary context lazily, at the first call that needs it).
+// Kernel attributes and device-symbol addresses belong to one context: a second context on
+// the same device, or the primary context re-created after cudaDeviceReset, gets a new id
+// even where the driver reuses the old handle value.
+uint64_t current_context_id();
+
+// A small thread-safe map from context id to a pointer-sized value: what a one-time set-up
+// produced in that context. Ids that do not fit (more than kSlots contexts) are not cached,
+// so their set-up simply runs again on every call.
+class ContextCache {
+ public:
+  static constexpr int kSlots = 64;
+  bool find(uint64_t ctx, void** value);
+  void put(uint64_t ctx, void* value);
+
+ private:
+  std::mutex mu_;
+  uint64_t ids_[kSlots] = {};
+  void* values_[kSlots] = {};
+  int n_ = 0;
+};
+
+// Sets `kernel`'s dynamic shared-memory limit to `bytes`, once per context (cached in `done`).
+bool set_smem_optin(const void* kernel, int bytes, ContextCache& done);
 
 // Launch `kernel` as a programmatic dependent launch: it may be scheduled while the previous
 // kernel in the stream finishes, and waits for it (griddepcontrol.wait) before touching data

@@ -21,7 +21,6 @@
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>
-#include <mutex>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -538,23 +537,22 @@ static __device__ __align__(256) int32_t g_permute_scratch[MOE_NO_ALLOC_SCRATCH_
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+ContextCache g_scratch_addr;
 
-// Device address of g_permute_scratch on the current device. The host-side name is only a
-// stand-in, so the address is looked up once per device (with that device current) and kept.
+// Device address of g_permute_scratch in the current CUDA context. The host-side name is
+// only a stand-in, so the address is looked up (with the device current) the first time a
+// context calls, and kept per context: another context on the same device, or the primary
+// context re-created after cudaDeviceReset, gets its own lookup.
 moe_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr)
-      return MOE_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+  void* p = nullptr;
+  if (g_scratch_addr.find(current_context_id(), &p)) {
+    *out = p;
+    return MOE_OK;
   }
-  *out = g_scratch_addr[dev];
+  if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr)
+    return MOE_ERR_CUDA;
+  g_scratch_addr.put(current_context_id(), p);  // the lookup made the context current
+  *out = p;
   return MOE_OK;
 }
 

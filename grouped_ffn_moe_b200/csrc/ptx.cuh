@@ -288,25 +288,11 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Named barrier over `nthreads` threads; threads of a warp may arrive diverged.
-// ----------------------------------------------------------------------------- CTA pairs
-// (a cluster of two CTAs working as one tcgen05 pair: cta_group::2)
+// ----------------------------------------------------------------------------- clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t cluster_id_x() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t num_clusters_x() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
   return r;
 }
 
@@ -317,7 +303,8 @@ __device__ __forceinline__ uint32_t map_to_cta(uint32_t smem_addr, uint32_t rank
   return r;
 }
 
-// All threads of both CTAs of the cluster.
+// All threads of all CTAs of the cluster: shared-memory writes before it are visible to
+// every CTA's reads after it.
 __device__ __forceinline__ void cluster_sync() {
   asm volatile(
       "barrier.cluster.arrive.release.aligned;\n\t"
@@ -325,80 +312,14 @@ __device__ __forceinline__ void cluster_sync() {
           : "memory");
 }
 
-// Arrive on an mbarrier given by its cluster address (possibly in the other CTA).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
+// 32-bit load from the shared memory of a CTA of this cluster (address from map_to_cta).
+__device__ __forceinline__ int32_t ld_shared_cluster(uint32_t cluster_addr) {
+  int32_t v;
+  asm volatile("ld.shared::cluster.b32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
 }
 
-// Tiled TMA loads of a CTA pair: data land in this CTA's shared memory, completion bytes
-// are counted on `bar_cluster_addr`, which may be the other CTA's barrier (no multicast).
-__device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* map,
-                                                 uint32_t bar_cluster_addr, int32_t x, int32_t y,
-                                                 int32_t z, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y), "r"(z),
-      "l"(policy)
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map,
-                                                 uint32_t bar_cluster_addr, int32_t x, int32_t y,
-                                                 uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y), "l"(policy)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(dst)),
-               "r"(ncols)
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
-// D (+)= A * B over the CTA pair: A rows 0-127 and B columns 0..N/2-1 come from CTA 0's
-// shared memory, A rows 128-255 and columns N/2..N-1 from CTA 1's, at the same addresses;
-// D rows 0-127 land in CTA 0's TMEM, rows 128-255 in CTA 1's. Issued by CTA 0 only.
-__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                              uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive once on the barrier at this shared offset in both CTAs of the pair when all
-// previously issued pair MMAs complete.
-__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .b16 m;\n\t"
-      "mov.b16 m, 3;\n\t"
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], m;\n\t}\n" ::"r"(smem_u32(bar))
-      : "memory");
-}
-
-// Instruction descriptor (kind::f16, bf16 x bf16 -> f32, A MN-major, B K-major) for M rows.
-__device__ __forceinline__ uint32_t idesc_bf16_amn_bk(uint32_t m, uint32_t n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((n >> 3) << 17) | ((m >> 4) << 24);
-}
-
+// Named barrier over `nthreads` threads; threads of a warp may arrive diverged.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

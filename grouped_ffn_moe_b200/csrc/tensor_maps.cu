@@ -37,7 +37,7 @@ bool make_row_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows
 }
 
 bool make_row_maps(RowMaps* maps, const void* ptr, uint64_t inner, uint64_t rows) {
-  for (int i = 0; i < kNumBoxHeights + 1; ++i)
+  for (int i = 0; i < kNumBoxHeights; ++i)
     if (!make_row_map(&maps->m[i], ptr, inner, rows, static_cast<uint32_t>(kNMax >> i)))
       return false;
   return true;

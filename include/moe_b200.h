@@ -121,8 +121,10 @@ moe_status moe_permute(const void* x, const int32_t* topk_ids, int64_t S, int64_
  *     (4 MiB: e.g. S*K up to 524288 routed slots with E up to 1024); larger problems return
  *     MOE_ERR_UNSUPPORTED_SHAPE and launch nothing. Use moe_permute with a workspace then.
  *   - Every GPU that loads the library holds this array until the process exits.
- *   - The first call on a device looks up the array's device address (once per device, with
- *     that device current) and keeps it; make that first call before any stream capture.
+ *   - The first call in each CUDA context looks up the array's device address (with the
+ *     device current) and keeps it for that context; a second context on the device, or the
+ *     primary context re-created after cudaDeviceReset, does its own lookup on its first
+ *     call. Make that first call before any stream capture.
  *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *   - All calls on a device share the one array, and it keeps the last call's contents.
  *     Nothing in it has to start at zero (each call writes every entry it reads), but calls

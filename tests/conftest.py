@@ -20,3 +20,20 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.fail("this test needs a CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(autouse=True)
+def _guard_bands(request):
+    """For GPU tests: output buffers allocated through helpers.GUARD sit between sentinel
+    guard bands; after the test every guard byte must be unchanged."""
+    if request.node.get_closest_marker("gpu") is None:
+        yield
+        return
+    from helpers import GUARD
+
+    GUARD.reset()
+    yield
+    try:
+        GUARD.check()
+    finally:
+        GUARD.reset()

@@ -83,3 +83,68 @@ def assert_close_fp32_sums(got, ref, abs_sum, n_terms: int, what: str = "", adde
     nr = np.linalg.norm(r)
     return {"rel_fro": float(np.linalg.norm(g - r) / max(nr, 1e-30)),
             "max_err_over_bound": float((err / np.maximum(bound, 1e-38)).max()) if err.size else 0.0}
+
+
+# ----------------------------------------------------------------------------- guard bands
+#
+# An out-of-bounds check for the GPU tests in place of a memory sanitizer: every output buffer
+# is carved out of a larger allocation with GUARD_BYTES of a sentinel byte before and after
+# it. A kernel that stores past either end of its buffer (a ragged tail, a wrong row) changes
+# a guard byte, and the check after the test finds it.
+
+GUARD_BYTES = 64 << 10
+GUARD_SENTINEL = 0xA5
+
+
+class GuardedAllocator:
+    def __init__(self):
+        self.regions = []
+
+    def reset(self):
+        self.regions = []
+
+    def __call__(self, shape, dtype, device=None, fill_byte=0xFF):
+        """A tensor of `shape` and `dtype` inside guard bands; its own bytes are `fill_byte`
+        (0xFF: NaN for floating types, -1 for integers) so that unwritten outputs show."""
+        device = device if device is not None else torch.device("cuda:0")
+        shape = tuple(int(d) for d in shape)
+        n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        tail = GUARD_BYTES + ((-n) % 256)
+        raw = torch.empty(GUARD_BYTES + n + tail, dtype=torch.uint8, device=device)
+        raw[:GUARD_BYTES].fill_(GUARD_SENTINEL)
+        raw[GUARD_BYTES + n:].fill_(GUARD_SENTINEL)
+        inner = raw[GUARD_BYTES:GUARD_BYTES + n]
+        inner.fill_(fill_byte)
+        self.regions.append((raw, n))
+        return inner.view(dtype).view(shape)
+
+    def full(self, shape, value, dtype, device=None):
+        t = self(shape, dtype, device)
+        t.fill_(value)
+        return t
+
+    def zeros(self, shape, dtype, device=None):
+        return self(shape, dtype, device, fill_byte=0)
+
+    def for_device(self, device):
+        """The allocator as LayerBuffers / LayerGrads / MxBuffers.allocate take it."""
+        return lambda shape, dtype: self(shape, dtype, device)
+
+    def check(self):
+        """Every guard byte still holds the sentinel (synchronises first)."""
+        if not self.regions:
+            return
+        torch.cuda.synchronize()
+        bad = []
+        for i, (raw, n) in enumerate(self.regions):
+            head = raw[:GUARD_BYTES]
+            tail = raw[GUARD_BYTES + n:]
+            nh = int((head != GUARD_SENTINEL).sum().item())
+            nt = int((tail != GUARD_SENTINEL).sum().item())
+            if nh or nt:
+                bad.append(f"buffer {i} ({n} bytes): {nh} guard bytes changed before it, "
+                           f"{nt} after it")
+        assert not bad, "out-of-bounds writes: " + "; ".join(bad)
+
+
+GUARD = GuardedAllocator()

@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import grouped_ffn_moe_b200 as moe
 
@@ -173,3 +174,30 @@ def test_host_validation_of_mxfp8_calls():
                                    null) == 1
     assert L.moe_grouped_ffn_mxfp8(a, a, a, a, a, a, a, a, a, 64, 256, 256, 0, a, a, a, null,
                                    null) == 1
+
+
+@pytest.mark.parametrize("fn", ["moe_permute", "moe_permute_no_alloc"])
+def test_permute_wrappers_refuse_short_buffers_before_any_launch(fn):
+    """The C ABI cannot see buffer sizes: the Python wrappers of both permutation entry points
+    refuse a buffer of the wrong size with ValueError (here on CPU tensors, so nothing could
+    launch even if the check were missing)."""
+    S, K, E, H = 16, 2, 4, 8
+    i32 = dict(dtype=torch.int32)
+    ok = dict(x=torch.zeros(S, H, dtype=torch.bfloat16), topk_ids=torch.zeros(S, K, **i32),
+              x_perm=torch.zeros(S * K, H, dtype=torch.bfloat16), counts=torch.zeros(E, **i32),
+              cu_seqlens=torch.zeros(E + 1, **i32), row_id_map=torch.zeros(S * K, **i32),
+              perm_src=torch.zeros(S * K, **i32))
+    call = getattr(moe, fn)
+    bad = {"x_perm": torch.zeros(S * K - 1, H, dtype=torch.bfloat16),
+           "counts": torch.zeros(E - 1, **i32), "cu_seqlens": torch.zeros(E, **i32),
+           "row_id_map": torch.zeros(S * K - 1, **i32), "perm_src": torch.zeros(S, **i32),
+           "x": torch.zeros(S + 1, H, dtype=torch.bfloat16)}
+    for name, t in bad.items():
+        args = dict(ok, **{name: t})
+        with pytest.raises(ValueError, match=r"expected|sizes|rows"):
+            call(args["x"], args["topk_ids"], E, args["x_perm"], args["counts"],
+                 args["cu_seqlens"], args["row_id_map"], args["perm_src"])
+    # right sizes: refused only because these are not CUDA tensors
+    with pytest.raises(ValueError, match="CUDA"):
+        call(ok["x"], ok["topk_ids"], E, ok["x_perm"], ok["counts"], ok["cu_seqlens"],
+             ok["row_id_map"], ok["perm_src"])

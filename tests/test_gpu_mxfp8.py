@@ -21,7 +21,7 @@ import torch
 
 import grouped_ffn_moe_b200 as moe
 import synth
-from helpers import assert_close_bf16, bits
+from helpers import GUARD, assert_close_bf16, bits
 from oracle import moe_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -122,12 +122,12 @@ def test_mx_permute_quantize_bit_exact(cuda_device, S, H, K, E):
     ids_np, _ = synth.route_es(7, S, K, E)
     ids = torch.from_numpy(ids_np.reshape(S, K)).to(dev)
     M = S * K
-    i32 = dict(dtype=torch.int32, device=dev)
-    counts, cu = torch.empty(E, **i32), torch.empty(E + 1, **i32)
-    rmap, psrc = torch.empty(M, **i32), torch.empty(M, **i32)
+    i32 = torch.int32
+    counts, cu = GUARD((E,), i32, dev), GUARD((E + 1,), i32, dev)
+    rmap, psrc = GUARD((M,), i32, dev), GUARD((M,), i32, dev)
     moe.moe_permute(to_dev(x, dev), ids, E, None, counts, cu, rmap, psrc)
-    x_q = torch.full((M, H), 0xEE, dtype=torch.uint8, device=dev)
-    x_sf = torch.full((M, H // 32), 0xEE, dtype=torch.uint8, device=dev)
+    x_q = GUARD.full((M, H), 0xEE, torch.uint8, dev)
+    x_sf = GUARD.full((M, H // 32), 0xEE, torch.uint8, dev)
     moe.moe_mx_permute_quantize(to_dev(x, dev), rmap, K, x_q, x_sf)
     torch.cuda.synchronize()
     _, _, rmap_ref, psrc_ref = O.permute_metadata(ids_np.reshape(S, K), E)
@@ -158,15 +158,15 @@ def test_mx_grouped_ffn_parity(cuda_device, case):
     x[min(3, M - 1), 32:64] = 0
     wg, wu, wd = make_weights(13, E, H, Hp)
     mw = moe.MxWeights.from_bf16(to_dev(wg, dev), to_dev(wu, dev), to_dev(wd, dev))
-    u8 = dict(dtype=torch.uint8, device=dev)
-    x_q, x_sf = torch.empty(M, H, **u8), torch.empty(M, H // 32, **u8)
+    u8 = torch.uint8
+    x_q, x_sf = GUARD((M, H), u8, dev), GUARD((M, H // 32), u8, dev)
     ident = torch.arange(M, dtype=torch.int32, device=dev)
     moe.moe_mx_permute_quantize(to_dev(x, dev), ident, 1, x_q, x_sf)
     cu = torch.from_numpy(cu_np).to(dev)
-    h_q = torch.full((M, Hp), 0xEE, **u8)
-    h_sf = torch.full((M, Hp // 32), 0xEE, **u8)
-    y = torch.full((M, H), float("nan"), dtype=torch.bfloat16, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    h_q = GUARD.full((M, Hp), 0xEE, u8, dev)
+    h_sf = GUARD.full((M, Hp // 32), 0xEE, u8, dev)
+    y = GUARD.full((M, H), float("nan"), torch.bfloat16, dev)
+    status = GUARD.zeros((1,), torch.int32, dev)
     moe.moe_grouped_ffn_mxfp8(x_q, x_sf, mw, cu, h_q, h_sf, y, status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
@@ -203,8 +203,8 @@ def test_mx_layer_end_to_end(cuda_device):
     rw = synth.route_weights(17, S, K)
     wg, wu, wd = make_weights(19, E, H, Hp)
     mw = moe.MxWeights.from_bf16(to_dev(wg, dev), to_dev(wu, dev), to_dev(wd, dev))
-    buf = moe.LayerBuffers.allocate(S, H, Hp, E, K, dev)
-    mxbuf = moe.MxBuffers.allocate(S, H, Hp, K, dev)
+    buf = moe.LayerBuffers.allocate(S, H, Hp, E, K, dev, alloc=GUARD.for_device(dev))
+    mxbuf = moe.MxBuffers.allocate(S, H, Hp, K, dev, alloc=GUARD.for_device(dev))
     ids = torch.from_numpy(ids_np).to(dev)
     route_w = torch.from_numpy(np.asarray(rw, np.float32).reshape(S, K)).to(dev)
     out = moe.moe_layer_forward_mxfp8(to_dev(x, dev), ids, route_w, mw, buf, mxbuf)

@@ -15,7 +15,7 @@ import torch
 
 import grouped_ffn_moe_b200 as moe
 import synth
-from helpers import assert_close_bf16, bf16_ulp, bits, f64
+from helpers import GUARD, assert_close_bf16, bf16_ulp, bits, f64
 from oracle import moe_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -29,13 +29,13 @@ def gpu_permute(x, ids, E, with_rows=True):
     dev = ids.device
     H = x.shape[1]
     M = S * K
-    i32 = dict(dtype=torch.int32, device=dev)
+    i32 = torch.int32
     r = dict(
-        x_perm=torch.full((M, H), float("nan"), dtype=torch.bfloat16, device=dev) if with_rows else None,
-        counts=torch.full((E,), -7, **i32), cu=torch.full((E + 1,), -7, **i32),
-        rmap=torch.full((M,), -7, **i32), psrc=torch.full((M,), -7, **i32),
-        maxvio=torch.full((1,), -7.0, dtype=torch.float64, device=dev),
-        max_count=torch.full((1,), -7, **i32), status=torch.zeros(1, **i32))
+        x_perm=GUARD.full((M, H), float("nan"), torch.bfloat16, dev) if with_rows else None,
+        counts=GUARD.full((E,), -7, i32, dev), cu=GUARD.full((E + 1,), -7, i32, dev),
+        rmap=GUARD.full((M,), -7, i32, dev), psrc=GUARD.full((M,), -7, i32, dev),
+        maxvio=GUARD.full((1,), -7.0, torch.float64, dev),
+        max_count=GUARD.full((1,), -7, i32, dev), status=GUARD.zeros((1,), i32, dev))
     moe.moe_permute(x, ids, E, r["x_perm"], r["counts"], r["cu"], r["rmap"], r["psrc"], r["maxvio"],
                     r["max_count"], d_status=r["status"])
     torch.cuda.synchronize()
@@ -78,7 +78,8 @@ def weights_getter(inp):
 
 
 def run_layer(inp, w, dev):
-    buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev, with_ffn=not w.identity_ffn)
+    buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev, with_ffn=not w.identity_ffn,
+                                    alloc=GUARD.for_device(dev))
     moe.moe_layer_forward(inp["x"], inp["topk_ids"], inp["route_w"], inp.get("w_gate"),
                           inp.get("w_up"), inp.get("w_down"), buf)
     torch.cuda.synchronize()
@@ -174,8 +175,8 @@ def test_bad_routing_is_flagged(cuda_device):
 
 def test_maxvio_entry_point(cuda_device):
     counts = torch.tensor([3584] + [161] * 383, dtype=torch.int32, device=cuda_device)
-    mv = torch.zeros(1, dtype=torch.float64, device=cuda_device)
-    mc = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    mv = GUARD((1,), torch.float64, cuda_device)
+    mc = GUARD((1,), torch.int32, cuda_device)
     moe.moe_maxvio(counts, 8192, 8, mv, mc)
     torch.cuda.synchronize()
     assert mc.item() == 3584
@@ -184,17 +185,51 @@ def test_maxvio_entry_point(cuda_device):
 
 # ----------------------------------------------------------------------------- combine
 
-@pytest.mark.parametrize("wname", ["permute_combine_S1024_mv0", "permute_combine_S4096_mv20"])
+IDENTITY_FULL = ["permute_combine_S1024_mv0", "permute_combine_S1024_mv1",
+                 "permute_combine_S4096_mv1", "permute_combine_S4096_mv20",
+                 "permute_combine_S16384_mv1"]
+IDENTITY_SAMPLED = ["permute_combine_S65536_mv0", "permute_combine_S65536_mv1",
+                    "permute_combine_S65536_mv20"]
+
+
+@pytest.mark.parametrize("wname", IDENTITY_FULL + IDENTITY_SAMPLED)
 def test_identity_expert_layer(cuda_device, wname):
+    """The permute/combine workloads (identity experts, H = 7168, E = 384, K = 8) against the
+    oracle's layer: metadata and maxvio exact; x_perm exact and out within the bar, in full
+    up to S = 16384 (the oracle's combine taken 1024 tokens at a time) and on 2048 sampled
+    tokens (with their K rows each) at S = 65536."""
     w = synth.WORKLOADS[wname]
     inp = layer_inputs(w, cuda_device)
     buf = run_layer(inp, w, cuda_device)
-    ref = O.moe_layer(bits(inp["x"]), inp["topk_ids"].cpu().numpy(), inp["route_w"].cpu().numpy(),
-                      w.E, None, 0, identity_ffn=True)
-    assert np.array_equal(buf.cu_seqlens.cpu().numpy(), ref["cu_seqlens"])
-    assert np.array_equal(buf.row_id_map.cpu().numpy(), ref["row_id_map"])
-    assert buf.maxvio.item() == ref["maxvio"]
-    assert_close_bf16(bits(buf.out), ref["out"], "out")
+    ids_np = inp["topk_ids"].cpu().numpy()
+    counts, cu, rmap, psrc = check_permute_exact(
+        dict(counts=buf.counts, cu=buf.cu_seqlens, rmap=buf.row_id_map, psrc=buf.perm_src,
+             maxvio=buf.maxvio, max_count=buf.max_count, status=buf.d_status, x_perm=None),
+        ids_np, w.E)
+    x_bits = bits(inp["x"])
+    rw = inp["route_w"].cpu().numpy()
+    S, K = w.S, w.K
+    if wname in IDENTITY_FULL:
+        x_perm_ref = O.permute_rows(x_bits, psrc, K)
+        assert np.array_equal(bits(buf.x_perm), x_perm_ref)
+        out_gpu = bits(buf.out)
+        out_ref = np.zeros_like(out_gpu)
+        for t0 in range(0, S, 1024):
+            t1 = min(S, t0 + 1024)
+            ys = x_perm_ref[rmap[t0 * K:t1 * K]]  # y = x_perm: the token's K rows, slot order
+            out_ref[t0:t1] = O.unpermute_combine(ys, np.arange((t1 - t0) * K), rw[t0:t1],
+                                                 t1 - t0, K)
+        print(f"[{wname}] out: {assert_close_bf16(out_gpu, out_ref, 'out')}")
+    else:
+        rng = np.random.default_rng(7)
+        toks = np.sort(rng.choice(S, 2048, replace=False))
+        rows = rmap.reshape(S, K)[toks].reshape(-1)
+        xp = bits(buf.x_perm[torch.as_tensor(rows, device=cuda_device)])
+        assert np.array_equal(xp, x_bits[psrc[rows] // K])
+        out_ref = np.stack([O.combine_token(x_bits[psrc[rmap[t * K:(t + 1) * K]] // K], rw[t])
+                            for t in toks])
+        out_gpu = bits(buf.out[torch.as_tensor(toks, device=cuda_device)])
+        print(f"[{wname}] out (sampled): {assert_close_bf16(out_gpu, out_ref, 'out (sampled)')}")
 
 
 def test_combine_unit_weight_invariants(cuda_device):
@@ -204,14 +239,16 @@ def test_combine_unit_weight_invariants(cuda_device):
     ids = ids.to(cuda_device)
     x = synth.normal_bf16_into(torch.empty(S, H, dtype=torch.bfloat16, device=cuda_device), 3,
                                synth.TAG_X)
-    buf = moe.LayerBuffers.allocate(S, H, 0, E, K, cuda_device, with_ffn=False)
+    buf = moe.LayerBuffers.allocate(S, H, 0, E, K, cuda_device, with_ffn=False,
+                                    alloc=GUARD.for_device(cuda_device))
     ones = torch.ones(S, K, dtype=torch.float32, device=cuda_device)
     moe.moe_layer_forward(x, ids, ones, None, None, None, buf)
     torch.cuda.synchronize()
     # unpermute o permute with identity experts and unit weights: exactly bf16(K * x)
     assert torch.equal(buf.out, (x.float() * K).to(torch.bfloat16))
     # K = 1, weight 1: exactly x
-    buf1 = moe.LayerBuffers.allocate(S, H, 0, E, 1, cuda_device, with_ffn=False)
+    buf1 = moe.LayerBuffers.allocate(S, H, 0, E, 1, cuda_device, with_ffn=False,
+                                     alloc=GUARD.for_device(cuda_device))
     moe.moe_layer_forward(x, ids[:, :1].contiguous(), ones[:, :1].contiguous(), None, None, None, buf1)
     torch.cuda.synchronize()
     assert torch.equal(buf1.out, x)
@@ -297,10 +334,11 @@ def _sampled_rows(cu, hot, rng, per=6):
     return np.array(rows, dtype=np.int64)
 
 
-@pytest.mark.parametrize("wname", ["large", "skew20", "skew20_last"])
+@pytest.mark.parametrize("wname", ["large", "skew1", "skew10", "skew20", "skew20_last"])
 def test_layer_full_size_sampled(cuda_device, wname):
-    """Full-size layers on sampled rows; skew20_last puts the hot expert (maxvio 20) last, so
-    its units come at the end of the persistent schedule."""
+    """Full-size layers (S = 8192, H = 7168, H' = 2048, E = 384, K = 8) on sampled rows, at
+    maxvio 0.2 (large), 1, 10 and 20; skew20_last puts the hot expert (maxvio 20) last, so its
+    units come at the end of the persistent schedule."""
     w = synth.WORKLOADS[wname]
     inp = layer_inputs(w, cuda_device)
     buf = run_layer(inp, w, cuda_device)
@@ -360,33 +398,6 @@ def test_generator_twin_matches_host(cuda_device):
                                    synth.TAG_W_GATE, 0.125, offset=off)
         host = synth.normal_bf16_bits(2, synth.TAG_W_GATE, n, 0.125, offset=off)
         assert (bits(t) != host).sum() <= 2
-
-
-def test_down_kernel_variants_agree(cuda_device, tmp_path):
-    """The two down-projection kernels ("pair", default, and "single") give bit-identical y:
-    both accumulate every output in the same order. The variant is chosen per process."""
-    import subprocess
-    import sys
-
-    script = (
-        "import sys, torch, synth, grouped_ffn_moe_b200 as moe\n"
-        "w = synth.WORKLOADS['medium']\n"
-        "inp = synth.make_layer_inputs(w, device='cuda:0')\n"
-        "buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, torch.device('cuda:0'))\n"
-        "moe.moe_layer_forward(inp['x'], inp['topk_ids'], inp['route_w'], inp['w_gate'],"
-        " inp['w_up'], inp['w_down'], buf)\n"
-        "torch.cuda.synchronize()\n"
-        "assert int(buf.d_status.item()) == 0\n"
-        "torch.save(buf.y.cpu(), sys.argv[1])\n")
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    outs = {}
-    for mode in ("pair", "single"):
-        env = dict(os.environ, MOE_DOWN_KERNEL=mode, PYTHONPATH=root)
-        path = str(tmp_path / f"y_{mode}.pt")
-        subprocess.run([sys.executable, "-c", script, path], check=True, env=env, cwd=root,
-                       timeout=600)
-        outs[mode] = torch.load(path)
-    assert torch.equal(outs["pair"], outs["single"])
 
 
 @pytest.mark.parametrize("wname", ["permute_combine_S4096_mv20", "permute_combine_S16384_mv1",
@@ -456,36 +467,6 @@ def test_device_wait_timeout_reports_status_and_keeps_context(cuda_device, tmp_p
     assert int(buf.d_status.item()) == 0
 
 
-def test_swiglu_kernel_variants_agree(cuda_device, tmp_path):
-    """The one-CTA SwiGLU kernel (default) and the CTA-pair kernel (MOE_SWIGLU_KERNEL=pair,
-    tcgen05 cta_group::2) give bit-identical h (and therefore y and out)."""
-    import subprocess
-    import sys
-
-    script = (
-        "import sys, torch, synth, grouped_ffn_moe_b200 as moe\n"
-        "w = synth.WORKLOADS[sys.argv[2]]\n"
-        "inp = synth.make_layer_inputs(w, device='cuda:0')\n"
-        "buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, torch.device('cuda:0'))\n"
-        "moe.moe_layer_forward(inp['x'], inp['topk_ids'], inp['route_w'], inp['w_gate'],"
-        " inp['w_up'], inp['w_down'], buf)\n"
-        "torch.cuda.synchronize()\n"
-        "assert int(buf.d_status.item()) == 0\n"
-        "torch.save({k: getattr(buf, k).cpu() for k in ('h', 'y', 'out')}, sys.argv[1])\n")
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    for wl in ("tiny", "medium"):
-        outs = {}
-        for mode in ("pair", "single"):
-            env = dict(os.environ, MOE_SWIGLU_KERNEL=mode, PYTHONPATH=root)
-            path = str(tmp_path / f"s_{wl}_{mode}.pt")
-            subprocess.run([sys.executable, "-c", script, path, wl], check=True, env=env,
-                           cwd=root, timeout=600)
-            outs[mode] = torch.load(path)
-        for k in outs["pair"]:
-            assert torch.equal(outs["pair"][k].view(torch.int16),
-                               outs["single"][k].view(torch.int16)), (wl, k)
-
-
 # ----------------------------------------------------------------------------- backward
 
 @pytest.mark.parametrize("wname,sample", [("medium", None), ("permute_combine_S65536_mv20", 4096)])
@@ -502,9 +483,9 @@ def test_combine_and_permute_backward(cuda_device, wname, sample):
                                w.seed, synth.TAG_GRAD)
     gxp = synth.normal_bf16_into(torch.empty(M, w.H, dtype=torch.bfloat16, device=cuda_device),
                                  w.seed + 100, synth.TAG_GRAD)
-    grad_y = torch.empty(M, w.H, dtype=torch.bfloat16, device=cuda_device)
-    grad_w = torch.empty(w.S, w.K, dtype=torch.float32, device=cuda_device)
-    grad_x = torch.empty(w.S, w.H, dtype=torch.bfloat16, device=cuda_device)
+    grad_y = GUARD((M, w.H), torch.bfloat16, cuda_device)
+    grad_w = GUARD((w.S, w.K), torch.float32, cuda_device)
+    grad_x = GUARD((w.S, w.H), torch.bfloat16, cuda_device)
     moe.moe_combine_backward(g, y, buf.row_id_map, inp["route_w"], grad_y, grad_w)
     moe.moe_permute_backward(gxp, buf.row_id_map, grad_x, w.K)
     torch.cuda.synchronize()
@@ -549,12 +530,13 @@ def test_backward_unit_weight_and_adjoint_exactness(cuda_device):
     ids = ids.to(cuda_device)
     x = synth.normal_bf16_into(torch.empty(S, H, dtype=torch.bfloat16, device=cuda_device), 4,
                                synth.TAG_X)
-    buf = moe.LayerBuffers.allocate(S, H, 0, E, K, cuda_device, with_ffn=False)
+    buf = moe.LayerBuffers.allocate(S, H, 0, E, K, cuda_device, with_ffn=False,
+                                    alloc=GUARD.for_device(cuda_device))
     ones = torch.ones(S, K, dtype=torch.float32, device=cuda_device)
     moe.moe_layer_forward(x, ids, ones, None, None, None, buf)
-    grad_y = torch.empty(S * K, H, dtype=torch.bfloat16, device=cuda_device)
+    grad_y = GUARD((S * K, H), torch.bfloat16, cuda_device)
     moe.moe_combine_backward(x, None, buf.row_id_map, ones, grad_y)
-    grad_x = torch.empty(S, H, dtype=torch.bfloat16, device=cuda_device)
+    grad_x = GUARD((S, H), torch.bfloat16, cuda_device)
     moe.moe_permute_backward(buf.x_perm, buf.row_id_map, grad_x, K)
     torch.cuda.synchronize()
     assert torch.equal(grad_y, buf.x_perm)  # w = 1: the backward re-dispatch is the permutation
@@ -564,10 +546,10 @@ def test_backward_unit_weight_and_adjoint_exactness(cuda_device):
 # ----------------------------------------------------------------------------- zero copy
 
 def _gather_vs_copy(inp, w, dev):
-    ref = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev)
+    ref = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev, alloc=GUARD.for_device(dev))
     moe.moe_layer_forward(inp["x"], inp["topk_ids"], inp["route_w"], inp["w_gate"], inp["w_up"],
                           inp["w_down"], ref)
-    zc = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev)
+    zc = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev, alloc=GUARD.for_device(dev))
     zc.x_perm.fill_(float("nan"))  # the zero-copy path must not read x_perm
     moe.moe_layer_forward(inp["x"], inp["topk_ids"], inp["route_w"], inp["w_gate"], inp["w_up"],
                           inp["w_down"], zc, zero_copy=True)
@@ -581,8 +563,8 @@ def _gather_vs_copy(inp, w, dev):
 
 @pytest.mark.parametrize("wname", ["tiny", "medium", "large", "skew20"])
 def test_zero_copy_gather_equals_copy_path(cuda_device, wname):
-    """The SwiGLU pass gathering its token rows from x through perm_src (TMA tile::gather4)
-    gives h, y and out bit-identical to the path through x_perm, which is itself checked
+    """The SwiGLU pass gathering its token rows from x through perm_src (16-byte cp.async
+    copies by four gather warps) gives h, y and out bit-identical to the path through x_perm, which is itself checked
     against the oracle above; the tiny layer is also checked against the oracle directly."""
     w = synth.WORKLOADS[wname]
     inp = layer_inputs(w, cuda_device)
@@ -622,11 +604,13 @@ def test_zero_copy_gather_training_preactivations(cuda_device):
     """The gather pass stores the same pre-activations as the training forward on x_perm."""
     w = synth.WORKLOADS["medium"]
     inp = layer_inputs(w, cuda_device)
-    buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, cuda_device, train=True)
+    buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, cuda_device, train=True,
+                                    alloc=GUARD.for_device(cuda_device))
     moe.moe_layer_forward(inp["x"], inp["topk_ids"], inp["route_w"], inp["w_gate"], inp["w_up"],
                           inp["w_down"], buf)
-    h2 = torch.empty_like(buf.h)
-    g2, u2 = torch.empty_like(buf.gate_pre), torch.empty_like(buf.up_pre)
+    h2 = GUARD(buf.h.shape, buf.h.dtype, cuda_device)
+    g2 = GUARD(buf.gate_pre.shape, buf.gate_pre.dtype, cuda_device)
+    u2 = GUARD(buf.up_pre.shape, buf.up_pre.dtype, cuda_device)
     moe.moe_grouped_ffn_up_gate_gather(inp["x"], buf.perm_src, w.K, inp["w_gate"], inp["w_up"],
                                        buf.cu_seqlens, h2, g2, u2, buf.d_status)
     torch.cuda.synchronize()
@@ -648,13 +632,13 @@ def test_shared_expert_layer(cuda_device, wname, n_shared):
     inp = synth.make_layer_inputs(w, device=str(dev), n_shared=n_shared)
     S, K, E = w.S, w.K, w.E
     K2, E2 = K + n_shared, E + n_shared
-    ids2 = torch.empty(S, K2, dtype=torch.int32, device=dev)
-    w2 = torch.empty(S, K2, dtype=torch.float32, device=dev)
+    ids2 = GUARD((S, K2), torch.int32, dev)
+    w2 = GUARD((S, K2), torch.float32, dev)
     moe.moe_append_shared(inp["topk_ids"], inp["route_w"], E, n_shared, ids2, w2)
-    buf = moe.LayerBuffers.allocate(S, w.H, w.Hp, E2, K2, dev)
+    buf = moe.LayerBuffers.allocate(S, w.H, w.Hp, E2, K2, dev, alloc=GUARD.for_device(dev))
     moe.moe_layer_forward(inp["x"], ids2, w2, inp["w_gate"], inp["w_up"], inp["w_down"], buf)
-    mv = torch.empty(1, dtype=torch.float64, device=dev)
-    mc = torch.empty(1, dtype=torch.int32, device=dev)
+    mv = GUARD((1,), torch.float64, dev)
+    mc = GUARD((1,), torch.int32, dev)
     moe.moe_maxvio(buf.counts[:E], S, K, mv, mc)
     torch.cuda.synchronize()
     assert int(buf.d_status.item()) == 0

@@ -659,3 +659,76 @@ def test_mxfp8_expert_ffn_close_to_bf16_expert():
     r = O.bf16_bits_to_f64(y_bf16)
     rel = np.linalg.norm(O.bf16_bits_to_f64(y_mx) - r) / np.linalg.norm(r)
     assert 1e-2 < rel < 0.2, rel
+    # the band alone would also pass an expert that skips the quantisation of h or of x;
+    # on these inputs both variants give outputs that differ from the oracle's
+    xq = O.mx_dequantize(*O.mx_quantize(O.bf16_bits_to_f64(x)))
+    wgd, wud, wdd = (O.mx_dequantize(*O.mx_weights(w), axis=-2) for w in (wg, wu, wd))
+    y_no_h = O.f64_to_bf16_bits((O.silu(xq @ wgd) * (xq @ wud)) @ wdd)
+    xr = O.bf16_bits_to_f64(x)
+    h_no_x = O.mx_dequantize(*O.mx_quantize(O.silu(xr @ wgd) * (xr @ wud)))
+    y_no_x = O.f64_to_bf16_bits(h_no_x @ wdd)
+    for variant in (y_no_h, y_no_x):
+        assert (variant != y_mx).mean() > 0.5
+
+
+def test_mxfp8_expert_exact_hand_case():
+    """One token, H = H' = 32 (one MXFP8 block per row and column), every value worked out by
+    hand. Each quantisation step of the MXFP8 expert changes at least one output, so dropping
+    any of them (x, the up/gate weights, h, the down weights) or quantising a weight along the
+    wrong axis fails this pin.
+
+    x = [2, 1.0625, 0, ...]: amax 2 gives scale 2^(1-8); x*128 = [256, 136] and 136 is a tie
+    in the [128, 256) binade (step 16), so x dequantises to [2, 1].
+    W_gate[0, :] = 64 (on the grid) gives g = 128 for every feature, where
+    1 + e^-128 == 1 in float64, so silu(g) = g exactly and h_j = 128 * u_j.
+    W_up rows 0 and 1 hold (a_j, b_j), on the grid of their column's block except a_9 = 1.0625
+    (amax 1.0625, scale 2^-8: 272 is a tie, kept 256, so a_9 becomes 1.0); u_j = 2 a_j + b_j.
+    h = 128 u = [448, 264, 272, 304, 288, 144, 136, 68, 2.5 * 2^-9, 264] has amax 448, so
+    scale 1 and E4M3 codes [448 (max), 256 (nearest), 256 (tie, even below), 320 (tie, even
+    above), 288, 144, 128 (tie), 64 (tie), 2^-8 (subnormal tie), 256].
+    W_down is the identity on features 0..9, so y_j is h's code; column 31 holds 2 at row 10
+    (h_10 = 0) and 1.25 * 2^-15 at row 0: its block's scale is 2^(1-8), the entry scales to
+    2.5 * 2^-9, a subnormal tie rounded to 2 * 2^-9, so y_31 = 448 * 2^-15.
+    """
+    H = Hp = 32
+    x = np.zeros((1, H))
+    x[0, :2] = (2.0, 1.0625)
+    wg = np.zeros((H, Hp))
+    wg[0, :] = 64.0
+    a = [1.5, 1.0, 0.5625, 1.125, 1.0, 0.5, 0.5, 0.25, 1.25 * 2 ** -16, 1.0625]
+    b = [0.5, 0.0625, 1.0, 0.125, 0.25, 0.125, 0.0625, 0.03125, 0.0, 0.0625]
+    wu = np.zeros((H, Hp))
+    wu[0, :10], wu[1, :10] = a, b
+    wd = np.zeros((Hp, H))
+    wd[np.arange(10), np.arange(10)] = 1.0
+    wd[0, 31], wd[10, 31] = 1.25 * 2 ** -15, 2.0
+    bits = {k: O.f64_to_bf16_bits(v) for k, v in (("x", x), ("wg", wg), ("wu", wu), ("wd", wd))}
+    for k, v in (("x", x), ("wg", wg), ("wu", wu), ("wd", wd)):
+        np.testing.assert_array_equal(O.bf16_bits_to_f64(bits[k]), v)  # inputs are bf16 values
+
+    codes = np.zeros(Hp)
+    codes[:10] = [448, 256, 256, 320, 288, 144, 128, 64, 2.0 ** -8, 256]
+    y_want = np.zeros(H)
+    y_want[:10] = codes[:10]
+    y_want[31] = 448 * 2.0 ** -15
+
+    xq, xs = O.mx_quantize(O.bf16_bits_to_f64(bits["x"]))
+    np.testing.assert_array_equal(xq[0, :3], [256.0, 128.0, 0.0])
+    assert xs[0, 0] == -7
+    hq, hs, y = O.expert_ffn_rows_mxfp8(bits["x"], O.mx_weights(bits["wg"]),
+                                        O.mx_weights(bits["wu"]), O.mx_weights(bits["wd"]))
+    np.testing.assert_array_equal(hq[0], codes)
+    assert hs.shape == (1, 1) and hs[0, 0] == 0
+    np.testing.assert_array_equal(O.bf16_bits_to_f64(y)[0], y_want)
+
+    # what each dropped step would give instead (worked out by hand from the values above)
+    no_x_quant = 128 * (2 * 0.5625 + 1.0625 * 1.0)       # h_2 = 280 -> code 288, not 256
+    no_h_quant = 264.0                                     # y_1 = bf16(264) = 264, not 256
+    no_up_weight_quant = 128 * (2 * 1.0625 + 0.0625)      # h_9 = 280 -> code 288, not 256
+    no_down_weight_quant = 448 * 1.25 * 2.0 ** -15        # also the row-wise (wrong axis) value
+    assert O.e4m3_round(np.array([no_x_quant]))[0] == 288 != y_want[2]
+    assert no_h_quant != y_want[1]
+    assert O.e4m3_round(np.array([no_up_weight_quant]))[0] == 288 != y_want[9]
+    assert no_down_weight_quant != y_want[31]
+    row_wise = O.mx_quantize(O.bf16_bits_to_f64(bits["wd"]), axis=-1)  # wrong axis for Down
+    assert O.mx_dequantize(*row_wise, axis=-1)[0, 31] == 1.25 * 2 ** -15
