@@ -31,7 +31,8 @@ MOE_ERR_UNSUPPORTED_SHAPE = 2
 MOE_ERR_CUDA = 3
 MOE_ERR_BAD_ROUTING = 4
 MOE_ERR_DEVICE_TIMEOUT = 8
-MOE_MAX_EXPERTS = 1024
+MOE_MAX_EXPERTS = 65535
+MOE_MAX_FFN_EXPERTS = 1024
 
 # Kernels launched by one call of each entry point (permute with a row copy).
 LAUNCHES = {"moe_permute": 2, "moe_grouped_ffn": 2, "moe_grouped_ffn_up_gate": 1,

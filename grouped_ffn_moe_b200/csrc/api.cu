@@ -120,6 +120,7 @@ int32_t moe_abi_version(void) { return (1 << 16) | 2; }
 
 size_t moe_permute_workspace_bytes(int64_t S, int32_t K, int32_t E) {
   if (S <= 0 || K <= 0 || E <= 0) return 0;
+  if (moe::permute_uses_cluster(S * K, E)) return 0;  // metadata in one cluster's shared memory
   const int64_t nchunk = moe::permute_num_chunks(S * K);
   const size_t bytes = sizeof(int32_t) * static_cast<size_t>(nchunk) * static_cast<size_t>(E);
   return (bytes + 255) & ~static_cast<size_t>(255);
@@ -155,7 +156,7 @@ moe_status moe_permute(const void* x, const int32_t* topk_ids, int64_t S, int64_
     return MOE_OK;
   }
   const size_t need = moe_permute_workspace_bytes(S, K, E);
-  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16))
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)))
     return MOE_ERR_INVALID_ARGUMENT;
   return moe::launch_permute(x, topk_ids, S, H, K, E, x_perm, counts, cu_seqlens, row_id_map,
                              perm_src, maxvio, max_count, static_cast<int32_t*>(workspace),
@@ -166,7 +167,7 @@ namespace {
 
 moe_status check_ffn_shapes(int64_t M, int64_t H, int64_t Hp, int32_t E) {
   if (M < 0 || H <= 0 || Hp <= 0 || E < 1) return MOE_ERR_INVALID_ARGUMENT;
-  if (E > MOE_MAX_EXPERTS || M > moe::kMaxRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (E > MOE_MAX_FFN_EXPERTS || M > moe::kMaxRows) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (H % 128 != 0 || Hp % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (static_cast<int64_t>(E) * H > moe::kMaxRows || static_cast<int64_t>(E) * Hp > moe::kMaxRows)
     return MOE_ERR_UNSUPPORTED_SHAPE;

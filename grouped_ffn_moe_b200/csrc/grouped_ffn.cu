@@ -69,8 +69,8 @@ struct Cfg {
   static constexpr int kPipeBytes = kStages * kStageBytes;
   static constexpr int kOffOut = kPipeBytes;
   static constexpr int kOffCu = kOffOut + kEpiGroups * kOutBytes;
-  static constexpr int kOffUnits = kOffCu + 4 * (MOE_MAX_EXPERTS + 1);
-  static constexpr int kOffBars = (kOffUnits + 4 * (MOE_MAX_EXPERTS + 1) + 7) & ~7;
+  static constexpr int kOffUnits = kOffCu + 4 * (MOE_MAX_FFN_EXPERTS + 1);
+  static constexpr int kOffBars = (kOffUnits + 4 * (MOE_MAX_FFN_EXPERTS + 1) + 7) & ~7;
   static constexpr int kNumBars = 2 * kStages + 2 * 2 + 1;
   static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 128 + 1024;  // + alignment slack

@@ -52,8 +52,8 @@ struct DCfg {
   static constexpr int kPipeBytes = kStages * kStageBytes;
   static constexpr int kOffEpi = kPipeBytes;
   static constexpr int kOffCu = kOffEpi + kEpiBytes;
-  static constexpr int kOffUnits = kOffCu + 4 * (MOE_MAX_EXPERTS + 1);
-  static constexpr int kOffBars = (kOffUnits + 4 * (MOE_MAX_EXPERTS + 1) + 7) & ~7;
+  static constexpr int kOffUnits = kOffCu + 4 * (MOE_MAX_FFN_EXPERTS + 1);
+  static constexpr int kOffBars = (kOffUnits + 4 * (MOE_MAX_FFN_EXPERTS + 1) + 7) & ~7;
   static constexpr int kNumBars = 2 * kStages + 2 * 2 + 1;
   static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
@@ -357,7 +357,7 @@ constexpr int kWOffEpi = kWStages * kWStageBytes;
 constexpr int kWOffCu = kWOffEpi + (kEpiThreads / 32) * kWEpiTiles * kWEpiTileBytes;
 // expert row offsets: a shared copy of cu_seqlens, or (when the pipeline needs the room)
 // two cached global loads per unit
-constexpr int kWCuBytes = MOE_WGRAD_SMEM_CU ? 4 * (MOE_MAX_EXPERTS + 1) : 0;
+constexpr int kWCuBytes = MOE_WGRAD_SMEM_CU ? 4 * (MOE_MAX_FFN_EXPERTS + 1) : 0;
 constexpr int kWOffBars = (kWOffCu + kWCuBytes + 7) & ~7;
 constexpr int kWNumBars = 2 * kWStages + 2 * 2 + 1;
 constexpr int kWOffMisc = kWOffBars + 8 * kWNumBars;

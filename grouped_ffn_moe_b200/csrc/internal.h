@@ -11,21 +11,23 @@
 
 namespace moe {
 
-// Flat routing slots handled by one warp in the permutation kernels: 512 for large tables,
-// 64 up to 65536 slots, where 512-slot chunks would leave all but a few SMs idle (a chunk
-// is walked 32 slots at a time by one warp).
-constexpr int kChunkMax = 512;
-constexpr int kChunkSmall = 64;
-constexpr int64_t kSmallTableSlots = 65536;
-constexpr int kWarpsPerTile = 8;
-
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-inline int32_t permute_chunk_slots(int64_t F) {
-  return F <= kSmallTableSlots ? kChunkSmall : kChunkMax;
+// The permutation's metadata (counts, cu_seqlens, stable ranks) is computed by one
+// thread-block cluster, with no workspace, for routing tables of up to kClusterMaxSlots flat
+// slots and for any table with more experts than the cooperative kernel's shared-memory
+// histograms hold; larger tables go to a cooperative grid over all SMs that keeps per-chunk
+// counts in the caller's workspace.
+constexpr int64_t kClusterMaxSlots = int64_t{1} << 20;
+constexpr int kCoopMaxExperts = 1024;
+constexpr int kChunkSlots = 512;  // flat slots per warp (one chunk) in the cooperative kernel
+constexpr int kWarpsPerTile = 8;
+
+inline bool permute_uses_cluster(int64_t F, int32_t E) {
+  return F <= kClusterMaxSlots || E > kCoopMaxExperts;
 }
 
-inline int64_t permute_num_chunks(int64_t F) { return ceil_div(F, permute_chunk_slots(F)); }
+inline int64_t permute_num_chunks(int64_t F) { return ceil_div(F, kChunkSlots); }
 
 // Number of SMs of the current device (cached per device).
 int num_sms();
@@ -81,6 +83,7 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
   return err;
 }
 
+// chunk_counts: the workspace (used by the cooperative path only; may be null otherwise).
 moe_status launch_permute(const void* x, const int32_t* topk_ids, int64_t S, int64_t H, int32_t K,
                           int32_t E, void* x_perm, int32_t* counts, int32_t* cu_seqlens,
                           int32_t* row_id_map, int32_t* perm_src, double* maxvio,

@@ -39,8 +39,9 @@
  *     on device data are OR-ed into *d_status (a device int32 the caller zeroes and reads
  *     when it chooses; may be NULL to skip reporting).
  *   - Preconditions, checked on the host: pointers non-NULL and 16-byte aligned (unless
- *     documented nullable), H and Hp multiples of 8 (of 128 for moe_grouped_ffn),
- *     1 <= K <= E <= MOE_MAX_EXPERTS, S*K < 2^31. S = 0 is a legal no-op.
+ *     documented nullable), H and Hp multiples of 8 (of 128 for the grouped FFN calls),
+ *     1 <= K <= E <= MOE_MAX_EXPERTS (E <= MOE_MAX_FFN_EXPERTS for the grouped FFN calls),
+ *     S*K < 2^31. S = 0 is a legal no-op.
  *   - Results are deterministic: no floating-point atomics; every sum has a fixed order.
  */
 #ifndef MOE_B200_H_
@@ -62,8 +63,14 @@ typedef int32_t moe_status;
 #define MOE_ERR_BAD_ROUTING 4       /* device: an expert id outside [0, E)               */
 #define MOE_ERR_DEVICE_TIMEOUT 8    /* device: a bounded wait in a kernel ran out        */
 
-/* Largest E the kernels accept (per-expert tables live in shared memory). */
-#define MOE_MAX_EXPERTS 1024
+/* Largest E of the routing calls (moe_permute, moe_permute_no_alloc, moe_maxvio,
+ * moe_append_shared): expert ids fit in 16 bits. */
+#define MOE_MAX_EXPERTS 65535
+
+/* Largest E of the grouped FFN calls (forward, backward, MXFP8): every CTA of their
+ * persistent grids keeps the per-expert row offsets and work-unit offsets in shared memory
+ * (2 x 4 KiB at 1024 experts, next to 192 KiB of operand pipeline). */
+#define MOE_MAX_FFN_EXPERTS 1024
 
 /* Static description of a status code. Never NULL. */
 const char* moe_status_string(moe_status s);
@@ -72,8 +79,10 @@ const char* moe_status_string(moe_status s);
 int32_t moe_abi_version(void);
 
 /*
- * Bytes of device workspace moe_permute needs for (S, K, E): per-expert counts of every
- * 512-slot chunk of the flat routing table, rounded up to 256 bytes. 0 when S == 0.
+ * Bytes of device workspace moe_permute needs for (S, K, E). 0 when S*K <= 2^20 or
+ * E > 1024: the metadata is then computed in one thread-block cluster's shared memory.
+ * Otherwise the per-expert counts of every 512-slot chunk of the flat routing table,
+ * rounded up to 256 bytes.
  */
 size_t moe_permute_workspace_bytes(int64_t S, int32_t K, int32_t E);
 
@@ -95,7 +104,7 @@ size_t moe_permute_workspace_bytes(int64_t S, int32_t K, int32_t E);
  *   maxvio     device double out, nullable: as moe_maxvio on the counts.
  *   max_count  device int32 out, nullable: max_e counts[e].
  *   workspace  device scratch of moe_permute_workspace_bytes(S, K, E) bytes (contents
- *              ignored on entry, undefined on exit).
+ *              ignored on entry, undefined on exit); may be NULL when that size is 0.
  *   d_status   nullable device int32: MOE_ERR_BAD_ROUTING is OR-ed in if any id is outside
  *              [0, E); such slots are dropped (row_id_map[f] = -1) and counts no longer sum
  *              to S*K.
@@ -156,7 +165,7 @@ moe_status moe_permute_no_alloc(const void* x, const int32_t* topk_ids, int64_t 
  *               [0, M) are never written.
  *   h_scratch   [M, Hp] bf16 out: the SwiGLU activations (kept: the backward pass needs them).
  *   y           [M, H] bf16 out: expert outputs, row-aligned with x_perm.
- *   Requires H % 128 == 0, Hp % 128 == 0, 1 <= E <= MOE_MAX_EXPERTS, M < 2^31.
+ *   Requires H % 128 == 0, Hp % 128 == 0, 1 <= E <= MOE_MAX_FFN_EXPERTS, M < 2^31.
  *   d_status    nullable: MOE_ERR_DEVICE_TIMEOUT is OR-ed in if a pipeline wait in the kernel
  *               exceeded its bound (outputs are then incomplete).
  */
@@ -195,7 +204,8 @@ moe_status moe_grouped_ffn_down(const void* h_scratch, const void* w_down,
  *   holding its column slices (SwiGLU is element-wise over H', so the slices' down
  *   projections add up to the full one). The routed imbalance is moe_maxvio on the first E
  *   counts with the routed K; moe_permute's own maxvio covers all E + n_shared experts.
- * Requires E + n_shared <= MOE_MAX_EXPERTS, S*(K+n_shared) < 2^31.
+ * Requires E + n_shared <= MOE_MAX_EXPERTS (<= MOE_MAX_FFN_EXPERTS to run the grouped FFN on
+ * the result), S*(K+n_shared) < 2^31.
  */
 moe_status moe_append_shared(const int32_t* topk_ids, const float* route_w, int64_t S, int32_t K,
                              int32_t E, int32_t n_shared, int32_t* ids_out, float* w_out,

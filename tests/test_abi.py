@@ -48,9 +48,13 @@ def test_status_strings_and_version():
 
 def test_workspace_bytes():
     assert moe.moe_permute_workspace_bytes(0, 8, 384) == 0
-    # 65536 tokens x 8 slots = 1024 chunks of 512, times 384 experts, int32
-    assert moe.moe_permute_workspace_bytes(65536, 8, 384) == 1024 * 384 * 4
-    assert moe.moe_permute_workspace_bytes(3, 2, 8) % 256 == 0
+    # up to 2^20 routed slots, or more than 1024 experts: one cluster, no workspace
+    assert moe.moe_permute_workspace_bytes(65536, 8, 384) == 0
+    assert moe.moe_permute_workspace_bytes(1 << 17, 8, 1024) == 0
+    assert moe.moe_permute_workspace_bytes(1 << 18, 8, 4096) == 0
+    # above: 2^21 slots = 4096 chunks of 512, times 384 experts, int32
+    assert moe.moe_permute_workspace_bytes(1 << 18, 8, 384) == 4096 * 384 * 4
+    assert moe.moe_permute_workspace_bytes((1 << 18) + 1, 8, 100) % 256 == 0
 
 
 P = ctypes.c_void_p
@@ -66,8 +70,8 @@ def test_host_validation_rejects_without_launch():
     null = P(0)
     # K > E
     assert L.moe_permute(a, a, 4, 64, 9, 8, a, a, a, a, null, null, null, a, 1 << 20, null, null) == 1
-    # E beyond the supported maximum
-    assert L.moe_permute(a, a, 4, 64, 2, 5000, a, a, a, a, null, null, null, a, 1 << 20, null,
+    # E beyond the supported maximum (65535)
+    assert L.moe_permute(a, a, 4, 64, 2, 70000, a, a, a, a, null, null, null, a, 1 << 20, null,
                          null) == 2
     # missing outputs
     assert L.moe_permute(a, a, 4, 64, 2, 8, a, null, a, a, null, null, null, a, 1 << 20, null,
@@ -77,8 +81,11 @@ def test_host_validation_rejects_without_launch():
     # misaligned x_perm
     assert L.moe_permute(a, a, 4, 64, 2, 8, fake(0x10008), a, a, a, null, null, null, a, 1 << 20,
                          null, null) == 1
-    # workspace too small
-    assert L.moe_permute(a, a, 4096, 64, 8, 384, a, a, a, a, null, null, null, a, 16, null, null) == 1
+    # workspace too small (2^21 slots need one)
+    assert L.moe_permute(a, a, 1 << 18, 64, 8, 384, a, a, a, a, null, null, null, a, 16, null,
+                         null) == 1
+    # grouped FFN: more experts than its shared-memory tables hold
+    assert L.moe_grouped_ffn(a, a, a, a, a, 16, 256, 256, 1025, a, a, null, null) == 2
     # grouped FFN: H' not a multiple of 128, then a null weight
     assert L.moe_grouped_ffn(a, a, a, a, a, 16, 256, 200, 4, a, a, null, null) == 2
     assert L.moe_grouped_ffn(a, null, a, a, a, 16, 256, 256, 4, a, a, null, null) == 1
@@ -130,7 +137,7 @@ def test_host_validation_of_backward_gather_and_shared_calls():
                                             null) == 1
     assert L.moe_grouped_ffn_gather(a, a, 0, 2, a, a, a, a, 256, 256, 4, a, a, null, null) == 0
     # shared experts: E + n beyond the maximum, n < 1, S = 0 no-op
-    assert L.moe_append_shared(a, a, 4, 2, 1024, 1, a, a, null) == 2
+    assert L.moe_append_shared(a, a, 4, 2, 65535, 1, a, a, null) == 2
     assert L.moe_append_shared(a, a, 4, 2, 8, 0, a, a, null) == 1
     assert L.moe_append_shared(a, a, 0, 2, 8, 1, a, a, null) == 0
 

@@ -16,7 +16,7 @@ import torch
 
 import grouped_ffn_moe_b200 as moe
 import synth
-from helpers import assert_close_bf16, assert_close_fp32_sums, bits
+from helpers import GUARD, assert_close_bf16, assert_close_fp32_sums, bits
 from oracle import moe_oracle as O
 
 pytestmark = pytest.mark.gpu

@@ -119,12 +119,32 @@ def _routing_case(name):
         return rng.integers(0, 1024, size=(3000, 8)).astype(np.int32), 1024
     if name == "many_chunks":
         return rng.integers(0, 384, size=(20000, 8)).astype(np.int32), 384
+    if name == "e4096":  # four expert windows of the cluster kernel
+        return rng.integers(0, 4096, size=(3000, 8)).astype(np.int32), 4096
+    if name == "e65535":  # the largest E: 64 windows, ids at both ends of the range
+        ids = rng.integers(0, 65535, size=(4001, 6)).astype(np.int32)
+        ids[:50, 0], ids[50:100, 1], ids[100:140, 2] = 0, 65534, 1023
+        return ids, 65535
+    if name == "e3000_hot":  # a hot expert in the last, partial window
+        ids = rng.integers(0, 3000, size=(5000, 4)).astype(np.int32)
+        ids[::3, 1] = 2999
+        return ids, 3000
+    if name == "cluster_max":  # exactly 2^20 slots: the cluster kernel's largest table
+        return rng.integers(0, 384, size=(131072, 8)).astype(np.int32), 384
+    if name == "coop_e64":  # above 2^20 slots: the cooperative kernel and its workspace
+        return rng.integers(0, 64, size=(262147, 6)).astype(np.int32), 64
+    if name == "coop_e1024":
+        return rng.integers(0, 1024, size=(135001, 8)).astype(np.int32), 1024
     raise KeyError(name)
 
 
 @pytest.mark.parametrize("name", ["one_expert_k1", "empty_experts", "duplicates", "ragged", "e_max",
-                                  "many_chunks"])
+                                  "many_chunks", "e4096", "e65535", "e3000_hot", "cluster_max",
+                                  "coop_e64", "coop_e1024"])
 def test_permute_edge_cases(cuda_device, name):
+    """Metadata and rows bit-exact against the oracle: edge routings, E up to 65535 (the
+    cluster kernel's expert windows), and tables on both sides of 2^20 slots (the cluster
+    kernel without workspace, the cooperative kernel with one)."""
     ids_np, E = _routing_case(name)
     S, K = ids_np.shape
     H = 64
@@ -161,16 +181,21 @@ def test_permute_metadata_only_and_zero_tokens(cuda_device):
     assert np.isnan(r0["maxvio"].item())
 
 
-def test_bad_routing_is_flagged(cuda_device):
-    ids_np = np.array([[0, 1], [2, 7], [3, -1], [1, 2]], dtype=np.int32)
+@pytest.mark.parametrize("E,bad_id", [(4, 7), (3000, 3000), (3000, 70000)])
+def test_bad_routing_is_flagged(cuda_device, E, bad_id):
+    """Ids outside [0, E) set MOE_ERR_BAD_ROUTING, get row -1 and are not counted; with
+    E = 3000 the valid ids fall in different expert windows of the cluster kernel."""
+    ids_np = np.array([[0, 1], [2, bad_id], [3, -1], [1, E - 1]], dtype=np.int32)
     ids = torch.from_numpy(ids_np).to(cuda_device)
     x = torch.ones(4, 64, dtype=torch.bfloat16, device=cuda_device)
-    r = gpu_permute(x, ids, 4)
+    r = gpu_permute(x, ids, E)
     assert int(r["status"].item()) & moe.MOE_ERR_BAD_ROUTING
     rmap = r["rmap"].cpu().numpy()
     assert rmap[3] == -1 and rmap[5] == -1
     good = ids_np.reshape(-1)[[0, 1, 2, 4, 6, 7]]
-    assert r["counts"].tolist() == np.bincount(good, minlength=4).tolist()
+    assert r["counts"].tolist() == np.bincount(good, minlength=E).tolist()
+    ok = np.sort(rmap[rmap >= 0])
+    assert np.array_equal(ok, np.arange(6))  # the valid slots fill rows 0..5
 
 
 def test_maxvio_entry_point(cuda_device):
@@ -181,6 +206,12 @@ def test_maxvio_entry_point(cuda_device):
     torch.cuda.synchronize()
     assert mc.item() == 3584
     assert mv.item() == O.maxvio(counts.cpu().numpy(), 8192, 8)[0] == 20.0
+    # the largest E, hot expert last: 65535 experts, S*K = 65535 * 2 rows
+    c = np.full(65535, 2, np.int32)
+    c[0], c[-1] = 1, 3
+    moe.moe_maxvio(torch.from_numpy(c).to(cuda_device), 65535, 2, mv, mc)
+    torch.cuda.synchronize()
+    assert mc.item() == 3 and mv.item() == O.maxvio(c, 65535, 2)[0] == 0.5
 
 
 # ----------------------------------------------------------------------------- combine
@@ -398,40 +429,6 @@ def test_generator_twin_matches_host(cuda_device):
                                    synth.TAG_W_GATE, 0.125, offset=off)
         host = synth.normal_bf16_bits(2, synth.TAG_W_GATE, n, 0.125, offset=off)
         assert (bits(t) != host).sum() <= 2
-
-
-@pytest.mark.parametrize("wname", ["permute_combine_S4096_mv20", "permute_combine_S16384_mv1",
-                                   "medium"])
-def test_permute_variants_agree(cuda_device, tmp_path, wname):
-    """The fused cooperative permutation (default) and the three-launch staged one
-    (MOE_PERMUTE_KERNEL=staged) give bit-identical metadata and rows."""
-    import subprocess
-    import sys
-
-    script = (
-        "import sys, torch, synth, grouped_ffn_moe_b200 as moe\n"
-        f"w = synth.WORKLOADS['{wname}']\n"
-        "inp = synth.make_layer_inputs(w, device='cuda:0')\n"
-        "buf = moe.LayerBuffers.allocate(w.S, w.H, 0, w.E, w.K, torch.device('cuda:0'),"
-        " with_ffn=False)\n"
-        "moe.moe_layer_forward(inp['x'], inp['topk_ids'], inp['route_w'], None, None, None, buf)\n"
-        "torch.cuda.synchronize()\n"
-        "assert int(buf.d_status.item()) == 0\n"
-        "torch.save({k: getattr(buf, k).cpu() for k in ('x_perm', 'counts', 'cu_seqlens',"
-        " 'row_id_map', 'perm_src', 'maxvio', 'max_count', 'out')}, sys.argv[1])\n")
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    outs = {}
-    for mode in ("fused", "staged"):
-        env = dict(os.environ, MOE_PERMUTE_KERNEL=mode, PYTHONPATH=root)
-        path = str(tmp_path / f"p_{mode}.pt")
-        subprocess.run([sys.executable, "-c", script, path], check=True, env=env, cwd=root,
-                       timeout=600)
-        outs[mode] = torch.load(path)
-    for k, v in outs["fused"].items():
-        a, b = v, outs["staged"][k]
-        if a.dtype == torch.bfloat16:
-            a, b = a.view(torch.int16), b.view(torch.int16)
-        assert torch.equal(a, b), k
 
 
 def test_device_wait_timeout_reports_status_and_keeps_context(cuda_device, tmp_path):

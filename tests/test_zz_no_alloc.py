@@ -14,17 +14,18 @@ import torch
 
 import grouped_ffn_moe_b200 as moe
 import synth
+from helpers import GUARD
 
 pytestmark = pytest.mark.gpu
 
 
 def _outputs(S, K, E, H, dev):
-    i32 = dict(dtype=torch.int32, device=dev)
-    return dict(x_perm=torch.full((S * K, H), float("nan"), dtype=torch.bfloat16, device=dev),
-                counts=torch.full((E,), -9, **i32), cu=torch.full((E + 1,), -9, **i32),
-                rmap=torch.full((S * K,), -9, **i32), psrc=torch.full((S * K,), -9, **i32),
-                maxvio=torch.full((1,), -9.0, dtype=torch.float64, device=dev),
-                max_count=torch.full((1,), -9, **i32), status=torch.zeros(1, **i32))
+    i32 = torch.int32
+    return dict(x_perm=GUARD.full((S * K, H), float("nan"), torch.bfloat16, dev),
+                counts=GUARD.full((E,), -9, i32, dev), cu=GUARD.full((E + 1,), -9, i32, dev),
+                rmap=GUARD.full((S * K,), -9, i32, dev), psrc=GUARD.full((S * K,), -9, i32, dev),
+                maxvio=GUARD.full((1,), -9.0, torch.float64, dev),
+                max_count=GUARD.full((1,), -9, i32, dev), status=GUARD.zeros((1,), i32, dev))
 
 
 def _call(fn_name, x, ids, E, o, workspace=None):
@@ -41,15 +42,19 @@ def _call(fn_name, x, ids, E, o, workspace=None):
     assert st == 0, moe.moe_status_string(st)
 
 
-def test_no_alloc_permute_matches_workspace_permute_twice(cuda_device):
+@pytest.mark.parametrize("S,K,E,H", [(262147, 6, 64, 64), (4096, 6, 64, 2048)])
+def test_no_alloc_permute_matches_workspace_permute_twice(cuda_device, S, K, E, H):
+    """Above 2^20 routed slots the permutation keeps per-chunk counts in its scratch (the
+    library's array here, a caller workspace for moe_permute); up to 2^20 it needs none."""
     dev = cuda_device
-    S, K, E, H = 4096, 6, 64, 2048
+    need = moe.moe_permute_workspace_bytes(S, K, E)
+    assert (need > 0) == (S * K > (1 << 20)) and need <= moe.MOE_NO_ALLOC_SCRATCH_BYTES
     x = synth.normal_bf16_into(torch.empty(S, H, dtype=torch.bfloat16, device=dev), 1, synth.TAG_X)
     routings = [synth.route_es(1, S, K, E)[0],
-                synth.route_capped_for_maxvio(5, S, K, E, 20.0, hot_e=E - 1)[0]]
+                synth.route_es(5, S, K, E, hot_e=E - 1, w_hot=20.0)[0]]
     for ids_np in routings:  # two calls in a row; the second reuses the library's array
         ids = torch.from_numpy(ids_np).to(dev)
-        ws = torch.empty(moe.moe_permute_workspace_bytes(S, K, E), dtype=torch.uint8, device=dev)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         ref, got = _outputs(S, K, E, H, dev), _outputs(S, K, E, H, dev)
         _call("moe_permute", x, ids, E, ref, ws)
         _call("moe_permute_no_alloc", x, ids, E, got)
