@@ -17,8 +17,13 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // thread-block cluster, with no workspace, for routing tables of up to kClusterMaxSlots flat
 // slots and for any table with more experts than the cooperative kernel's shared-memory
 // histograms hold; larger tables go to a cooperative grid over all SMs that keeps per-chunk
-// counts in the caller's workspace.
-constexpr int64_t kClusterMaxSlots = int64_t{1} << 20;
+// counts in the caller's workspace. (Measured on B200: the cluster kernel takes 10 us at 8K
+// slots and 29 us at 128K, the cooperative one 29-35 us over that range and 33 us at 512K,
+// where the cluster kernel's 16 SMs need 80 us.)
+#ifndef MOE_CLUSTER_MAX_SLOTS
+#define MOE_CLUSTER_MAX_SLOTS (int64_t{1} << 17)
+#endif
+constexpr int64_t kClusterMaxSlots = MOE_CLUSTER_MAX_SLOTS;
 constexpr int kCoopMaxExperts = 1024;
 constexpr int kChunkSlots = 512;  // flat slots per warp (one chunk) in the cooperative kernel
 constexpr int kWarpsPerTile = 8;

@@ -9,7 +9,7 @@
 // Two launches, no host synchronisation, no atomics on data:
 //
 //   metadata  counts, cu_seqlens, maxvio and the stable ranks (row_id_map, perm_src). Up to
-//             2^20 flat slots (and for any E above 1024) by one thread-block cluster: every
+//             2^17 flat slots (and for any E above 1024) by one thread-block cluster: every
 //             warp owns a contiguous run of slots, counts them per expert in its own shared
 //             histogram (__match_any_sync finds the lanes holding the same expert), the CTA
 //             scans its warps' counts, the CTAs exchange their totals through distributed
@@ -53,6 +53,11 @@ constexpr int kClThreads = 32 * kClWarps;  // 1024: one expert of a window per t
 constexpr int kClWindow = kClThreads;      // experts per window
 constexpr int kClRegSteps = 8;             // 32-slot steps per warp whose ids stay in registers
 constexpr size_t kClSmemBytes = sizeof(int32_t) * (kClWarps + 1) * kClWindow;
+#ifndef MOE_CLUSTER_CTAS
+#define MOE_CLUSTER_CTAS 16
+#endif
+constexpr int kClMaxCtas = MOE_CLUSTER_CTAS;  // largest cluster tried (16: non-portable size)
+static_assert(kClMaxCtas >= 1 && kClMaxCtas <= 16, "cluster size");
 
 struct ClusterArgs {
   const int32_t* ids;
@@ -132,23 +137,31 @@ __global__ void __launch_bounds__(kClThreads, 1) route_cluster_kernel(const Clus
   const int64_t f_begin = min(g * a.per_warp, a.F);
   const int64_t f_end = min(f_begin + a.per_warp, a.F);
   const int nsteps = static_cast<int>((f_end - f_begin + 31) / 32);  // warp-uniform
+  // ids of the warp's first kClRegSteps steps stay in registers; later steps are read in
+  // batches of kClRegSteps (all loads of a batch in flight before its first use)
   int32_t idr[kClRegSteps];
+  auto load_batch = [&](int j0, int32_t (&v)[kClRegSteps]) {
 #pragma unroll
-  for (int j = 0; j < kClRegSteps; ++j) {
-    const int64_t f = f_begin + j * 32 + lane;
-    idr[j] = (j < nsteps && f < f_end) ? __ldg(a.ids + f) : -1;
-  }
-  // the id of step j for this lane (-1 past the warp's slots)
-  auto id_at = [&](int j) -> int32_t {
-    if (j < kClRegSteps) {
-      int32_t v = -1;
+    for (int i = 0; i < kClRegSteps; ++i) {
+      const int64_t f = f_begin + (j0 + i) * 32 + lane;
+      v[i] = (j0 + i < nsteps && f < f_end) ? __ldg(a.ids + f) : -1;
+    }
+  };
+  load_batch(0, idr);
+  // body(j, f, e) for every step j of the warp's run, in order
+  auto for_each_step = [&](auto&& body) {
+    for (int j0 = 0; j0 < nsteps; j0 += kClRegSteps) {
+      int32_t v[kClRegSteps];
+      if (j0 == 0) {
+#pragma unroll
+        for (int i = 0; i < kClRegSteps; ++i) v[i] = idr[i];
+      } else {
+        load_batch(j0, v);
+      }
 #pragma unroll
       for (int i = 0; i < kClRegSteps; ++i)
-        if (i == j) v = idr[i];
-      return v;
+        if (j0 + i < nsteps) body(f_begin + (j0 + i) * 32 + lane, v[i]);  // warp-uniform
     }
-    const int64_t f = f_begin + j * 32 + lane;
-    return f < f_end ? __ldg(a.ids + f) : -1;
   };
 
   bool bad = false;
@@ -158,16 +171,14 @@ __global__ void __launch_bounds__(kClThreads, 1) route_cluster_kernel(const Clus
     for (int i = lane; i < ew; i += 32) my[i] = 0;
     __syncwarp();
     // A
-    for (int j = 0; j < nsteps; ++j) {
-      const int64_t f = f_begin + j * 32 + lane;
-      const int32_t e = id_at(j);
+    for_each_step([&](int64_t f, int32_t e) {
       if (e0 == 0) bad |= (f < f_end) && (e < 0 || e >= a.E);
       const bool in = (f < f_end) && e >= e0 && e < e0 + ew;
       const int32_t key = in ? e - e0 : -1;
       const unsigned peers = __match_any_sync(kFull, key);
       if (in && lane == __ffs(peers) - 1) my[key] += __popc(peers);
       __syncwarp();
-    }
+    });
     __syncthreads();
     // B
     int32_t cta_total = 0;
@@ -184,10 +195,13 @@ __global__ void __launch_bounds__(kClThreads, 1) route_cluster_kernel(const Clus
     int32_t base = 0, total = 0;
     if (tid < ew) {
       const uint32_t addr = smem_u32(tot + tid);
-      for (uint32_t r = 0; r < ncta; ++r) {
-        const int32_t v = ld_shared_cluster(map_to_cta(addr, r));
-        base += r < rank ? v : 0;
-        total += v;
+      int32_t v[16];  // all of the (at most 16) reads in flight before the sums
+#pragma unroll
+      for (uint32_t r = 0; r < 16; ++r) v[r] = r < ncta ? ld_shared_cluster(map_to_cta(addr, r)) : 0;
+#pragma unroll
+      for (uint32_t r = 0; r < 16; ++r) {
+        base += r < rank ? v[r] : 0;
+        total += v[r];
       }
     }
     cluster_arrive();  // this CTA is done reading the others' totals
@@ -205,9 +219,7 @@ __global__ void __launch_bounds__(kClThreads, 1) route_cluster_kernel(const Clus
     run_max = max(run_max, wmax);
     __syncthreads();
     // D
-    for (int j = 0; j < nsteps; ++j) {
-      const int64_t f = f_begin + j * 32 + lane;
-      const int32_t e = id_at(j);
+    for_each_step([&](int64_t f, int32_t e) {
       const bool in = (f < f_end) && e >= e0 && e < e0 + ew;
       const int32_t key = in ? e - e0 : -1;
       const unsigned peers = __match_any_sync(kFull, key);
@@ -221,7 +233,7 @@ __global__ void __launch_bounds__(kClThreads, 1) route_cluster_kernel(const Clus
       } else if (e0 == 0 && f < f_end && (e < 0 || e >= a.E)) {
         a.row_id_map[f] = -1;  // dropped slot
       }
-    }
+    });
     cluster_wait();  // no CTA still reads this CTA's totals: they may be rewritten
     __syncthreads();
   }
@@ -516,7 +528,7 @@ int cluster_size() {
     return 0;
   }
   int best = 0;
-  for (int c = 16; c >= 1 && best == 0; c >>= 1) {
+  for (int c = kClMaxCtas; c >= 1 && best == 0; c >>= 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(c);
     cfg.blockDim = dim3(kClThreads);

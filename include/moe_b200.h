@@ -79,7 +79,7 @@ const char* moe_status_string(moe_status s);
 int32_t moe_abi_version(void);
 
 /*
- * Bytes of device workspace moe_permute needs for (S, K, E). 0 when S*K <= 2^20 or
+ * Bytes of device workspace moe_permute needs for (S, K, E). 0 when S*K <= 2^17 or
  * E > 1024: the metadata is then computed in one thread-block cluster's shared memory.
  * Otherwise the per-expert counts of every 512-slot chunk of the flat routing table,
  * rounded up to 256 bytes.

@@ -48,13 +48,13 @@ def test_status_strings_and_version():
 
 def test_workspace_bytes():
     assert moe.moe_permute_workspace_bytes(0, 8, 384) == 0
-    # up to 2^20 routed slots, or more than 1024 experts: one cluster, no workspace
-    assert moe.moe_permute_workspace_bytes(65536, 8, 384) == 0
-    assert moe.moe_permute_workspace_bytes(1 << 17, 8, 1024) == 0
+    # up to 2^17 routed slots, or more than 1024 experts: one cluster, no workspace
+    assert moe.moe_permute_workspace_bytes(16384, 8, 384) == 0
+    assert moe.moe_permute_workspace_bytes(1 << 14, 8, 1024) == 0
     assert moe.moe_permute_workspace_bytes(1 << 18, 8, 4096) == 0
-    # above: 2^21 slots = 4096 chunks of 512, times 384 experts, int32
-    assert moe.moe_permute_workspace_bytes(1 << 18, 8, 384) == 4096 * 384 * 4
-    assert moe.moe_permute_workspace_bytes((1 << 18) + 1, 8, 100) % 256 == 0
+    # above: 65536 tokens x 8 slots = 1024 chunks of 512, times 384 experts, int32
+    assert moe.moe_permute_workspace_bytes(65536, 8, 384) == 1024 * 384 * 4
+    assert moe.moe_permute_workspace_bytes((1 << 14) + 1, 8, 100) % 256 == 0
 
 
 P = ctypes.c_void_p

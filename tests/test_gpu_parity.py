@@ -129,21 +129,25 @@ def _routing_case(name):
         ids = rng.integers(0, 3000, size=(5000, 4)).astype(np.int32)
         ids[::3, 1] = 2999
         return ids, 3000
-    if name == "cluster_max":  # exactly 2^20 slots: the cluster kernel's largest table
-        return rng.integers(0, 384, size=(131072, 8)).astype(np.int32), 384
-    if name == "coop_e64":  # above 2^20 slots: the cooperative kernel and its workspace
+    if name == "cluster_max":  # exactly 2^17 slots: the cluster kernel's largest table
+        return rng.integers(0, 384, size=(16384, 8)).astype(np.int32), 384
+    if name == "coop_min":  # one slot more: the cooperative kernel
+        return rng.integers(0, 384, size=(16385, 8)).astype(np.int32)[:, :8], 384
+    if name == "coop_e64":  # the cooperative kernel and its workspace at 1.57 M slots
         return rng.integers(0, 64, size=(262147, 6)).astype(np.int32), 64
     if name == "coop_e1024":
         return rng.integers(0, 1024, size=(135001, 8)).astype(np.int32), 1024
+    if name == "e4096_large":  # E > 1024 above 2^17 slots: still the cluster kernel
+        return rng.integers(0, 4096, size=(40000, 4)).astype(np.int32), 4096
     raise KeyError(name)
 
 
 @pytest.mark.parametrize("name", ["one_expert_k1", "empty_experts", "duplicates", "ragged", "e_max",
                                   "many_chunks", "e4096", "e65535", "e3000_hot", "cluster_max",
-                                  "coop_e64", "coop_e1024"])
+                                  "coop_min", "coop_e64", "coop_e1024", "e4096_large"])
 def test_permute_edge_cases(cuda_device, name):
     """Metadata and rows bit-exact against the oracle: edge routings, E up to 65535 (the
-    cluster kernel's expert windows), and tables on both sides of 2^20 slots (the cluster
+    cluster kernel's expert windows), and tables on both sides of 2^17 slots (the cluster
     kernel without workspace, the cooperative kernel with one)."""
     ids_np, E = _routing_case(name)
     S, K = ids_np.shape

@@ -44,11 +44,11 @@ def _call(fn_name, x, ids, E, o, workspace=None):
 
 @pytest.mark.parametrize("S,K,E,H", [(262147, 6, 64, 64), (4096, 6, 64, 2048)])
 def test_no_alloc_permute_matches_workspace_permute_twice(cuda_device, S, K, E, H):
-    """Above 2^20 routed slots the permutation keeps per-chunk counts in its scratch (the
-    library's array here, a caller workspace for moe_permute); up to 2^20 it needs none."""
+    """Above 2^17 routed slots the permutation keeps per-chunk counts in its scratch (the
+    library's array here, a caller workspace for moe_permute); up to 2^17 it needs none."""
     dev = cuda_device
     need = moe.moe_permute_workspace_bytes(S, K, E)
-    assert (need > 0) == (S * K > (1 << 20)) and need <= moe.MOE_NO_ALLOC_SCRATCH_BYTES
+    assert (need > 0) == (S * K > (1 << 17)) and need <= moe.MOE_NO_ALLOC_SCRATCH_BYTES
     x = synth.normal_bf16_into(torch.empty(S, H, dtype=torch.bfloat16, device=dev), 1, synth.TAG_X)
     routings = [synth.route_es(1, S, K, E)[0],
                 synth.route_es(5, S, K, E, hot_e=E - 1, w_hot=20.0)[0]]
