@@ -127,7 +127,8 @@ moe_status moe_permute(const void* x, const int32_t* topk_ids, int64_t S, int64_
  * a fixed array inside this library's own device memory instead of from the caller.
  *
  *   - Limit: moe_permute_workspace_bytes(S, K, E) must be at most MOE_NO_ALLOC_SCRATCH_BYTES
- *     (4 MiB: e.g. S*K up to 524288 routed slots with E up to 1024); larger problems return
+ *     (4 MiB: every table of up to 2^17 routed slots, or with E > 1024, needs none; above
+ *     that e.g. S*K up to 524288 routed slots with E up to 1024); larger problems return
  *     MOE_ERR_UNSUPPORTED_SHAPE and launch nothing. Use moe_permute with a workspace then.
  *   - Every GPU that loads the library holds this array until the process exits.
  *   - The first call in each CUDA context looks up the array's device address (with the
