@@ -71,6 +71,7 @@ def parse_args():
 KERNEL_SOURCES = {
     # the files a kernel is compiled from: a recorded traffic figure holds only for them
     "up_gate": ["grouped_ffn.cu", "gemm_common.cuh", "ptx.cuh"],
+    "up_gate_zc": ["grouped_ffn.cu", "gemm_common.cuh", "ptx.cuh"],
     "weight_grad": ["grouped_ffn_bwd.cu", "gemm_common.cuh", "ptx.cuh"],
     "up_gate_mx": ["grouped_ffn_mx.cu", "gemm_common.cuh", "ptx.cuh"],
 }
@@ -135,12 +136,15 @@ def work_model(w, counts=None):
     active = E if counts is None else int((counts > 0).sum())
     m = {
         "permute_bytes": 2 * (S + M) * H + 12 * M + 8 * E,
+        "permute_meta_bytes": 12 * M + 8 * E,  # metadata only (zero copy): ids in, maps out
         "combine_bytes": 2 * (M + S) * H + 8 * M,
         "active_experts": active,
     }
     if not w.identity_ffn:
         m["up_gate_flops"] = 4 * M * H * Hp
         m["up_gate_bytes"] = 2 * 2 * active * H * Hp + 2 * M * H + 2 * M * Hp
+        # zero copy: the token rows come from x itself (each token's row at least once)
+        m["up_gate_zc_bytes"] = 2 * 2 * active * H * Hp + 2 * S * H + 2 * M * Hp
         m["down_flops"] = 2 * M * H * Hp
         m["down_bytes"] = 2 * active * Hp * H + 2 * M * Hp + 2 * M * H
         # backward (weights read once per pass; fp32 weight gradients written once)
@@ -641,7 +645,8 @@ def run_ours(args):
         wm = work_model(dataclasses.replace(w, E=E, K=K), counts)
         stages = {
             "permute": {"ms": mean["permute"],
-                        "GB/s": wm["permute_mx_bytes" if mx else "permute_bytes"]
+                        "GB/s": wm["permute_mx_bytes" if mx else
+                                   ("permute_meta_bytes" if zero_copy else "permute_bytes")]
                         / (mean["permute"] / 1e3) / 1e9},
             "combine": {"ms": mean["combine"],
                         "GB/s": wm["combine_bytes"] / (mean["combine"] / 1e3) / 1e9},
@@ -656,9 +661,11 @@ def run_ours(args):
                 "TFLOP/s": (wm["up_gate_flops"] + wm["down_flops"]) / (mean["ffn"] / 1e3) / 1e12}
             # dominant kernel: the SwiGLU (up/gate) pass
             flops, t_s = wm["up_gate_flops"], mean["up_gate"] / 1e3
-            byts = wm["up_gate_mx_bytes" if mx else "up_gate_bytes"]
+            byts = wm["up_gate_mx_bytes" if mx else
+                      ("up_gate_zc_bytes" if zero_copy else "up_gate_bytes")]
             kname = ("grouped_ffn_mx_kernel<true> (MXFP8 up/gate + SwiGLU + h quantisation)" if mx
-                     else "grouped_ffn_kernel<0> (up/gate + SwiGLU)")
+                     else "grouped_ffn_kernel<3> (zero-copy up/gate + SwiGLU, gathered rows)"
+                     if zero_copy else "grouped_ffn_kernel<0> (up/gate + SwiGLU)")
             # MXFP8: the measured bf16 peak times the nominal fp8:bf16 ratio (4.5 / 2.25)
             tpeak = peaks["bf16_tflops"] * (2.0 if mx else 1.0)
             ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -676,8 +683,8 @@ def run_ours(args):
         roof["peak_source"] = f"{peak_src} (burst)"
         if mx and roof["bound"] == "tensor":
             roof["peak_source"] = f"{peak_src} bf16 (burst) x 2, the nominal fp8:bf16 ratio"
-        roof["traffic"] = (profiled_traffic(f"{'up_gate_mx' if mx else 'up_gate'}/{w.name}")
-                           if not w.identity_ffn else None)
+        kind = "up_gate_mx" if mx else ("up_gate_zc" if zero_copy else "up_gate")
+        roof["traffic"] = (profiled_traffic(f"{kind}/{w.name}") if not w.identity_ffn else None)
         line = {
             "metric": METRIC, "value": job_throughput(w.S, world, ms_step), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,

@@ -322,7 +322,9 @@ __global__ void __launch_bounds__(Cfg<kMode>::kBlock, 1)
   } else {
     // Epilogue: warps 2..9 in two groups of four (warps 2-5 and 6-9); group g drains the
     // 32-token chunks c with (c / 32) % 2 == g. Warp w reads TMEM lanes 32*(w%4) .. +31, i.e.
-    // 32 of the unit's 128 features, and within a group the four warps cover all 128.
+    // 32 of the unit's 128 features, and within a group the four warps cover all 128. A warp
+    // releases the accumulator as soon as its last chunk of the unit is in registers, so the
+    // next unit's MMAs overlap that chunk's SwiGLU, conversion and stores.
     const int q = warp & 3;
     const int grp = (warp - 2) >> 2;
     const int f_local = q * 32 + lane;
@@ -341,11 +343,14 @@ __global__ void __launch_bounds__(Cfg<kMode>::kBlock, 1)
       tc_fence_after();
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + astage * kAccCols;
+      bool released = false;
+      const int nhalf = (kMode == kPair && U.fb * C::kFeatPerUnit + kBM < args.n_feat) ? 2 : 1;
       for (int c = grp * kOutChunk; c < U.nrows; c += kEpiGroups * kOutChunk) {
+        const bool last_chunk = c + kEpiGroups * kOutChunk >= U.nrows;
         // kPair: two 128-feature halves per chunk; otherwise one
-        for (int half = 0; half < (kMode == kPair ? 2 : 1); ++half) {
+        for (int half = 0; half < nhalf; ++half) {
           const int f0 = U.fb * C::kFeatPerUnit + half * kBM;
-          if (f0 >= args.n_feat) break;  // uniform across the group
+          const bool last = last_chunk && half == nhalf - 1;
           __syncwarp();  // tcgen05.ld is .sync.aligned: whole warp, converged
           // staged chunk [32 tokens][128 features] -> rows of dst (row stride n_feat)
           auto store_chunk = [&](__nv_bfloat16* dst_base) {
@@ -370,6 +375,12 @@ __global__ void __launch_bounds__(Cfg<kMode>::kBlock, 1)
           if (C::kSwi) {
             tmem_ld_32x32b_x32(tbase + C::kUpOff + c, r1);
             tmem_ld_wait();
+            if (last) {  // the unit's accumulator is all in registers: release it
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[astage]);
+              released = true;
+            }
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               // silu(g) * u = g / (1 + e^-g) * u (fast exp and divide; the result is rounded
@@ -380,6 +391,12 @@ __global__ void __launch_bounds__(Cfg<kMode>::kBlock, 1)
             }
           } else {
             tmem_ld_wait();
+            if (last) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[astage]);
+              released = true;
+            }
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               so[j * kBM + f_local] = __float2bfloat16_rn(__uint_as_float(r0[j]));
@@ -398,9 +415,11 @@ __global__ void __launch_bounds__(Cfg<kMode>::kBlock, 1)
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[astage]);
+      if (!released) {  // this group had no chunk of the unit
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[astage]);
+      }
       if (++astage == C::kAccStages) {
         astage = 0;
         aphase ^= 1u;

@@ -429,6 +429,16 @@ __global__ void __launch_bounds__(MxCfg<kSwi>::kBlock, 1)
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + astage * kMxAccCols;
       const int f0 = U.fb * kBM;
+      bool released = false;
+      // release the accumulator once this warp's last chunk of the unit is in registers
+      auto release_if_last = [&](int c) {
+        if (c + kEpiGroups * kOutChunk >= U.nrows) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[astage]);
+          released = true;
+        }
+      };
       for (int c = grp * kOutChunk; c < U.nrows; c += kEpiGroups * kOutChunk) {
         __syncwarp();
         uint32_t r0[32];
@@ -437,6 +447,7 @@ __global__ void __launch_bounds__(MxCfg<kSwi>::kBlock, 1)
           uint32_t r1[32];
           tmem_ld_32x32b_x32(tbase + kMxAccCols + c, r1);
           tmem_ld_wait();
+          release_if_last(c);
           uint32_t my_sf = 127;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -467,6 +478,7 @@ __global__ void __launch_bounds__(MxCfg<kSwi>::kBlock, 1)
           named_bar_sync(bar_grp, 128);
         } else {
           tmem_ld_wait();
+          release_if_last(c);
           __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(so_bytes);
 #pragma unroll
           for (int j = 0; j < 32; ++j) so[j * kBM + f_local] = __float2bfloat16_rn(__uint_as_float(r0[j]));
@@ -486,9 +498,11 @@ __global__ void __launch_bounds__(MxCfg<kSwi>::kBlock, 1)
           named_bar_sync(bar_grp, 128);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[astage]);
+      if (!released) {  // this group had no chunk of the unit
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[astage]);
+      }
       if (++astage == C::kAccStages) {
         astage = 0;
         aphase ^= 1u;
