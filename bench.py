@@ -603,39 +603,68 @@ def run_ours(args):
                     else cpu_baseline(w, inp, args.cpu_seconds))
 
     # flat in maxvio: the same step on the full-size geometry's skewed routings (maxvio 1, 10
-    # and 20), each workload's inputs made afresh (the previous ones freed first)
+    # and 20: each workload's own topk ids, route weights and x; the full-size layer's weights,
+    # whose values do not change the work), timed interleaved with the default routing -- one
+    # step per routing per round, the starting routing rotating from round to round, L2
+    # flushed before every step -- so that clock and power drift over the run reaches all
+    # four alike
     sweep = None
     if (w.name == "large" and not (mx or ns or zero_copy) and not args.no_sweep):
-        sweep = {"large": {"ms_per_step": ms_step, "maxvio_measured": maxvio,
-                           "tokens_per_s": job_throughput(w.S, world, ms_step)}}
-        for sname in ("skew1", "skew10", "skew20"):
+        names = ("large", "skew1", "skew10", "skew20")
+        base_inp = inp
+        variants = {"large": base_inp}
+        for sname in names[1:]:
             sw = synth.WORKLOADS[sname]
-            inp = None
-            torch.cuda.empty_cache()
-            inp = synth.make_layer_inputs(sw, device=str(dev))
+            ids_np, rw_np = synth.routing_for(sw)
+            v = dict(base_inp)
+            v["topk_ids"] = torch.from_numpy(ids_np).to(dev)
+            v["route_w"] = torch.from_numpy(rw_np).to(dev)
+            v["x"] = synth.normal_bf16_into(torch.empty(sw.S, sw.H, dtype=torch.bfloat16,
+                                                        device=dev), sw.seed, synth.TAG_X)
+            variants[sname] = v
+
+        def use(name):
+            nonlocal inp, ids_step, w_step
+            inp = variants[name]
             ids_step, w_step = inp["topk_ids"], inp["route_w"]
+
+        mv_of = {}
+        for name in names:  # warm-up, and each routing's measured maxvio
+            use(name)
             for _ in range(args.warmup):
                 flush()
                 step()
-            swevs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
-                     for _ in range(args.steps)]
-            if world > 1:
-                dist.barrier()
             torch.cuda.synchronize()
-            for i in range(args.steps):
+            mv_of[name] = float(buf.maxvio.item())
+        swevs = {n: [] for n in names}
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            for j in range(len(names)):
+                name = names[(i + j) % len(names)]
+                use(name)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 flush(i)
-                swevs[i][0].record()
+                e0.record()
                 step()
-                swevs[i][1].record()
-            torch.cuda.synchronize()
-            if int(buf.d_status.item()) != 0:
-                raise RuntimeError(f"device status {int(buf.d_status.item())} in {sname}")
-            sms = reduce_step_time(sum(e[0].elapsed_time(e[1]) for e in swevs) / args.steps,
+                e1.record()
+                swevs[name].append((e0, e1))
+        torch.cuda.synchronize()
+        if int(buf.d_status.item()) != 0:
+            raise RuntimeError(f"device status {int(buf.d_status.item())} in the maxvio sweep")
+        use("large")
+        inp = base_inp
+        sweep = {"method": "interleaved: one step per routing per round, rotating order, L2 "
+                           "flushed before each step; skewed routings on the same weights"}
+        for name in names:
+            sms = reduce_step_time(sum(a.elapsed_time(b) for a, b in swevs[name]) / args.steps,
                                    world, dev)
-            sweep[sname] = {"ms_per_step": sms, "maxvio_measured": float(buf.maxvio.item()),
-                            "tokens_per_s": job_throughput(sw.S, world, sms)}
-        t_all = [v["ms_per_step"] for v in sweep.values()]
+            sweep[name] = {"ms_per_step": sms, "maxvio_measured": mv_of[name],
+                           "tokens_per_s": job_throughput(w.S, world, sms)}
+        t_all = [sweep[n]["ms_per_step"] for n in names]
         sweep["spread"] = (max(t_all) - min(t_all)) / min(t_all)
+        variants = None
 
     if clocks is not None:
         clocks.stop()
@@ -684,7 +713,9 @@ def run_ours(args):
         if mx and roof["bound"] == "tensor":
             roof["peak_source"] = f"{peak_src} bf16 (burst) x 2, the nominal fp8:bf16 ratio"
         kind = "up_gate_mx" if mx else ("up_gate_zc" if zero_copy else "up_gate")
-        roof["traffic"] = (profiled_traffic(f"{kind}/{w.name}") if not w.identity_ffn else None)
+        # a capture holds for its own workload only (shared experts change the launch)
+        roof["traffic"] = (profiled_traffic(f"{kind}/{w.name}")
+                           if not (w.identity_ffn or ns) else None)
         line = {
             "metric": METRIC, "value": job_throughput(w.S, world, ms_step), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
