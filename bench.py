@@ -688,6 +688,18 @@ def run_ours(args):
             stages["grouped_ffn"] = {
                 "ms": mean["ffn"],
                 "TFLOP/s": (wm["up_gate_flops"] + wm["down_flops"]) / (mean["ffn"] / 1e3) / 1e12}
+            # both fractions of each GEMM pass: of the tensor peak (for its dtype) and of HBM
+            tpk = peaks["bf16_tflops"] * (2.0 if mx else 1.0)
+            ug_b = wm["up_gate_mx_bytes" if mx else
+                      ("up_gate_zc_bytes" if zero_copy else "up_gate_bytes")]
+            dn_b = wm["down_mx_bytes" if mx else "down_bytes"]
+            for key, byts in (("up_gate", ug_b), ("down", dn_b), ("grouped_ffn", ug_b + dn_b)):
+                st = stages[key]
+                st["GB/s"] = byts / (st["ms"] / 1e3) / 1e9
+                st["frac_tensor"] = st["TFLOP/s"] / tpk
+                st["frac_hbm"] = st["GB/s"] / peaks["hbm_gbs"]
+        for key in ("permute", "combine"):
+            stages[key]["frac_hbm"] = stages[key]["GB/s"] / peaks["hbm_gbs"]
             # dominant kernel: the SwiGLU (up/gate) pass
             flops, t_s = wm["up_gate_flops"], mean["up_gate"] / 1e3
             byts = wm["up_gate_mx_bytes" if mx else
