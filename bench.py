@@ -164,6 +164,71 @@ def work_model(w, counts=None):
     return m
 
 
+def stage_report(w, E, K, counts, mean, peaks, peak_src, mx=False, zero_copy=False,
+                 shared=False):
+    """Per-stage throughput and fractions of the measured peaks, and the roofline of the
+    dominant kernel (the SwiGLU pass; the permutation for identity-expert workloads).
+    mean: stage times in ms ("permute", "up_gate", "down", "ffn", "combine")."""
+    wm = work_model(dataclasses.replace(w, E=E, K=K), counts)
+    stages = {
+        "permute": {"ms": mean["permute"],
+                    "GB/s": wm["permute_mx_bytes" if mx else
+                               ("permute_meta_bytes" if zero_copy else "permute_bytes")]
+                    / (mean["permute"] / 1e3) / 1e9},
+        "combine": {"ms": mean["combine"],
+                    "GB/s": wm["combine_bytes"] / (mean["combine"] / 1e3) / 1e9},
+    }
+    if not w.identity_ffn:
+        stages["up_gate"] = {"ms": mean["up_gate"],
+                             "TFLOP/s": wm["up_gate_flops"] / (mean["up_gate"] / 1e3) / 1e12}
+        stages["down"] = {"ms": mean["down"],
+                          "TFLOP/s": wm["down_flops"] / (mean["down"] / 1e3) / 1e12}
+        stages["grouped_ffn"] = {
+            "ms": mean["ffn"],
+            "TFLOP/s": (wm["up_gate_flops"] + wm["down_flops"]) / (mean["ffn"] / 1e3) / 1e12}
+        # both fractions of each GEMM pass: of the tensor peak (for its dtype) and of HBM
+        tpk = peaks["bf16_tflops"] * (2.0 if mx else 1.0)
+        ug_b = wm["up_gate_mx_bytes" if mx else
+                  ("up_gate_zc_bytes" if zero_copy else "up_gate_bytes")]
+        dn_b = wm["down_mx_bytes" if mx else "down_bytes"]
+        for key, byts in (("up_gate", ug_b), ("down", dn_b), ("grouped_ffn", ug_b + dn_b)):
+            st = stages[key]
+            st["GB/s"] = byts / (st["ms"] / 1e3) / 1e9
+            st["frac_tensor"] = st["TFLOP/s"] / tpk
+            st["frac_hbm"] = st["GB/s"] / peaks["hbm_gbs"]
+        # dominant kernel: the SwiGLU (up/gate) pass
+        flops, t_s = wm["up_gate_flops"], mean["up_gate"] / 1e3
+        byts = wm["up_gate_mx_bytes" if mx else
+                  ("up_gate_zc_bytes" if zero_copy else "up_gate_bytes")]
+        kname = ("grouped_ffn_mx_kernel<true> (MXFP8 up/gate + SwiGLU + h quantisation)" if mx
+                 else "grouped_ffn_kernel<3> (zero-copy up/gate + SwiGLU, gathered rows)"
+                 if zero_copy else "grouped_ffn_kernel<0> (up/gate + SwiGLU)")
+        # MXFP8: the measured bf16 peak times the nominal fp8:bf16 ratio (4.5 / 2.25)
+        tpeak = peaks["bf16_tflops"] * (2.0 if mx else 1.0)
+        ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        if flops / byts >= ridge:
+            roof = {"kernel": kname, "bound": "tensor", "achieved": flops / t_s / 1e12,
+                    "peak": tpeak, "unit": "TFLOP/s"}
+        else:
+            roof = {"kernel": kname, "bound": "hbm", "achieved": byts / t_s / 1e9,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        byts, t_s = wm["permute_bytes"], mean["permute"] / 1e3
+        roof = {"kernel": "moe_permute (2 kernels)", "bound": "hbm", "achieved": byts / t_s / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    for key in ("permute", "combine"):
+        stages[key]["frac_hbm"] = stages[key]["GB/s"] / peaks["hbm_gbs"]
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = f"{peak_src} (burst)"
+    if mx and roof["bound"] == "tensor":
+        roof["peak_source"] = f"{peak_src} bf16 (burst) x 2, the nominal fp8:bf16 ratio"
+    kind = "up_gate_mx" if mx else ("up_gate_zc" if zero_copy else "up_gate")
+    # a capture holds for its own workload only (shared experts change the launch)
+    roof["traffic"] = (profiled_traffic(f"{kind}/{w.name}")
+                       if not (w.identity_ffn or shared) else None)
+    return stages, roof
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -671,63 +736,8 @@ def run_ours(args):
 
     if rank == 0:
         peaks, peak_src = load_peaks()
-        wm = work_model(dataclasses.replace(w, E=E, K=K), counts)
-        stages = {
-            "permute": {"ms": mean["permute"],
-                        "GB/s": wm["permute_mx_bytes" if mx else
-                                   ("permute_meta_bytes" if zero_copy else "permute_bytes")]
-                        / (mean["permute"] / 1e3) / 1e9},
-            "combine": {"ms": mean["combine"],
-                        "GB/s": wm["combine_bytes"] / (mean["combine"] / 1e3) / 1e9},
-        }
-        if not w.identity_ffn:
-            stages["up_gate"] = {"ms": mean["up_gate"],
-                                 "TFLOP/s": wm["up_gate_flops"] / (mean["up_gate"] / 1e3) / 1e12}
-            stages["down"] = {"ms": mean["down"],
-                              "TFLOP/s": wm["down_flops"] / (mean["down"] / 1e3) / 1e12}
-            stages["grouped_ffn"] = {
-                "ms": mean["ffn"],
-                "TFLOP/s": (wm["up_gate_flops"] + wm["down_flops"]) / (mean["ffn"] / 1e3) / 1e12}
-            # both fractions of each GEMM pass: of the tensor peak (for its dtype) and of HBM
-            tpk = peaks["bf16_tflops"] * (2.0 if mx else 1.0)
-            ug_b = wm["up_gate_mx_bytes" if mx else
-                      ("up_gate_zc_bytes" if zero_copy else "up_gate_bytes")]
-            dn_b = wm["down_mx_bytes" if mx else "down_bytes"]
-            for key, byts in (("up_gate", ug_b), ("down", dn_b), ("grouped_ffn", ug_b + dn_b)):
-                st = stages[key]
-                st["GB/s"] = byts / (st["ms"] / 1e3) / 1e9
-                st["frac_tensor"] = st["TFLOP/s"] / tpk
-                st["frac_hbm"] = st["GB/s"] / peaks["hbm_gbs"]
-        for key in ("permute", "combine"):
-            stages[key]["frac_hbm"] = stages[key]["GB/s"] / peaks["hbm_gbs"]
-            # dominant kernel: the SwiGLU (up/gate) pass
-            flops, t_s = wm["up_gate_flops"], mean["up_gate"] / 1e3
-            byts = wm["up_gate_mx_bytes" if mx else
-                      ("up_gate_zc_bytes" if zero_copy else "up_gate_bytes")]
-            kname = ("grouped_ffn_mx_kernel<true> (MXFP8 up/gate + SwiGLU + h quantisation)" if mx
-                     else "grouped_ffn_kernel<3> (zero-copy up/gate + SwiGLU, gathered rows)"
-                     if zero_copy else "grouped_ffn_kernel<0> (up/gate + SwiGLU)")
-            # MXFP8: the measured bf16 peak times the nominal fp8:bf16 ratio (4.5 / 2.25)
-            tpeak = peaks["bf16_tflops"] * (2.0 if mx else 1.0)
-            ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)
-            if flops / byts >= ridge:
-                roof = {"kernel": kname, "bound": "tensor", "achieved": flops / t_s / 1e12,
-                        "peak": tpeak, "unit": "TFLOP/s"}
-            else:
-                roof = {"kernel": kname, "bound": "hbm", "achieved": byts / t_s / 1e9,
-                        "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-        else:
-            byts, t_s = wm["permute_bytes"], mean["permute"] / 1e3
-            roof = {"kernel": "moe_permute (2 kernels)", "bound": "hbm", "achieved": byts / t_s / 1e9,
-                    "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-        roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["peak_source"] = f"{peak_src} (burst)"
-        if mx and roof["bound"] == "tensor":
-            roof["peak_source"] = f"{peak_src} bf16 (burst) x 2, the nominal fp8:bf16 ratio"
-        kind = "up_gate_mx" if mx else ("up_gate_zc" if zero_copy else "up_gate")
-        # a capture holds for its own workload only (shared experts change the launch)
-        roof["traffic"] = (profiled_traffic(f"{kind}/{w.name}")
-                           if not (w.identity_ffn or ns) else None)
+        stages, roof = stage_report(w, E, K, counts, mean, peaks, peak_src, mx=mx,
+                                    zero_copy=zero_copy, shared=bool(ns))
         line = {
             "metric": METRIC, "value": job_throughput(w.S, world, ms_step), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
