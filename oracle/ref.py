@@ -1,0 +1,117 @@
+"""ctypes loader of the plain C++ oracle (moe_oracle_ref.cpp) and numpy-facing wrappers.
+
+TEST INFRASTRUCTURE ONLY, like moe_oracle.py: tests/ use it to cross-check the numpy
+oracle; `build()` compiles it with g++ next to its source (the library is not part of the
+product and is never loaded by it).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "moe_oracle_ref.cpp")
+LIB = os.path.join(HERE, "libmoe_oracle_ref.so")
+
+_lib = None
+
+
+def build(verbose: bool = False) -> str:
+    """Compile the oracle with g++ (no floating-point contraction: every product and sum is
+    rounded as written)."""
+    cmd = ["g++", "-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-shared",
+           "-fPIC", SRC, "-o", LIB]
+    if verbose:
+        print(" ".join(cmd))
+    subprocess.run(cmd, check=True)
+    return LIB
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+            build()
+        L = ctypes.CDLL(LIB)
+        P = ctypes.c_void_p
+        i64, i32 = ctypes.c_int64, ctypes.c_int32
+        L.ref_round_bf16.argtypes = [P, i64, P]
+        L.ref_round_bf16.restype = None
+        L.ref_permute.argtypes = [P, i64, i32, i32, P, P, P, P]
+        L.ref_permute.restype = ctypes.c_int
+        L.ref_permute_rows.argtypes = [P, P, i64, i32, i64, P]
+        L.ref_permute_rows.restype = None
+        L.ref_maxvio.argtypes = [P, i32, i64, i32, P]
+        L.ref_maxvio.restype = ctypes.c_double
+        L.ref_grouped_ffn.argtypes = [P, P, P, P, P, i32, i64, i64, P, P]
+        L.ref_grouped_ffn.restype = None
+        L.ref_combine.argtypes = [P, P, P, i64, i32, i64, P]
+        L.ref_combine.restype = None
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def round_bf16(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    lib().ref_round_bf16(_p(v), v.size, _p(out))
+    return out
+
+
+def permute(topk_ids, E: int):
+    """(counts, cu_seqlens, row_id_map, perm_src); ValueError on an id outside [0, E)."""
+    ids = np.ascontiguousarray(topk_ids, dtype=np.int32)
+    S, K = ids.shape
+    counts = np.empty(E, np.int32)
+    cu = np.empty(E + 1, np.int32)
+    rmap = np.empty(S * K, np.int32)
+    psrc = np.empty(S * K, np.int32)
+    if lib().ref_permute(_p(ids), S, K, E, _p(counts), _p(cu), _p(rmap), _p(psrc)) != 0:
+        raise ValueError("expert id outside [0, E)")
+    return counts, cu, rmap, psrc
+
+
+def permute_rows(x_bits, perm_src, K: int) -> np.ndarray:
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    ps = np.ascontiguousarray(perm_src, dtype=np.int32)
+    out = np.empty((ps.size, x.shape[1]), np.uint16)
+    lib().ref_permute_rows(_p(x), _p(ps), ps.size, K, x.shape[1], _p(out))
+    return out
+
+
+def maxvio(counts, S: int, K: int):
+    c = np.ascontiguousarray(counts, dtype=np.int32)
+    mc = np.zeros(1, np.int32)
+    v = lib().ref_maxvio(_p(c), c.size, S, K, _p(mc))
+    return v, int(mc[0])
+
+
+def grouped_ffn(x_perm_bits, cu_seqlens, w_gate, w_up, w_down):
+    """(h bits [M,Hp], y bits [M,H]); weights [E,H,Hp], [E,H,Hp], [E,Hp,H] as bf16 bits."""
+    x = np.ascontiguousarray(x_perm_bits, dtype=np.uint16)
+    wg = np.ascontiguousarray(w_gate, dtype=np.uint16)
+    wu = np.ascontiguousarray(w_up, dtype=np.uint16)
+    wd = np.ascontiguousarray(w_down, dtype=np.uint16)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    M, H = x.shape
+    E, _, Hp = wg.shape
+    h = np.zeros((M, Hp), np.uint16)
+    y = np.zeros((M, H), np.uint16)
+    lib().ref_grouped_ffn(_p(x), _p(wg), _p(wu), _p(wd), _p(cu), E, H, Hp, _p(h), _p(y))
+    return h, y
+
+
+def combine(y_bits, row_id_map, route_w, S: int, K: int) -> np.ndarray:
+    y = np.ascontiguousarray(y_bits, dtype=np.uint16)
+    rm = np.ascontiguousarray(row_id_map, dtype=np.int32)
+    w = np.ascontiguousarray(route_w, dtype=np.float32)
+    out = np.empty((S, y.shape[1]), np.uint16)
+    lib().ref_combine(_p(y), _p(rm), _p(w), S, K, y.shape[1], _p(out))
+    return out
