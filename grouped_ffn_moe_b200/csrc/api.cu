@@ -184,10 +184,11 @@ moe_status moe_grouped_ffn_up_gate(const void* x_perm, const void* w_gate, const
                                    void* cuda_stream) {
   const moe_status st = check_ffn_shapes(M, H, Hp, E);
   if (st != MOE_OK) return st;
+  // no rows: nothing is read or written (row buffers may be NULL)
+  if (M == 0) return MOE_OK;
   if (!ok_ptr16(x_perm) || !ok_ptr16(w_gate) || !ok_ptr16(w_up) || !ok_ptr16(h_scratch) ||
       cu_seqlens == nullptr || !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARGUMENT;
-  if (M == 0) return MOE_OK;
   return moe::launch_ffn_pass(true, x_perm, w_gate, w_up, cu_seqlens, M, H, Hp, E, h_scratch,
                               nullptr, nullptr, d_status, static_cast<cudaStream_t>(cuda_stream));
 }
@@ -197,10 +198,10 @@ moe_status moe_grouped_ffn_down(const void* h_scratch, const void* w_down,
                                 int32_t E, void* y, int32_t* d_status, void* cuda_stream) {
   const moe_status st = check_ffn_shapes(M, H, Hp, E);
   if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
   if (!ok_ptr16(h_scratch) || !ok_ptr16(w_down) || !ok_ptr16(y) || cu_seqlens == nullptr ||
       !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARGUMENT;
-  if (M == 0) return MOE_OK;
   return moe::launch_ffn_pass(false, h_scratch, w_down, nullptr, cu_seqlens, M, H, Hp, E, y,
                               nullptr, nullptr, d_status, static_cast<cudaStream_t>(cuda_stream));
 }
@@ -211,12 +212,12 @@ moe_status moe_grouped_ffn(const void* x_perm, const void* w_gate, const void* w
                            void* cuda_stream) {
   const moe_status st = check_ffn_shapes(M, H, Hp, E);
   if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
   // validate both passes before launching either
   if (!ok_ptr16(x_perm) || !ok_ptr16(w_gate) || !ok_ptr16(w_up) || !ok_ptr16(w_down) ||
       !ok_ptr16(h_scratch) || !ok_ptr16(y) || cu_seqlens == nullptr || !aligned(cu_seqlens, 4) ||
       !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARGUMENT;
-  if (M == 0) return MOE_OK;
   const moe_status s1 = moe_grouped_ffn_up_gate(x_perm, w_gate, w_up, cu_seqlens, M, H, Hp, E,
                                                 h_scratch, d_status, cuda_stream);
   if (s1 != MOE_OK) return s1;
@@ -234,13 +235,13 @@ moe_status moe_grouped_ffn_up_gate_gather(const void* x, const int32_t* perm_src
   const int64_t M = S * K;
   const moe_status st = check_ffn_shapes(M, H, Hp, E);
   if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
   if ((gate_pre == nullptr) != (up_pre == nullptr)) return MOE_ERR_INVALID_ARGUMENT;
   if (!ok_ptr16(x) || perm_src == nullptr || !aligned(perm_src, 4) || !ok_ptr16(w_gate) ||
       !ok_ptr16(w_up) || !ok_ptr16(h_scratch) || !aligned(gate_pre, 16) ||
       !aligned(up_pre, 16) || cu_seqlens == nullptr || !aligned(cu_seqlens, 4) ||
       !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARGUMENT;
-  if (M == 0) return MOE_OK;
   return moe::launch_ffn_up_gate_gather(x, perm_src, S, K, w_gate, w_up, cu_seqlens, M, H, Hp, E,
                                         h_scratch, gate_pre, up_pre, d_status,
                                         static_cast<cudaStream_t>(cuda_stream));
@@ -256,12 +257,12 @@ moe_status moe_grouped_ffn_gather(const void* x, const int32_t* perm_src, int64_
   const int64_t M = S * K;
   const moe_status st = check_ffn_shapes(M, H, Hp, E);
   if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
   // validate both passes before launching either
   if (!ok_ptr16(x) || perm_src == nullptr || !aligned(perm_src, 4) || !ok_ptr16(w_gate) ||
       !ok_ptr16(w_up) || !ok_ptr16(w_down) || !ok_ptr16(h_scratch) || !ok_ptr16(y) ||
       cu_seqlens == nullptr || !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARGUMENT;
-  if (M == 0) return MOE_OK;
   const moe_status s1 =
       moe_grouped_ffn_up_gate_gather(x, perm_src, S, K, w_gate, w_up, cu_seqlens, H, Hp, E,
                                      h_scratch, nullptr, nullptr, d_status, cuda_stream);
@@ -277,11 +278,11 @@ moe_status moe_grouped_ffn_up_gate_train(const void* x_perm, const void* w_gate,
                                          void* cuda_stream) {
   const moe_status st = check_ffn_shapes(M, H, Hp, E);
   if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
   if (!ok_ptr16(x_perm) || !ok_ptr16(w_gate) || !ok_ptr16(w_up) || !ok_ptr16(h_scratch) ||
       !ok_ptr16(gate_pre) || !ok_ptr16(up_pre) || cu_seqlens == nullptr ||
       !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARGUMENT;
-  if (M == 0) return MOE_OK;
   return moe::launch_ffn_pass(true, x_perm, w_gate, w_up, cu_seqlens, M, H, Hp, E, h_scratch,
                               gate_pre, up_pre, d_status, static_cast<cudaStream_t>(cuda_stream));
 }
@@ -293,11 +294,11 @@ moe_status moe_grouped_ffn_down_backward(const void* grad_y, const void* w_down,
                                          int32_t* d_status, void* cuda_stream) {
   const moe_status st = check_ffn_shapes(M, H, Hp, E);
   if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
   if (!ok_ptr16(grad_y) || !ok_ptr16(w_down) || !ok_ptr16(gate_pre) || !ok_ptr16(up_pre) ||
       !ok_ptr16(d_gate) || !ok_ptr16(d_up) || cu_seqlens == nullptr || !aligned(cu_seqlens, 4) ||
       !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARGUMENT;
-  if (M == 0) return MOE_OK;
   return moe::launch_ffn_down_backward(grad_y, w_down, gate_pre, up_pre, cu_seqlens, M, H, Hp, E,
                                        d_gate, d_up, d_status,
                                        static_cast<cudaStream_t>(cuda_stream));
@@ -310,11 +311,11 @@ moe_status moe_grouped_ffn_up_gate_backward(const void* d_gate, const void* d_up
                                             int32_t* d_status, void* cuda_stream) {
   const moe_status st = check_ffn_shapes(M, H, Hp, E);
   if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
   if (!ok_ptr16(d_gate) || !ok_ptr16(d_up) || !ok_ptr16(w_gate) || !ok_ptr16(w_up) ||
       !ok_ptr16(grad_x_perm) || cu_seqlens == nullptr || !aligned(cu_seqlens, 4) ||
       !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARGUMENT;
-  if (M == 0) return MOE_OK;
   return moe::launch_ffn_up_gate_backward(d_gate, d_up, w_gate, w_up, cu_seqlens, M, H, Hp, E,
                                           grad_x_perm, d_status,
                                           static_cast<cudaStream_t>(cuda_stream));
@@ -484,11 +485,11 @@ moe_status moe_grouped_ffn_up_gate_mxfp8(const void* x_q, const void* x_sf, cons
                                          int32_t* d_status, void* cuda_stream) {
   const moe_status st = check_ffn_shapes(M, H, Hp, E);
   if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
   if (!ok_ptr16(x_q) || !ok_ptr16(x_sf) || !ok_ptr16(w_gate_q) || !ok_ptr16(w_gate_sf) ||
       !ok_ptr16(w_up_q) || !ok_ptr16(w_up_sf) || !ok_ptr16(h_q) || !ok_ptr16(h_sf) ||
       cu_seqlens == nullptr || !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARGUMENT;
-  if (M == 0) return MOE_OK;
   return moe::launch_mx_ffn_pass(true, x_q, x_sf, w_gate_q, w_gate_sf, w_up_q, w_up_sf,
                                  cu_seqlens, M, H, Hp, E, h_q, h_sf, d_status,
                                  static_cast<cudaStream_t>(cuda_stream));
@@ -500,10 +501,10 @@ moe_status moe_grouped_ffn_down_mxfp8(const void* h_q, const void* h_sf, const v
                                       void* cuda_stream) {
   const moe_status st = check_ffn_shapes(M, H, Hp, E);
   if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
   if (!ok_ptr16(h_q) || !ok_ptr16(h_sf) || !ok_ptr16(w_down_q) || !ok_ptr16(w_down_sf) ||
       !ok_ptr16(y) || cu_seqlens == nullptr || !aligned(cu_seqlens, 4) || !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARGUMENT;
-  if (M == 0) return MOE_OK;
   return moe::launch_mx_ffn_pass(false, h_q, h_sf, w_down_q, w_down_sf, nullptr, nullptr,
                                  cu_seqlens, M, H, Hp, E, y, nullptr, d_status,
                                  static_cast<cudaStream_t>(cuda_stream));
@@ -517,6 +518,7 @@ moe_status moe_grouped_ffn_mxfp8(const void* x_q, const void* x_sf, const void* 
                                  void* cuda_stream) {
   const moe_status st = check_ffn_shapes(M, H, Hp, E);
   if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
   if (!ok_ptr16(w_down_q) || !ok_ptr16(w_down_sf) || !ok_ptr16(y))
     return MOE_ERR_INVALID_ARGUMENT;
   const moe_status s1 = moe_grouped_ffn_up_gate_mxfp8(x_q, x_sf, w_gate_q, w_gate_sf, w_up_q,

@@ -41,7 +41,10 @@
  *   - Preconditions, checked on the host: pointers non-NULL and 16-byte aligned (unless
  *     documented nullable), H and Hp multiples of 8 (of 128 for the grouped FFN calls),
  *     1 <= K <= E <= MOE_MAX_EXPERTS (E <= MOE_MAX_FFN_EXPERTS for the grouped FFN calls),
- *     S*K < 2^31. S = 0 is a legal no-op.
+ *     S*K < 2^31. S = 0 (M = 0 rows) is legal: a call returns MOE_OK after its shape
+ *     checks, reads and writes no row buffer (those may then be NULL, as a zero-size
+ *     tensor's data pointer is), and only moe_permute's counts/offsets/maxvio and the
+ *     weight gradients (zero when writing) are produced.
  *   - Results are deterministic: no floating-point atomics; every sum has a fixed order.
  */
 #ifndef MOE_B200_H_

@@ -90,6 +90,18 @@ def test_host_validation_rejects_without_launch():
     assert L.moe_grouped_ffn(a, a, a, a, a, 16, 256, 200, 4, a, a, null, null) == 2
     assert L.moe_grouped_ffn(a, null, a, a, a, 16, 256, 256, 4, a, a, null, null) == 1
     assert L.moe_grouped_ffn(a, a, a, a, a, 0, 256, 256, 4, a, a, null, null) == 0  # M = 0: no-op
+    # M = 0 with NULL row buffers (a zero-size tensor's data pointer): still a no-op; shapes
+    # are still checked
+    assert L.moe_grouped_ffn(null, a, a, a, a, 0, 256, 256, 4, null, null, null, null) == 0
+    assert L.moe_grouped_ffn_up_gate_train(null, a, a, a, 0, 256, 256, 4, null, null, null,
+                                           null, null) == 0
+    assert L.moe_grouped_ffn_down_backward(null, a, null, null, a, 0, 256, 256, 4, null, null,
+                                           null, null) == 0
+    assert L.moe_grouped_ffn_up_gate_backward(null, null, a, a, a, 0, 256, 256, 4, null, null,
+                                              null) == 0
+    assert L.moe_grouped_ffn_gather(null, null, 0, 2, a, a, a, a, 256, 256, 4, null, null, null,
+                                    null) == 0
+    assert L.moe_grouped_ffn(null, a, a, a, a, 0, 256, 200, 4, null, null, null, null) == 2
     # combine: H % 8, K < 1
     assert L.moe_unpermute_combine(a, a, a, 4, 12, 2, a, null) == 2
     assert L.moe_unpermute_combine(a, a, a, 4, 16, 0, a, null) == 1

@@ -204,3 +204,45 @@ def test_layer_backward_end_to_end_tiny(cuda_device):
     print(f"[tiny] end-to-end relative errors: {checks}")
     for k, v in checks.items():
         assert v <= 1e-2, (k, v)
+
+
+def test_backward_wait_timeout_reports_status_and_keeps_context(cuda_device):
+    """Failure detection of the backward GEMMs without a fault: with a 1 ns wait budget every
+    pipeline wait of the dgrad and weight-gradient kernels runs out; they record
+    MOE_ERR_DEVICE_TIMEOUT in d_status, drain their own copies and MMAs, free TMEM and
+    return, and the CUDA context stays usable. (The forward, run first in the same child,
+    times out as well; its status is cleared before the backward.)"""
+    import os
+    import subprocess
+    import sys
+
+    script = (
+        "import torch, synth, grouped_ffn_moe_b200 as moe\n"
+        "dev = torch.device('cuda:0')\n"
+        "w = synth.WORKLOADS['tiny']\n"
+        "inp = synth.make_layer_inputs(w, device='cuda:0')\n"
+        "buf = moe.LayerBuffers.allocate(w.S, w.H, w.Hp, w.E, w.K, dev, train=True)\n"
+        "moe.moe_layer_forward(inp['x'], inp['topk_ids'], inp['route_w'], inp['w_gate'],"
+        " inp['w_up'], inp['w_down'], buf)\n"
+        "torch.cuda.synchronize()\n"
+        "buf.d_status.zero_()\n"
+        "grads = moe.LayerGrads.allocate(w.S, w.H, w.Hp, w.E, w.K, dev)\n"
+        "g = torch.ones(w.S, w.H, dtype=torch.bfloat16, device=dev)\n"
+        "moe.moe_layer_backward(g, inp['route_w'], inp['w_gate'], inp['w_up'], inp['w_down'],"
+        " buf, grads)\n"
+        "torch.cuda.synchronize()\n"
+        "st = int(buf.d_status.item())\n"
+        "assert st & moe.MOE_ERR_DEVICE_TIMEOUT, st\n"
+        "z = torch.arange(1000, device='cuda:0').sum().item()\n"
+        "assert z == 499500\n"
+        "print('timeout status', st)\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, PYTHONPATH=root, MOE_WAIT_BUDGET_NS="1")
+    r = subprocess.run([sys.executable, "-c", script], env=env, cwd=root, timeout=600,
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "timeout status" in r.stdout
+    # this process (normal budget) still runs the training step correctly
+    w, inp = _ragged_inputs(cuda_device, 256, 384, [3, 0, 17])
+    buf, grads, _ = _run_train(inp, w, cuda_device)
+    assert int(buf.d_status.item()) == 0

@@ -416,6 +416,44 @@ def test_layer_full_size_sampled(cuda_device, wname):
     print(f"[{w.name}] out (stage): {assert_close_bf16(out_gpu, out_stage, 'out stage (sampled)')}")
 
 
+def test_empty_batch_layer(cuda_device):
+    """S = 0 tokens ("Distributed expert parallelism", "Empty experts": every expert empty):
+    the forward (copy and zero-copy), the training backward and the MXFP8 forward are legal
+    no-ops on the data -- zero counts and offsets, d_status 0, nothing written outside the
+    buffers."""
+    dev = cuda_device
+    S, H, Hp, E, K = 0, 256, 512, 8, 2
+    gen = torch.Generator().manual_seed(5)
+    # zero-row views inside guarded allocations (non-null pointers, as a caller's would be)
+    x = GUARD((S, H), torch.bfloat16, dev)
+    ids = GUARD((S, K), torch.int32, dev)
+    rw = GUARD((S, K), torch.float32, dev)
+    wg = (torch.randn(E, H, Hp, generator=gen) / 16).to(torch.bfloat16).to(dev)
+    wu = (torch.randn(E, H, Hp, generator=gen) / 16).to(torch.bfloat16).to(dev)
+    wd = (torch.randn(E, Hp, H, generator=gen) / 16).to(torch.bfloat16).to(dev)
+    for zero_copy in (False, True):
+        buf = moe.LayerBuffers.allocate(S, H, Hp, E, K, dev, train=True,
+                                        alloc=GUARD.for_device(dev))
+        moe.moe_layer_forward(x, ids, rw, wg, wu, wd, buf, zero_copy=zero_copy)
+        grads = moe.LayerGrads.allocate(S, H, Hp, E, K, dev, alloc=GUARD.for_device(dev))
+        moe.moe_layer_backward(GUARD((S, H), torch.bfloat16, dev), rw, wg, wu, wd, buf, grads)
+        torch.cuda.synchronize()
+        assert int(buf.d_status.item()) == 0
+        assert buf.counts.cpu().tolist() == [0] * E
+        assert buf.cu_seqlens.cpu().tolist() == [0] * (E + 1)
+        assert int(buf.max_count.item()) == 0 and np.isnan(buf.maxvio.item())
+        assert buf.out.shape == (0, H) and grads.grad_x.shape == (0, H)
+        # no rows: every expert's weight gradient is written as zero
+        for g in (grads.grad_w_gate, grads.grad_w_up, grads.grad_w_down):
+            assert torch.count_nonzero(g).item() == 0
+    mw = moe.MxWeights.from_bf16(wg, wu, wd)
+    buf = moe.LayerBuffers.allocate(S, H, Hp, E, K, dev, alloc=GUARD.for_device(dev))
+    mxb = moe.MxBuffers.allocate(S, H, Hp, K, dev, alloc=GUARD.for_device(dev))
+    moe.moe_layer_forward_mxfp8(x, ids, rw, mw, buf, mxb)
+    torch.cuda.synchronize()
+    assert int(buf.d_status.item()) == 0 and buf.counts.cpu().tolist() == [0] * E
+
+
 def test_layer_is_deterministic(cuda_device):
     w = synth.WORKLOADS["medium"]
     inp = layer_inputs(w, cuda_device)
