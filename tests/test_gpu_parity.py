@@ -352,6 +352,30 @@ def test_layer_ragged_chunks_full(cuda_device, H, Hp):
     _check_full_layer(inp, w, run_layer(inp, w, cuda_device))
 
 
+@pytest.mark.parametrize("E", [1000, 1024])
+def test_layer_many_experts_full(cuda_device, E):
+    """The grouped FFN's largest expert count (its per-expert row and unit tables fill the
+    shared memory they are sized for): 1000 or 1024 experts, most with 0-3 rows, a few
+    larger, one hot expert in the last window of the table; whole layer against the oracle."""
+    H, Hp, K = 128, 256, 4
+    rng = np.random.default_rng(E)
+    S = 700
+    ids_np = np.stack([rng.choice(E, size=K, replace=False) for _ in range(S)]).astype(np.int32)
+    ids_np[:150, 0] = E - 1  # a hot expert, last in the table
+    w = synth.Workload("many_experts", S, H, Hp, E, K, 23)
+    inp = {"topk_ids": torch.from_numpy(ids_np).to(cuda_device),
+           "route_w": torch.from_numpy(rng.random((S, K)).astype(np.float32)).to(cuda_device)}
+    inp["x"] = synth.normal_bf16_into(torch.empty(S, H, dtype=torch.bfloat16, device=cuda_device),
+                                      23, synth.TAG_X)
+    for name, tag, shape in (("w_gate", synth.TAG_W_GATE, (E, H, Hp)),
+                             ("w_up", synth.TAG_W_UP, (E, H, Hp)),
+                             ("w_down", synth.TAG_W_DOWN, (E, Hp, H))):
+        inp[name] = synth.normal_bf16_into(torch.empty(*shape, dtype=torch.bfloat16,
+                                                       device=cuda_device), 23, tag,
+                                           synth.weight_scale(w, name[2:]))
+    _check_full_layer(inp, w, run_layer(inp, w, cuda_device))
+
+
 def test_layer_medium_full(cuda_device):
     w = synth.WORKLOADS["medium"]
     inp = layer_inputs(w, cuda_device)
