@@ -145,6 +145,8 @@ FFN_CASES = {
     "tiny": (4, 256, 256, [0, 17, 100, 250]),
     "ragged": (6, 384, 512, [1, 224, 225, 0, 31, 480]),
     "wide": (3, 1024, 768, [300, 64, 129]),
+    # the largest expert count (full per-expert tables): mostly 0-3 rows, a hot expert last
+    "many": (1024, 128, 256, [i % 4 for i in range(1023)] + [150]),
 }
 
 
