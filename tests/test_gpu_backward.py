@@ -152,6 +152,19 @@ def test_ffn_backward_ragged_full(cuda_device, H, Hp):
     _check_stages(inp, w, buf, grads)
 
 
+def test_ffn_backward_many_experts_full(cuda_device):
+    """1024 experts (the grouped FFN's largest count), most with 0-2 rows and a larger last
+    one: every backward pass decodes units over full per-expert tables, and the weight
+    gradients of the ~340 empty experts are written as zeros."""
+    sizes = [i % 3 for i in range(1023)] + [40]
+    w, inp = _ragged_inputs(cuda_device, 128, 128, sizes, seed=31)
+    buf, grads, _ = _run_train(inp, w, cuda_device)
+    _check_stages(inp, w, buf, grads)
+    empty = [e for e, n in enumerate(sizes) if n == 0]
+    for g in (grads.grad_w_gate, grads.grad_w_up, grads.grad_w_down):
+        assert torch.count_nonzero(g[empty]).item() == 0
+
+
 def test_ffn_backward_medium_full_accumulate(cuda_device):
     """Medium layer; the weight gradients are added into random prior fp32 buffers."""
     w = synth.WORKLOADS["medium"]
