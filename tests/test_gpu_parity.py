@@ -267,6 +267,47 @@ def test_identity_expert_layer(cuda_device, wname):
         print(f"[{wname}] out (sampled): {assert_close_bf16(out_gpu, out_ref, 'out (sampled)')}")
 
 
+@pytest.mark.parametrize("K", [33, 40])
+def test_combine_and_its_backward_beyond_32_slots(cuda_device, K):
+    """K > 32 route slots per token (the combine then reads its slots' rows and weights from
+    memory instead of one lane each): permute, identity experts and combine against the
+    oracle, and the combine / permutation backward on the same plan."""
+    dev = cuda_device
+    S, H, E = 300, 64, 64
+    rng = np.random.default_rng(K)
+    ids_np = rng.integers(0, E, size=(S, K)).astype(np.int32)  # duplicates included
+    x_bits = O.f64_to_bf16_bits(rng.standard_normal((S, H)))
+    rw_np = rng.random((S, K)).astype(np.float32)
+    x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    ids, rw = torch.from_numpy(ids_np).to(dev), torch.from_numpy(rw_np).to(dev)
+    buf = moe.LayerBuffers.allocate(S, H, 0, E, K, dev, with_ffn=False,
+                                    alloc=GUARD.for_device(dev))
+    moe.moe_layer_forward(x, ids, rw, None, None, None, buf)
+    torch.cuda.synchronize()
+    assert int(buf.d_status.item()) == 0
+    counts, cu, rmap, psrc = O.permute_metadata(ids_np, E)
+    assert np.array_equal(buf.row_id_map.cpu().numpy(), rmap)
+    x_perm = O.permute_rows(x_bits, psrc, K)
+    assert np.array_equal(bits(buf.x_perm), x_perm)
+    out_ref = O.unpermute_combine(x_perm, rmap, rw_np, S, K)
+    print(f"K={K} out: {assert_close_bf16(bits(buf.out), out_ref, 'out')}")
+    # backward of the combine (y = x_perm) and of the permutation
+    g_bits = O.f64_to_bf16_bits(rng.standard_normal((S, H)))
+    g = torch.from_numpy(g_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    grad_y = GUARD((S * K, H), torch.bfloat16, dev)
+    grad_w = GUARD((S, K), torch.float32, dev)
+    moe.moe_combine_backward(g, buf.x_perm, buf.row_id_map, rw, grad_y, grad_w)
+    grad_x = GUARD((S, H), torch.bfloat16, dev)
+    moe.moe_permute_backward(grad_y, buf.row_id_map, grad_x, K)
+    torch.cuda.synchronize()
+    gy_ref, gw_ref = O.combine_backward(g_bits, x_perm, rmap, rw_np, S, K)
+    assert np.array_equal(bits(grad_y), gy_ref)
+    gw = grad_w.cpu().numpy().astype(np.float64)
+    assert np.abs(gw - gw_ref).max() <= 1e-4 * np.abs(gw_ref).max()
+    gx_ref = O.permute_backward(gy_ref, rmap, S, K)
+    print(f"K={K} grad_x: {assert_close_bf16(bits(grad_x), gx_ref, 'grad_x')}")
+
+
 def test_combine_unit_weight_invariants(cuda_device):
     S, K, E, H = 2000, 4, 16, 256
     rng = np.random.default_rng(7)
