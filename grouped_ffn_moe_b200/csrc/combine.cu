@@ -61,12 +61,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int64_t npass = (nvec + 32 * U - 1) / (32 * U);
   const int64_t items = S * npass;
-  for (int64_t it = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       it < items; it += nwarps) {
+  // the slot table of an item (lane k: row and weight of slot k), loaded one item ahead so
+  // that its latency overlaps the previous item's row loads
+  auto slot_of = [&](int64_t it, int32_t& row, float& wt) {
+    row = -1;
+    wt = 0.0f;
+    if (it < items && lane < K) {
+      const int64_t t = it / npass;
+      row = row_id_map[t * K + lane];
+      wt = route_w != nullptr ? route_w[t * K + lane] : 1.0f;
+    }
+  };
+  int64_t it = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  int32_t next_row;
+  float next_w;
+  slot_of(it, next_row, next_w);
+  for (; it < items; it += nwarps) {
     const int64_t t = it / npass;
     const int64_t v0 = (it - t * npass) * (32 * U);
-    const int32_t my_row = (lane < K) ? row_id_map[t * K + lane] : -1;
-    const float my_w = (lane < K) ? (route_w != nullptr ? route_w[t * K + lane] : 1.0f) : 0.0f;
+    const int32_t my_row = next_row;
+    const float my_w = next_w;
+    slot_of(it + nwarps, next_row, next_w);
     {
       float acc[U][8];
 #pragma unroll
@@ -181,6 +196,23 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(
   }
 }
 
+ContextCache g_combine_blocks;
+
+// Resident 256-thread blocks of the combine kernel per SM (queried once per context).
+int combine_blocks_per_sm() {
+  void* v = nullptr;
+  if (g_combine_blocks.find(current_context_id(), &v))
+    return static_cast<int>(reinterpret_cast<intptr_t>(v));
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+          &n, combine_kernel<MOE_COMBINE_U, MOE_COMBINE_SLOTS>, 256, 0) != cudaSuccess || n < 1) {
+    (void)cudaGetLastError();
+    n = 1;
+  }
+  g_combine_blocks.put(current_context_id(), reinterpret_cast<void*>(static_cast<intptr_t>(n)));
+  return n;
+}
+
 }  // namespace
 
 moe_status launch_combine_backward(const void* grad_out, const void* y, const int32_t* row_id_map,
@@ -199,7 +231,10 @@ moe_status launch_combine(const void* y, const int32_t* row_id_map, const float*
                           int64_t S, int64_t H, int32_t K, void* out, cudaStream_t stream) {
   const int64_t nvec = H / 8;
   const int64_t items = S * ceil_div(nvec, 32 * MOE_COMBINE_U);
-  const int64_t blocks = std::min<int64_t>(ceil_div(items, 8), static_cast<int64_t>(num_sms()) * 8);
+  // one resident wave of blocks: every warp strides over several items, loading each next
+  // item's slot table while the current item's rows are in flight
+  const int64_t blocks = std::min<int64_t>(
+      ceil_div(items, 8), static_cast<int64_t>(num_sms()) * combine_blocks_per_sm());
   const cudaError_t err = launch_dependent(
       combine_kernel<MOE_COMBINE_U, MOE_COMBINE_SLOTS>, dim3(static_cast<unsigned>(blocks)),
       dim3(256), 0, stream, static_cast<const uint4*>(y), row_id_map, route_w, S, nvec, K,
