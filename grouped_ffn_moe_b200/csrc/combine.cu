@@ -139,58 +139,86 @@ __device__ __forceinline__ float mul_round_odd(float w, float g) {
 }
 
 // Backward of the combine (MoonEP README, "combine bwd": the output gradient goes back to the
-// expert-grouped rows along the saved plan), one warp per token, for each slot k in order:
+// expert-grouped rows along the saved plan), for every token t and slot k:
 //   grad_y[r(t,k)] = bf16(w[t,k] * grad_out[t])   (one rounding of the exact product)
-//   grad_w[t,k]    = <grad_out[t], y[r(t,k)]>  (fp32; per-lane partial sums in vector order,
-//                    then a fixed butterfly reduction: deterministic)
-// The token's gradient row is re-read per slot from L1/L2; HBM traffic stays grad_out once,
-// grad_y and y once each.
-__global__ void __launch_bounds__(256) combine_backward_kernel(
+//   grad_w[t,k]    = <grad_out[t], y[r(t,k)]>      (fp32, fixed summation order)
+// One CTA of 8 warps per token: warp i takes the i-th eighth of the row's 16-byte vectors,
+// and the slots go in groups of kBwdSlots whose rows' loads are in flight together. The dot
+// product is summed per lane in vector order, then over the lanes by a fixed butterfly, then
+// over the 8 warps in warp order through shared memory: deterministic. HBM traffic: grad_out
+// once (re-read per slot group from L1/L2), y and grad_y once each.
+constexpr int kBwdSlots = 4;
+constexpr int kBwdWarps = 8;
+
+__global__ void __launch_bounds__(32 * kBwdWarps) combine_backward_kernel(
     const uint4* __restrict__ grad_out, const uint4* __restrict__ y,
     const int32_t* __restrict__ row_id_map, const float* __restrict__ route_w, int64_t S,
     int64_t nvec, int32_t K, uint4* __restrict__ grad_y, float* __restrict__ grad_w) {
-  const int lane = threadIdx.x & 31;
+  __shared__ float s_dot[kBwdWarps][kBwdSlots];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   griddep_wait();
   griddep_launch_dependents();
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       t < S; t += nwarps) {
+  const int64_t per_warp = (nvec + kBwdWarps - 1) / kBwdWarps;
+  const int64_t vb = min(static_cast<int64_t>(warp) * per_warp, nvec);
+  const int64_t ve = min(vb + per_warp, nvec);
+  for (int64_t t = blockIdx.x; t < S; t += gridDim.x) {
     const uint4* g = grad_out + t * nvec;
-    for (int k = 0; k < K; ++k) {
-      const int32_t r = row_id_map[t * K + k];
-      const float wk = route_w[t * K + k];
-      float dot = 0.0f;
-      if (r >= 0) {
-        uint4* dst = grad_y + static_cast<int64_t>(r) * nvec;
-        const uint4* src = y != nullptr ? y + static_cast<int64_t>(r) * nvec : nullptr;
-        for (int64_t v = lane; v < nvec; v += 32) {
-          const uint4 gv = __ldg(g + v);
-          float gf[8];
-          const uint32_t gu[4] = {gv.x, gv.y, gv.z, gv.w};
+    for (int k0 = 0; k0 < K; k0 += kBwdSlots) {
+      int32_t rows[kBwdSlots];
+      float ws[kBwdSlots], dot[kBwdSlots];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            gf[2 * i] = __uint_as_float(gu[i] << 16);
-            gf[2 * i + 1] = __uint_as_float(gu[i] & 0xFFFF0000u);
-          }
+      for (int s = 0; s < kBwdSlots; ++s) {
+        const int k = k0 + s;
+        rows[s] = k < K ? row_id_map[t * K + k] : -1;
+        ws[s] = k < K ? route_w[t * K + k] : 0.0f;
+        dot[s] = 0.0f;
+      }
+      for (int64_t v = vb + lane; v < ve; v += 32) {
+        const uint4 gv = __ldg(g + v);
+        uint4 yv[kBwdSlots];
+#pragma unroll
+        for (int s = 0; s < kBwdSlots; ++s)
+          yv[s] = (rows[s] >= 0 && y != nullptr)
+                      ? __ldg(y + static_cast<int64_t>(rows[s]) * nvec + v)
+                      : make_uint4(0, 0, 0, 0);
+        float gf[8];
+        const uint32_t gu[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          gf[2 * i] = __uint_as_float(gu[i] << 16);
+          gf[2 * i + 1] = __uint_as_float(gu[i] & 0xFFFF0000u);
+        }
+#pragma unroll
+        for (int s = 0; s < kBwdSlots; ++s) {
+          if (rows[s] < 0) continue;
           float sc[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) sc[i] = mul_round_odd(wk, gf[i]);
-          dst[v] = pack_bf16x8(sc);
-          if (src != nullptr) {
-            const uint4 yv = __ldg(src + v);
-            const uint32_t yu[4] = {yv.x, yv.y, yv.z, yv.w};
+          for (int i = 0; i < 8; ++i) sc[i] = mul_round_odd(ws[s], gf[i]);
+          grad_y[static_cast<int64_t>(rows[s]) * nvec + v] = pack_bf16x8(sc);
+          const uint32_t yu[4] = {yv[s].x, yv[s].y, yv[s].z, yv[s].w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              dot = fmaf(gf[2 * i], __uint_as_float(yu[i] << 16), dot);
-              dot = fmaf(gf[2 * i + 1], __uint_as_float(yu[i] & 0xFFFF0000u), dot);
-            }
+          for (int i = 0; i < 4; ++i) {
+            dot[s] = fmaf(gf[2 * i], __uint_as_float(yu[i] << 16), dot[s]);
+            dot[s] = fmaf(gf[2 * i + 1], __uint_as_float(yu[i] & 0xFFFF0000u), dot[s]);
           }
         }
       }
       if (grad_w != nullptr) {
 #pragma unroll
-        for (int d = 16; d > 0; d >>= 1) dot += __shfl_xor_sync(kFull, dot, d);
-        if (lane == 0) grad_w[t * K + k] = dot;
+        for (int s = 0; s < kBwdSlots; ++s) {
+#pragma unroll
+          for (int d = 16; d > 0; d >>= 1) dot[s] += __shfl_xor_sync(kFull, dot[s], d);
+        }
+        if (lane == 0)
+#pragma unroll
+          for (int s = 0; s < kBwdSlots; ++s) s_dot[warp][s] = dot[s];
+        __syncthreads();
+        if (threadIdx.x < kBwdSlots && k0 + static_cast<int>(threadIdx.x) < K) {
+          float sum = 0.0f;
+          for (int i = 0; i < kBwdWarps; ++i) sum += s_dot[i][threadIdx.x];
+          grad_w[t * K + k0 + threadIdx.x] = sum;
+        }
+        __syncthreads();  // s_dot is rewritten by the next slot group
       }
     }
   }
@@ -219,9 +247,10 @@ moe_status launch_combine_backward(const void* grad_out, const void* y, const in
                                    const float* route_w, int64_t S, int64_t H, int32_t K,
                                    void* grad_y, float* grad_w, cudaStream_t stream) {
   const int64_t nvec = H / 8;
-  const int64_t blocks = std::min<int64_t>(ceil_div(S, 8), static_cast<int64_t>(num_sms()) * 8);
+  const int64_t blocks = std::min<int64_t>(S, static_cast<int64_t>(num_sms()) * 8);
   const cudaError_t err = launch_dependent(
-      combine_backward_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+      combine_backward_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32 * kBwdWarps), 0,
+      stream,
       static_cast<const uint4*>(grad_out), static_cast<const uint4*>(y), row_id_map, route_w, S,
       nvec, K, static_cast<uint4*>(grad_y), grad_w);
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
