@@ -1,5 +1,6 @@
-// Plain C++ CPU oracle of the MoE layer's forward hot path (permutation, maxvio, grouped
-// SwiGLU FFN, weighted combine).
+// Plain C++ CPU oracle of the MoE layer's hot path: the forward (permutation, maxvio, grouped
+// SwiGLU FFN, weighted combine), the backward of the two data-movement steps, and the MXFP8
+// quantisation.
 //
 // TEST INFRASTRUCTURE ONLY: loaded by tests/ (through oracle/ref.py) to cross-check the
 // numpy oracle; the product path never links or loads it, and it shares no code, header or
@@ -186,6 +187,89 @@ void ref_combine(const uint16_t* y, const int32_t* row_id_map, const float* rout
       out[t * H + n] = double_to_bf16(acc);
     }
   }
+}
+
+// ---------------------------------------------------------------------------- backward
+// MoonEP README, "API walkthrough": combine bwd re-dispatches the output gradient along the
+// saved plan, dispatch bwd sums each token's K row gradients. With out[t] = sum_k w[t,k] *
+// y[r(t,k)]:
+//   grad_y[r(t,k)] = bf16(w[t,k] * grad_out[t])      grad_w[t,k] = <grad_out[t], y[r(t,k)]>
+//   grad_x[t]      = bf16(sum over k ascending of grad_x_perm[r(t,k)])
+
+// grad_w in double, summed over n ascending; rows no slot maps to are left as they are.
+void ref_combine_backward(const uint16_t* grad_out, const uint16_t* y,
+                          const int32_t* row_id_map, const float* route_w, int64_t S,
+                          int32_t K, int64_t H, uint16_t* grad_y, double* grad_w) {
+  for (int64_t t = 0; t < S; ++t) {
+    for (int32_t k = 0; k < K; ++k) {
+      const int64_t r = row_id_map[t * K + k];
+      const double w = static_cast<double>(route_w[t * K + k]);
+      double dot = 0.0;
+      for (int64_t n = 0; n < H; ++n) {
+        const double g = bf16_to_double(grad_out[t * H + n]);
+        grad_y[r * H + n] = double_to_bf16(w * g);  // exact product, one rounding
+        dot += g * bf16_to_double(y[r * H + n]);
+      }
+      grad_w[t * K + k] = dot;
+    }
+  }
+}
+
+void ref_permute_backward(const uint16_t* grad_x_perm, const int32_t* row_id_map, int64_t S,
+                          int32_t K, int64_t H, uint16_t* grad_x) {
+  for (int64_t t = 0; t < S; ++t)
+    for (int64_t n = 0; n < H; ++n) {
+      double acc = 0.0;
+      for (int32_t k = 0; k < K; ++k)
+        acc += bf16_to_double(grad_x_perm[static_cast<int64_t>(row_id_map[t * K + k]) * H + n]);
+      grad_x[t * H + n] = double_to_bf16(acc);
+    }
+}
+
+// ---------------------------------------------------------------------------- MXFP8
+// OCP Microscaling (MX) v1.0, MXFP8: blocks of 32 consecutive elements share a power-of-two
+// scale 2^s stored as E8M0, s = floor(log2(block max |v|)) - 8 (8 = the exponent of E4M3's
+// largest power of two), s = -127 for an all-zero block; elements are v / 2^s rounded to
+// E4M3 (nearest, ties to even; normal exponents -6..8 with 3 fraction bits, subnormal step
+// 2^-9), saturating at 448.
+
+// E4M3 rounding of one double, through frexp: a = m * 2^e, m in [0.5, 1), so the leading
+// bit's exponent is e - 1 and the E4M3 quantum there is 2^(e - 1 - 3) (at least 2^-9).
+static double e4m3_of(double v) {
+  const double a = std::fabs(v);
+  if (a == 0.0) return v;
+  int e;
+  std::frexp(a, &e);
+  int quantum = e - 1 - 3;
+  if (quantum < -9) quantum = -9;
+  double q = std::ldexp(std::nearbyint(std::ldexp(a, -quantum)), quantum);
+  if (q > 448.0) q = 448.0;
+  return std::copysign(q, v);
+}
+
+void ref_e4m3_round(const double* v, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_of(v[i]);
+}
+
+// Rows of length L (a multiple of 32) quantised along the row: q[r, j] (E4M3 values as
+// doubles) and sexp[r, j / 32].
+void ref_mx_quantize_rows(const double* v, int64_t rows, int64_t L, double* q, int32_t* sexp) {
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < L / 32; ++b) {
+      const double* blk = v + r * L + b * 32;
+      double amax = 0.0;
+      for (int i = 0; i < 32; ++i) amax = std::fmax(amax, std::fabs(blk[i]));
+      int s = -127;
+      if (amax > 0.0) {
+        int e;
+        std::frexp(amax, &e);
+        s = (e - 1) - 8;
+        if (s < -127) s = -127;
+        if (s > 127) s = 127;
+      }
+      sexp[r * (L / 32) + b] = s;
+      for (int i = 0; i < 32; ++i) q[r * L + b * 32 + i] = e4m3_of(std::ldexp(blk[i], -s));
+    }
 }
 
 }  // extern "C"

@@ -50,6 +50,14 @@ def lib() -> ctypes.CDLL:
         L.ref_grouped_ffn.restype = None
         L.ref_combine.argtypes = [P, P, P, i64, i32, i64, P]
         L.ref_combine.restype = None
+        L.ref_combine_backward.argtypes = [P, P, P, P, i64, i32, i64, P, P]
+        L.ref_combine_backward.restype = None
+        L.ref_permute_backward.argtypes = [P, P, i64, i32, i64, P]
+        L.ref_permute_backward.restype = None
+        L.ref_e4m3_round.argtypes = [P, i64, P]
+        L.ref_e4m3_round.restype = None
+        L.ref_mx_quantize_rows.argtypes = [P, i64, i64, P, P]
+        L.ref_mx_quantize_rows.restype = None
         _lib = L
     return _lib
 
@@ -115,3 +123,40 @@ def combine(y_bits, row_id_map, route_w, S: int, K: int) -> np.ndarray:
     out = np.empty((S, y.shape[1]), np.uint16)
     lib().ref_combine(_p(y), _p(rm), _p(w), S, K, y.shape[1], _p(out))
     return out
+
+
+def combine_backward(grad_out_bits, y_bits, row_id_map, route_w, S: int, K: int):
+    """(grad_y bits [M,H], grad_w float64 [S,K]); rows no slot maps to stay 0."""
+    g = np.ascontiguousarray(grad_out_bits, dtype=np.uint16)
+    y = np.ascontiguousarray(y_bits, dtype=np.uint16)
+    rm = np.ascontiguousarray(row_id_map, dtype=np.int32)
+    w = np.ascontiguousarray(route_w, dtype=np.float32)
+    gy = np.zeros(y.shape, np.uint16)
+    gw = np.zeros((S, K), np.float64)
+    lib().ref_combine_backward(_p(g), _p(y), _p(rm), _p(w), S, K, y.shape[1], _p(gy), _p(gw))
+    return gy, gw
+
+
+def permute_backward(grad_x_perm_bits, row_id_map, S: int, K: int) -> np.ndarray:
+    gxp = np.ascontiguousarray(grad_x_perm_bits, dtype=np.uint16)
+    rm = np.ascontiguousarray(row_id_map, dtype=np.int32)
+    out = np.empty((S, gxp.shape[1]), np.uint16)
+    lib().ref_permute_backward(_p(gxp), _p(rm), S, K, gxp.shape[1], _p(out))
+    return out
+
+
+def e4m3_round(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, np.float64)
+    lib().ref_e4m3_round(_p(v), v.size, _p(out))
+    return out
+
+
+def mx_quantize_rows(v):
+    """MXFP8 along the last axis of a 2-D array: (E4M3 values [rows, L], exponents [rows, L/32])."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    rows, L = v.shape
+    q = np.empty((rows, L), np.float64)
+    s = np.empty((rows, L // 32), np.int32)
+    lib().ref_mx_quantize_rows(_p(v), rows, L, _p(q), _p(s))
+    return q, s

@@ -104,3 +104,41 @@ def test_grouped_ffn_agrees_with_the_numpy_oracle():
     # dropping SiLU or swapping gate and up is visible
     h_swap, _ = R.grouped_ffn(x, cu, wu, wg, wd)
     assert np.count_nonzero(h_swap != h_c) > h_c.size // 2
+
+
+def test_combine_and_permute_backward_match():
+    rng = np.random.default_rng(4)
+    S, K, E, H = 150, 5, 7, 40
+    ids = rng.integers(0, E, size=(S, K)).astype(np.int32)
+    _, _, rmap, _ = O.permute_metadata(ids, E)
+    g = O.f64_to_bf16_bits(rng.standard_normal((S, H)))
+    y = O.f64_to_bf16_bits(rng.standard_normal((S * K, H)))
+    w = rng.random((S, K)).astype(np.float32)
+    gy_c, gw_c = R.combine_backward(g, y, rmap, w, S, K)
+    gy_n, gw_n = O.combine_backward(g, y, rmap, w, S, K)
+    assert np.array_equal(gy_c, gy_n)  # one rounding of an exact product on both sides
+    assert np.allclose(gw_c, gw_n, rtol=1e-12, atol=1e-12)  # double sums, orders differ
+    gxp = O.f64_to_bf16_bits(rng.standard_normal((S * K, H)))
+    assert np.array_equal(R.permute_backward(gxp, rmap, S, K), O.permute_backward(gxp, rmap, S, K))
+
+
+def test_e4m3_and_mx_quantisation_match():
+    rng = np.random.default_rng(5)
+    # E4M3 rounding: torch's float8_e4m3fn cast inside the finite range, and the numpy oracle
+    # (which saturates at 448) everywhere, ties and subnormals included
+    v = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-4, 3, 20000),
+                        np.array([0.0, -0.0, 448.0, 464.0, 480.0, 1e6, -1e6, 2 ** -9, 2 ** -10,
+                                  3 * 2 ** -11, 1.0625, 1.1875, 17.0, 19.0])])
+    got = R.e4m3_round(v)
+    assert np.array_equal(got, O.e4m3_round(v))
+    inside = np.abs(v) <= 448
+    t = torch.from_numpy(v[inside]).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(got[inside], t)
+    # MXFP8 blocks along rows: random magnitudes per block, zero blocks, exact powers of two
+    x = rng.standard_normal((64, 256)) * np.repeat(2.0 ** rng.integers(-20, 20, (64, 8)), 32, axis=1)
+    x[3, 32:64] = 0.0
+    x[5, :32] = 2.0 ** 7
+    q_c, s_c = R.mx_quantize_rows(x)
+    q_n, s_n = O.mx_quantize(x, axis=-1)
+    assert np.array_equal(q_c, q_n) and np.array_equal(s_c, s_n)
+    assert s_c[3, 1] == -127 and s_c[5, 0] == -1
