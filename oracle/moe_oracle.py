@@ -379,7 +379,8 @@ def e4m3_round(v: np.ndarray) -> np.ndarray:
     """Round float64 values to FP8 E4M3 (nearest, ties to even), saturating at +-448."""
     v = np.asarray(v, dtype=np.float64)
     a = np.abs(v)
-    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    _, fe = np.frexp(np.where(a > 0, a, 1.0))
+    e = (fe - 1).astype(np.float64)  # floor(log2 a), exactly
     e = np.maximum(e, -6.0)  # below 2^-6 the spacing is the subnormal step 2^-9
     step = np.ldexp(1.0, (e - 3).astype(np.int64))
     q = np.minimum(np.rint(a / step) * step, E4M3_MAX)
@@ -396,8 +397,10 @@ def mx_quantize(v: np.ndarray, axis: int = -1):
     assert n % MX_BLOCK == 0
     blocks = v.reshape(v.shape[:-1] + (n // MX_BLOCK, MX_BLOCK))
     amax = np.abs(blocks).max(axis=-1)
-    sexp = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - E4M3_EMAX,
-                    -127.0)
+    # floor(log2 amax) exactly: frexp gives amax = m * 2^e with m in [0.5, 1) (a rounded log2
+    # would be one too large just below a power of two)
+    _, e = np.frexp(np.where(amax > 0, amax, 1.0))
+    sexp = np.where(amax > 0, (e - 1).astype(np.float64) - E4M3_EMAX, -127.0)
     sexp = np.clip(sexp, -127, 127).astype(np.int64)
     q = e4m3_round(blocks / np.ldexp(1.0, sexp)[..., None])
     return (np.moveaxis(q.reshape(v.shape), -1, axis),

@@ -732,3 +732,20 @@ def test_mxfp8_expert_exact_hand_case():
     assert no_down_weight_quant != y_want[31]
     row_wise = O.mx_quantize(O.bf16_bits_to_f64(bits["wd"]), axis=-1)  # wrong axis for Down
     assert O.mx_dequantize(*row_wise, axis=-1)[0, 31] == 1.25 * 2 ** -15
+
+
+def test_mx_scale_exponent_just_below_a_power_of_two():
+    """The block scale is 2^(floor(log2 amax) - 8) with the floor taken exactly (OCP MX v1.0,
+    MXFP8): a block maximum one double ulp below 2^8 has floor(log2 amax) = 7, so its scale
+    exponent is -1; the scaled maximum (256 - ulp) * 2 then lies above 448 and saturates to
+    448, and an element 1.0 becomes 2.0. A maximum of exactly 2^8 gives exponent 0."""
+    x = np.zeros((1, 32))
+    x[0, 0] = np.nextafter(256.0, 0.0)
+    x[0, 1] = 1.0
+    q, s = O.mx_quantize(x, axis=-1)
+    assert s[0, 0] == -1
+    assert q[0, 0] == 448.0 and q[0, 1] == 2.0
+    # exactly 2^8 gives exponent 0 and the element 256
+    x[0, 0] = 256.0
+    q, s = O.mx_quantize(x, axis=-1)
+    assert s[0, 0] == 0 and q[0, 0] == 256.0
