@@ -272,4 +272,104 @@ void ref_mx_quantize_rows(const double* v, int64_t rows, int64_t L, double* q, i
     }
 }
 
+// ---------------------------------------------------------------------------- expert backward
+// Chain rule of one expert's forward ("Mixture of Kittens" digest, Step 1, The Math) at the
+// saved bf16 pre-activations g = bf16(x Wg), u = bf16(x Wu), with s = 1 / (1 + e^-g):
+//   grad_h = grad_y Wd^T (not stored)
+//   d_u = bf16(grad_h * g * s)      d_g = bf16(grad_h * u * s * (1 + g (1 - s)))
+//   grad_x = bf16(d_g Wg^T + d_u Wu^T)                     (one rounding)
+//   dWg = x^T d_g, dWu = x^T d_u, dWd = h^T grad_y          (double sums over the n rows)
+// x [n,H], g, u, h [n,Hp], grad_y [n,H]; Wg, Wu [H,Hp], Wd [Hp,H]; bf16 bits.
+void ref_expert_backward(const uint16_t* x, const uint16_t* g, const uint16_t* u,
+                         const uint16_t* h, const uint16_t* grad_y, const uint16_t* wg,
+                         const uint16_t* wu, const uint16_t* wd, int64_t n, int64_t H,
+                         int64_t Hp, uint16_t* d_g, uint16_t* d_u, uint16_t* grad_x,
+                         double* dwg, double* dwu, double* dwd) {
+  for (int64_t r = 0; r < n; ++r) {
+    for (int64_t j = 0; j < Hp; ++j) {
+      double gh = 0.0;
+      for (int64_t m = 0; m < H; ++m)
+        gh += bf16_to_double(grad_y[r * H + m]) * bf16_to_double(wd[j * H + m]);
+      const double gv = bf16_to_double(g[r * Hp + j]);
+      const double uv = bf16_to_double(u[r * Hp + j]);
+      const double sg = 1.0 / (1.0 + std::exp(-gv));
+      d_u[r * Hp + j] = double_to_bf16(gh * (gv * sg));
+      d_g[r * Hp + j] = double_to_bf16(gh * uv * (sg * (1.0 + gv * (1.0 - sg))));
+    }
+    for (int64_t i = 0; i < H; ++i) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < Hp; ++j)
+        acc += bf16_to_double(d_g[r * Hp + j]) * bf16_to_double(wg[i * Hp + j]);
+      for (int64_t j = 0; j < Hp; ++j)
+        acc += bf16_to_double(d_u[r * Hp + j]) * bf16_to_double(wu[i * Hp + j]);
+      grad_x[r * H + i] = double_to_bf16(acc);
+    }
+  }
+  for (int64_t i = 0; i < H; ++i)
+    for (int64_t j = 0; j < Hp; ++j) {
+      double a = 0.0, b = 0.0;
+      for (int64_t r = 0; r < n; ++r) {
+        a += bf16_to_double(x[r * H + i]) * bf16_to_double(d_g[r * Hp + j]);
+        b += bf16_to_double(x[r * H + i]) * bf16_to_double(d_u[r * Hp + j]);
+      }
+      dwg[i * Hp + j] = a;
+      dwu[i * Hp + j] = b;
+    }
+  for (int64_t j = 0; j < Hp; ++j)
+    for (int64_t m = 0; m < H; ++m) {
+      double c = 0.0;
+      for (int64_t r = 0; r < n; ++r)
+        c += bf16_to_double(h[r * Hp + j]) * bf16_to_double(grad_y[r * H + m]);
+      dwd[j * H + m] = c;
+    }
+}
+
+// ---------------------------------------------------------------------------- MXFP8 expert
+// One expert in MXFP8 ("Mixture of Kittens" digest, Step 8, MXFP8 mode; OCP MX v1.0): x
+// quantised along H, the weights along their reduction dimension (Wg, Wu [H,Hp] along H; Wd
+// [Hp,H] along Hp), h = silu(g) u from the dequantised operands quantised along Hp, and
+// y = bf16(deq(h) deq(Wd)); products exact, sums in double. Outputs the h codes as E4M3
+// values (doubles), their exponents, and y bits.
+void ref_expert_ffn_mxfp8(const uint16_t* x, const uint16_t* wg, const uint16_t* wu,
+                          const uint16_t* wd, int64_t n, int64_t H, int64_t Hp, double* hq,
+                          int32_t* hs, uint16_t* y) {
+  // weights: quantise column by column along the reduction (row) index
+  auto quant_cols = [&](const uint16_t* w, int64_t R, int64_t C, std::vector<double>& deq) {
+    deq.assign(static_cast<size_t>(R * C), 0.0);
+    std::vector<double> col(R), q(R);
+    std::vector<int32_t> sx(R / 32);
+    for (int64_t c = 0; c < C; ++c) {
+      for (int64_t r = 0; r < R; ++r) col[r] = bf16_to_double(w[r * C + c]);
+      ref_mx_quantize_rows(col.data(), 1, R, q.data(), sx.data());
+      for (int64_t r = 0; r < R; ++r) deq[r * C + c] = std::ldexp(q[r], sx[r / 32]);
+    }
+  };
+  std::vector<double> g_deq, u_deq, d_deq;
+  quant_cols(wg, H, Hp, g_deq);
+  quant_cols(wu, H, Hp, u_deq);
+  quant_cols(wd, Hp, H, d_deq);
+  std::vector<double> xr(H), xq(H), hv(Hp);
+  std::vector<int32_t> xs(H / 32);
+  for (int64_t r = 0; r < n; ++r) {
+    for (int64_t i = 0; i < H; ++i) xr[i] = bf16_to_double(x[r * H + i]);
+    ref_mx_quantize_rows(xr.data(), 1, H, xq.data(), xs.data());
+    for (int64_t i = 0; i < H; ++i) xr[i] = std::ldexp(xq[i], xs[i / 32]);
+    for (int64_t j = 0; j < Hp; ++j) {
+      double gg = 0.0, uu = 0.0;
+      for (int64_t i = 0; i < H; ++i) {
+        gg += xr[i] * g_deq[i * Hp + j];
+        uu += xr[i] * u_deq[i * Hp + j];
+      }
+      hv[j] = silu(gg) * uu;
+    }
+    ref_mx_quantize_rows(hv.data(), 1, Hp, hq + r * Hp, hs + r * (Hp / 32));
+    for (int64_t m = 0; m < H; ++m) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < Hp; ++j)
+        acc += std::ldexp(hq[r * Hp + j], hs[r * (Hp / 32) + j / 32]) * d_deq[j * H + m];
+      y[r * H + m] = double_to_bf16(acc);
+    }
+  }
+}
+
 }  // extern "C"

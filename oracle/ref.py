@@ -58,6 +58,10 @@ def lib() -> ctypes.CDLL:
         L.ref_e4m3_round.restype = None
         L.ref_mx_quantize_rows.argtypes = [P, i64, i64, P, P]
         L.ref_mx_quantize_rows.restype = None
+        L.ref_expert_backward.argtypes = [P] * 8 + [i64, i64, i64] + [P] * 6
+        L.ref_expert_backward.restype = None
+        L.ref_expert_ffn_mxfp8.argtypes = [P, P, P, P, i64, i64, i64, P, P, P]
+        L.ref_expert_ffn_mxfp8.restype = None
         _lib = L
     return _lib
 
@@ -160,3 +164,32 @@ def mx_quantize_rows(v):
     s = np.empty((rows, L // 32), np.int32)
     lib().ref_mx_quantize_rows(_p(v), rows, L, _p(q), _p(s))
     return q, s
+
+
+def expert_backward(x, g, u, h, grad_y, wg, wu, wd):
+    """One expert's backward on its n rows (all bf16 bits): (d_g, d_u, grad_x bits, dWg, dWu,
+    dWd as float64)."""
+    arrs = [np.ascontiguousarray(a, dtype=np.uint16) for a in (x, g, u, h, grad_y, wg, wu, wd)]
+    n, H = arrs[0].shape
+    Hp = arrs[1].shape[1]
+    d_g = np.empty((n, Hp), np.uint16)
+    d_u = np.empty((n, Hp), np.uint16)
+    gx = np.empty((n, H), np.uint16)
+    dwg = np.empty((H, Hp))
+    dwu = np.empty((H, Hp))
+    dwd = np.empty((Hp, H))
+    lib().ref_expert_backward(*[_p(a) for a in arrs], n, H, Hp, _p(d_g), _p(d_u), _p(gx),
+                              _p(dwg), _p(dwu), _p(dwd))
+    return d_g, d_u, gx, dwg, dwu, dwd
+
+
+def expert_ffn_mxfp8(x, wg, wu, wd):
+    """One MXFP8 expert on its n rows (bf16 bits in): (h E4M3 values, h exponents, y bits)."""
+    arrs = [np.ascontiguousarray(a, dtype=np.uint16) for a in (x, wg, wu, wd)]
+    n, H = arrs[0].shape
+    Hp = arrs[1].shape[1]
+    hq = np.empty((n, Hp))
+    hs = np.empty((n, Hp // 32), np.int32)
+    y = np.empty((n, H), np.uint16)
+    lib().ref_expert_ffn_mxfp8(*[_p(a) for a in arrs], n, H, Hp, _p(hq), _p(hs), _p(y))
+    return hq, hs, y

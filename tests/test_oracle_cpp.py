@@ -142,3 +142,44 @@ def test_e4m3_and_mx_quantisation_match():
     q_n, s_n = O.mx_quantize(x, axis=-1)
     assert np.array_equal(q_c, q_n) and np.array_equal(s_c, s_n)
     assert s_c[3, 1] == -127 and s_c[5, 0] == -1
+
+
+def _close_bits(a, b, max_diff=2):
+    """Equal, except at most max_diff elements one bf16 step apart (a double sum taken in a
+    different order can move a value next to a rounding boundary)."""
+    d = np.abs(a.astype(np.int32) - b.astype(np.int32))
+    assert np.count_nonzero(d) <= max_diff and d.max() <= 1
+
+
+def test_expert_backward_matches():
+    rng = np.random.default_rng(6)
+    n, H, Hp = 20, 64, 96
+    bf = O.f64_to_bf16_bits
+    x = bf(rng.standard_normal((n, H)))
+    wg, wu = bf(rng.standard_normal((H, Hp)) / 8), bf(rng.standard_normal((H, Hp)) / 8)
+    wd = bf(rng.standard_normal((Hp, H)) / 10)
+    g, u = O.expert_preact_rows(x, wg, wu)
+    h = bf(O.silu(O.bf16_bits_to_f64(g)) * O.bf16_bits_to_f64(u))
+    gy = bf(rng.standard_normal((n, H)))
+    got = R.expert_backward(x, g, u, h, gy, wg, wu, wd)
+    ref = O.expert_ffn_backward_rows(x, g, u, h, gy, wg, wu, wd)
+    for a, b in zip(got[:3], ref[:3]):  # d_g, d_u, grad_x
+        _close_bits(a, b)
+    if np.array_equal(got[0], ref[0]) and np.array_equal(got[1], ref[1]):
+        for a, b in zip(got[3:], ref[3:]):  # the weight gradients, double sums
+            assert np.allclose(a, b, rtol=1e-12, atol=1e-12 * np.abs(b).max())
+
+
+def test_mxfp8_expert_matches():
+    rng = np.random.default_rng(7)
+    n, H, Hp = 12, 128, 64
+    bf = O.f64_to_bf16_bits
+    x = bf(rng.standard_normal((n, H)))
+    wg, wu = bf(rng.standard_normal((H, Hp)) / 8), bf(rng.standard_normal((H, Hp)) / 8)
+    wd = bf(rng.standard_normal((Hp, H)) / 8)
+    hq_c, hs_c, y_c = R.expert_ffn_mxfp8(x, wg, wu, wd)
+    hq_n, hs_n, y_n = O.expert_ffn_rows_mxfp8(x, O.mx_weights(wg), O.mx_weights(wu),
+                                              O.mx_weights(wd))
+    assert np.array_equal(hs_c, hs_n)
+    assert np.count_nonzero(hq_c != hq_n) <= 2
+    _close_bits(y_c, y_n, max_diff=max(2, y_c.size // 1000))
